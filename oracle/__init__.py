@@ -1,0 +1,304 @@
+"""CPU oracle for structured-sparse quantized matmul -- TEST INFRASTRUCTURE.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never imports, links or calls it.
+
+This module is argument marshalling around ``ssref.c`` (plain C, see the
+citations there): numpy arrays in, numpy arrays out.  Inputs given as bf16 are
+upcast to fp32 exactly before they reach the C code.
+
+Pins (tests that tie each function to something other than itself) live in
+``tests/test_oracle_*.py``; every function below has at least one.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+INT8 = 0
+FP8_E4M3 = 1
+OUT_F32 = 0
+OUT_BF16 = 1
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        _lib = ctypes.CDLL(path)
+        i64, i32, p = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
+        sig = {
+            "ssref_slide_shape": [i32, i32, i64, p, p, p],
+            "ssref_prune_mask": [p, i64, i64, i32, i32, p],
+            "ssref_prune_pairwise_4of8": [p, i64, i64, p],
+            "ssref_assign_windows": [p, i64, i64, i32, p],
+            "ssref_compress_weight": [p, i64, i64, i32, i32, i32, p, p, p],
+            "ssref_quant_lift_act": [p, i64, i64, i32, i32, i32, p, p],
+            "ssref_prune_act_2to4": [p, i64, i64, i32, p, p, p],
+            "ssref_decompress_2to4": [p, p, i64, i64, p],
+            "ssref_matmul_q": [i32, p, p, p, p, i64, i64, i64, p, i64, i32, p],
+            "ssref_matmul_acc": [i32, p, p, i64, i64, i64, p, p],
+            "ssref_sparse_gemm": [i32, p, p, p, p, p, i64, i64, i64, i32, p, i64, i32, p],
+            "ssref_quantize_value": [ctypes.c_float, ctypes.c_float, i32, p],
+            "ssref_scale_from_absmax": [ctypes.c_float, i32, p, p],
+        }
+        for name, args in sig.items():
+            fn = getattr(_lib, name)
+            fn.argtypes = args
+            fn.restype = i32
+        _lib.ssref_e4m3_from_float.argtypes = [ctypes.c_float]
+        _lib.ssref_e4m3_from_float.restype = ctypes.c_uint8
+        _lib.ssref_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        _lib.ssref_e4m3_to_double.restype = ctypes.c_double
+        _lib.ssref_bf16_from_float.argtypes = [ctypes.c_float]
+        _lib.ssref_bf16_from_float.restype = ctypes.c_uint16
+        _lib.ssref_bits_per_element.argtypes = [i32, i32]
+        _lib.ssref_bits_per_element.restype = ctypes.c_double
+    return _lib
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def _ptr(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(st: int, what: str):
+    if st != 0:
+        raise OracleError(f"{what}: oracle status {st}")
+
+
+def _f32(x) -> np.ndarray:
+    """fp32 contiguous view; torch bf16/fp32 tensors are upcast exactly."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().to("cpu").float().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+
+
+def pattern(p: str) -> tuple[int, int]:
+    """'6:8' -> (6, 8); 'dense' -> (0, 0)."""
+    if p == "dense":
+        return 0, 0
+    keep, group = (int(v) for v in p.split(":"))
+    return keep, group
+
+
+def slide_shape(p: str, K: int) -> tuple[int, int, int]:
+    keep, group = pattern(p)
+    a, b, c = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().ssref_slide_shape(keep, group, K, ctypes.byref(a), ctypes.byref(b),
+                                   ctypes.byref(c)), "slide_shape")
+    return a.value, b.value, c.value
+
+
+def bits_per_element(value_bits: int, sparse_2to4: bool) -> float:
+    return lib().ssref_bits_per_element(value_bits, int(sparse_2to4))
+
+
+def e4m3_from_float(v: float) -> int:
+    return int(lib().ssref_e4m3_from_float(float(v)))
+
+
+def e4m3_to_float(b: int) -> float:
+    return float(lib().ssref_e4m3_to_double(int(b)))
+
+
+def e4m3_decode_array(a: np.ndarray) -> np.ndarray:
+    table = np.array([e4m3_to_float(b) for b in range(256)], dtype=np.float64)
+    return table[np.asarray(a, dtype=np.uint8)]
+
+
+def bf16_from_float(v: float) -> int:
+    return int(lib().ssref_bf16_from_float(float(v)))
+
+
+def scale_from_absmax(a: float, qdtype: int) -> tuple[float, float]:
+    inv, s = ctypes.c_float(), ctypes.c_float()
+    _check(lib().ssref_scale_from_absmax(float(a), qdtype, ctypes.byref(inv), ctypes.byref(s)),
+           "scale")
+    return inv.value, s.value
+
+
+def quantize_value(x: float, inv: float, qdtype: int) -> int:
+    out = ctypes.c_uint8()
+    _check(lib().ssref_quantize_value(float(x), float(inv), qdtype, ctypes.byref(out)), "quant")
+    return out.value
+
+
+def prune_mask(W, keep: int, group: int) -> np.ndarray:
+    W = _f32(W)
+    rows, K = W.shape
+    K_pad = -(-K // group) * group
+    mask = np.zeros((rows, K_pad), dtype=np.uint8)
+    _check(lib().ssref_prune_mask(_ptr(W), rows, K, keep, group, _ptr(mask)), "prune_mask")
+    return mask
+
+
+def prune_pairwise_4of8(W) -> np.ndarray:
+    W = _f32(W)
+    rows, K = W.shape
+    mask = np.zeros((rows, K), dtype=np.uint8)
+    _check(lib().ssref_prune_pairwise_4of8(_ptr(W), rows, K, _ptr(mask)), "pairwise")
+    return mask
+
+
+def assign_windows(mask: np.ndarray, group: int) -> np.ndarray:
+    mask = np.ascontiguousarray(mask, dtype=np.uint8)
+    rows, K_pad = mask.shape
+    win = np.zeros((rows, K_pad), dtype=np.int8)
+    _check(lib().ssref_assign_windows(_ptr(mask), rows, K_pad, group, _ptr(win)),
+           "assign_windows")
+    return win
+
+
+def compress_weight(W, p: str, qdtype: int):
+    """-> (Wv, Wm, s_w); Wm is None for 'dense'."""
+    W = _f32(W)
+    N, K = W.shape
+    keep, group = pattern(p)
+    _, _, K_lp = slide_shape(p, K)
+    if group == 0:
+        Wv = np.zeros((N, K_lp), dtype=np.uint8)
+        Wm = None
+    else:
+        Wv = np.zeros((N, K_lp // 2), dtype=np.uint8)
+        Wm = np.zeros((N, K_lp // 8), dtype=np.uint8)
+    s_w = np.zeros(N, dtype=np.float32)
+    _check(lib().ssref_compress_weight(_ptr(W), N, K, keep, group, qdtype, _ptr(Wv), _ptr(Wm),
+                                       _ptr(s_w)), "compress_weight")
+    return Wv, Wm, s_w
+
+
+def quant_lift_act(X, p: str, qdtype: int):
+    """-> (Xq_lift [M, K_lp], s_x [M])."""
+    X = _f32(X)
+    M, K = X.shape
+    keep, group = pattern(p)
+    _, _, K_lp = slide_shape(p, K)
+    Xq = np.zeros((M, K_lp), dtype=np.uint8)
+    s_x = np.zeros(M, dtype=np.float32)
+    _check(lib().ssref_quant_lift_act(_ptr(X), M, K, keep, group, qdtype, _ptr(Xq), _ptr(s_x)),
+           "quant_lift_act")
+    return Xq, s_x
+
+
+def act_2to4_k_lp(K: int) -> int:
+    return -(-(-(-K // 4) * 4) // 128) * 128
+
+
+def prune_act_2to4(X, qdtype: int):
+    """-> (Xv [M, K_lp/2], Xm [M, K_lp/8], s_x [M])."""
+    X = _f32(X)
+    M, K = X.shape
+    K_lp = act_2to4_k_lp(K)
+    Xv = np.zeros((M, K_lp // 2), dtype=np.uint8)
+    Xm = np.zeros((M, K_lp // 8), dtype=np.uint8)
+    s_x = np.zeros(M, dtype=np.float32)
+    _check(lib().ssref_prune_act_2to4(_ptr(X), M, K, qdtype, _ptr(Xv), _ptr(Xm), _ptr(s_x)),
+           "prune_act_2to4")
+    return Xv, Xm, s_x
+
+
+def decompress_2to4(Av: np.ndarray, Am: np.ndarray, K_lp: int) -> np.ndarray:
+    Av = np.ascontiguousarray(Av, dtype=np.uint8)
+    Am = np.ascontiguousarray(Am, dtype=np.uint8)
+    rows = Av.shape[0]
+    A = np.zeros((rows, K_lp), dtype=np.uint8)
+    _check(lib().ssref_decompress_2to4(_ptr(Av), _ptr(Am), rows, K_lp, _ptr(A)), "decompress")
+    return A
+
+
+def _rows(m_idx, M):
+    if m_idx is None:
+        return None, M
+    m_idx = np.ascontiguousarray(m_idx, dtype=np.int64)
+    return m_idx, len(m_idx)
+
+
+def _out(R, N, out_dtype):
+    return np.zeros((R, N), dtype=np.float32 if out_dtype == OUT_F32 else np.uint16)
+
+
+def matmul_q(qdtype: int, Xq, s_x, Wq, s_w, out_dtype: int, m_idx=None):
+    """Y = dequant(Xq . Wq^T); bf16 output comes back as raw uint16 bits."""
+    Xq = np.ascontiguousarray(Xq, dtype=np.uint8)
+    Wq = np.ascontiguousarray(Wq, dtype=np.uint8)
+    s_x = np.ascontiguousarray(s_x, dtype=np.float32)
+    s_w = np.ascontiguousarray(s_w, dtype=np.float32)
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    m_idx, R = _rows(m_idx, M)
+    Y = _out(R, N, out_dtype)
+    _check(lib().ssref_matmul_q(qdtype, _ptr(Xq), _ptr(s_x), _ptr(Wq), _ptr(s_w), M, N, K,
+                                _ptr(m_idx), R, out_dtype, _ptr(Y)), "matmul_q")
+    return Y
+
+
+def matmul_acc(qdtype: int, Xq, Wq):
+    """Raw accumulators: int64 for INT8, float64 for E4M3."""
+    Xq = np.ascontiguousarray(Xq, dtype=np.uint8)
+    Wq = np.ascontiguousarray(Wq, dtype=np.uint8)
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if qdtype == INT8:
+        acc = np.zeros((M, N), dtype=np.int64)
+        _check(lib().ssref_matmul_acc(qdtype, _ptr(Xq), _ptr(Wq), M, N, K, _ptr(acc), None),
+               "matmul_acc")
+    else:
+        acc = np.zeros((M, N), dtype=np.float64)
+        _check(lib().ssref_matmul_acc(qdtype, _ptr(Xq), _ptr(Wq), M, N, K, None, _ptr(acc)),
+               "matmul_acc")
+    return acc
+
+
+def sparse_gemm(sparse_operand: int, Av, Am, s_a, B, s_b, M: int, N: int, K_lp: int,
+                qdtype: int, out_dtype: int, m_idx=None):
+    Av = np.ascontiguousarray(Av, dtype=np.uint8)
+    Am = np.ascontiguousarray(Am, dtype=np.uint8)
+    B = np.ascontiguousarray(B, dtype=np.uint8)
+    s_a = np.ascontiguousarray(s_a, dtype=np.float32)
+    s_b = np.ascontiguousarray(s_b, dtype=np.float32)
+    m_idx, R = _rows(m_idx, M)
+    Y = _out(R, N, out_dtype)
+    _check(lib().ssref_sparse_gemm(sparse_operand, _ptr(Av), _ptr(Am), _ptr(s_a), _ptr(B),
+                                   _ptr(s_b), M, N, K_lp, qdtype, _ptr(m_idx), R, out_dtype,
+                                   _ptr(Y)), "sparse_gemm")
+    return Y
+
+
+def dense_gemm(Xq, s_x, Wq, s_w, qdtype: int, out_dtype: int, m_idx=None):
+    return matmul_q(qdtype, Xq, s_x, Wq, s_w, out_dtype, m_idx)
+
+
+def plain_linear(W, X, p: str, qdtype: int, out_dtype: int, m_idx=None):
+    """Path (i): prune W, quantise both operands, naive matmul over the
+    original (zero-padded) K -- no decomposition, no lifting."""
+    W = _f32(W)
+    X = _f32(X)
+    N, K = W.shape
+    keep, group = pattern(p)
+    if group:
+        mask = prune_mask(W, keep, group)[:, :K]
+        Wp = np.where(mask.astype(bool), W, np.float32(0))
+    else:
+        Wp = W
+    Wq, _, s_w = compress_weight(Wp, "dense", qdtype)
+    Xq, s_x = quant_lift_act(X, "dense", qdtype)
+    return matmul_q(qdtype, Xq, s_x, Wq, s_w, out_dtype, m_idx)
+
+
+def bf16_bits_to_float(y: np.ndarray) -> np.ndarray:
+    return (np.asarray(y, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
