@@ -1,0 +1,154 @@
+/*
+ * ss.h -- C ABI of libss: quantized matmul on the Blackwell (sm_100a) sparse
+ * tensor cores for structured-sparse weights.
+ *
+ * The method (SlideSparse, "SlideSparse: 布局稀疏边界", 66bd.net, and the
+ * "SlideSparse" write-up, omica.com.cn): a weight pattern (2Nh-2):2Nh --
+ * 2:4, 4:6, 6:8, 8:10 -- keeps 2Nh-2 of every 2Nh consecutive weights along
+ * K.  Nh-1 overlapping windows of width 4 and stride 2 cover each group; every
+ * window holds at most two non-zeros, so the weight becomes hardware 2:4 over
+ * a K grown by 2(Nh-1)/Nh (1.5x for 6:8).  The activation is "lifted" to match
+ * by an index map fused into its per-token quantisation.
+ *
+ * Conventions for every call:
+ *  - All data pointers are DEVICE pointers owned by the caller; the library
+ *    allocates no device memory.  Pointers must be 16-byte aligned.
+ *  - Matrices are row-major.  W is [N, K] (output channels x reduction),
+ *    X is [M, K] (tokens x reduction), Y is [M, N].
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  Argument, alignment and architecture errors are
+ *    returned before anything is launched.  Errors found on the device (a
+ *    NaN/Inf weight, a bounded wait that ran out) are recorded in a device
+ *    status word read by ss_get_device_status().
+ *  - Only sm_100 devices are supported; others return SS_ERR_ARCH.  There is
+ *    no CPU fallback.
+ *  - Buffer sizes follow from ss_slide_shape() / ss_act_2to4_shape().
+ */
+#ifndef SS_H_
+#define SS_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *ss_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    SS_OK = 0,
+    SS_ERR_INVALID_ARG = 1, /* bad size, pattern, dtype or NULL pointer   */
+    SS_ERR_UNSUPPORTED = 2, /* valid but beyond what the kernels handle   */
+    SS_ERR_ALIGNMENT = 3,   /* pointer not 16-byte aligned                 */
+    SS_ERR_ARCH = 4,        /* current device is not sm_100                */
+    SS_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed           */
+    SS_ERR_TIMEOUT = 6,     /* a device-side bounded wait ran out          */
+    SS_ERR_DATA = 7         /* NaN or Inf in a weight being compressed     */
+} ss_status;
+
+typedef enum { SS_IN_F32 = 0, SS_IN_BF16 = 1 } ss_in_dtype;
+typedef enum { SS_INT8 = 0, SS_FP8_E4M3 = 1 } ss_qdtype;
+typedef enum { SS_OUT_F32 = 0, SS_OUT_BF16 = 1 } ss_out_dtype;
+
+/* Sparsity pattern keep:group; {2,4},{4,6},{6,8},{8,10}; {0,0} = dense. */
+typedef struct {
+    int32_t keep;
+    int32_t group;
+} ss_pattern;
+
+/* Parse "2:4", "4:6", "6:8", "8:10" or "dense" (the pattern strings of the
+ * SlideSparse write-up, omica.com.cn, 4.1 and 6.1). */
+ss_status ss_parse_pattern(const char *s, ss_pattern *out);
+
+/* Shapes for a reduction length K under pattern p (SlideSparse, 66bd.net,
+ * Fig. 2: 8 elements become 12 for 6:8):
+ *   K_pad  = 2Nh * ceil(K / 2Nh)          (zero padding of K)
+ *   K_lift = 4 (Nh-1) * ceil(K / 2Nh)     (lifted reduction length)
+ *   K_lp   = K_lift rounded up to 128     (what the GEMM consumes)
+ * Dense: K_pad = K_lift = K, K_lp = K rounded up to 128. */
+ss_status ss_slide_shape(ss_pattern p, int64_t K, int64_t *K_pad, int64_t *K_lift,
+                         int64_t *K_lp);
+
+/* K_lp of an online-pruned 2:4 activation: K rounded up to 4, then to 128. */
+ss_status ss_act_2to4_shape(int64_t K, int64_t *K_lp);
+
+/* Offline weight compression (SlideSparse write-up, omica.com.cn, 2.2 weight
+ * preprocessing and 3.1; LLM-Compressor W8A8 rows: channel-wise weights).
+ * Per row of W[N, K] (f32 or bf16):
+ *   1. magnitude prune each group of 2Nh along K to its 2Nh-2 largest |w|
+ *      (ties keep the lower index; K zero-padded to K_pad);
+ *   2. s_w[n] = absmax of the kept weights / Q (Q = 127 INT8, 448 E4M3);
+ *      q = RNE(w * (Q / absmax)), INT8 clamped to [-127, 127], E4M3 saturated;
+ *   3. assign every kept position to one of the Nh-1 windows by ascending
+ *      first fit (window j covers 2j..2j+3 of its group);
+ *   4. pack each window as two values (ascending local index, padded with the
+ *      lowest unused indices, padded slots hold 0) and a nibble
+ *      idx0 | idx1 << 2.
+ * Outputs (pattern != dense):
+ *   Wv  [N, K_lp/2] bytes   stored values, window w at bytes 2w, 2w+1
+ *   Wm  [N, K_lp/8] bytes   nibbles, window w in byte w/2, low nibble = even w
+ *   s_w [N] fp32
+ * Dense: Wv is [N, K_lp] (per-channel quantised W, zero padded), Wm unused
+ * (may be NULL).  A NaN/Inf weight sets SS_ERR_DATA in the device status. */
+ss_status ss_compress_weight(const void *W, ss_in_dtype in_dtype, int64_t N, int64_t K,
+                             ss_pattern p, ss_qdtype q, void *Wv, void *Wm, float *s_w,
+                             ss_stream_t stream);
+
+/* Fused per-token quantisation + activation lifting (SlideSparse, 66bd.net:
+ * lifting is an index map fused into the per-token quant kernel; write-up
+ * 3.2: window i reads 4 consecutive activations at
+ * base = 2Nh * (i / (Nh-1)) + 2 * (i % (Nh-1)), four bytes packed per word).
+ * Per token m of X[M, K]: a = max_k |x|, s_x[m] = a / Q, q = RNE(x * (Q / a));
+ * Xq_lift[m, 4i + t] = q(X[m, base_i + t]) (0 past K and past K_lift).
+ * Outputs: Xq_lift [M, K_lp] bytes, s_x [M] fp32.  Dense: identity map. */
+ss_status ss_quant_lift_act(const void *X, ss_in_dtype in_dtype, int64_t M, int64_t K,
+                            ss_pattern p, ss_qdtype q, void *Xq_lift, float *s_x,
+                            ss_stream_t stream);
+
+/* Online 2:4 prune + compress of an activation (the "add 2:4 or drop a
+ * precision tier?" study, paper-daily 2610.28947, section 1: operands made on
+ * the fly must be pruned and compressed before every matmul).  Per token m:
+ * in each group of 4 along K keep the two largest |x| (ties keep the lower
+ * index), s_x[m] = row absmax / Q, quantise the kept values, pack as in
+ * ss_compress_weight.  Outputs Xv [M, K_lp/2], Xm [M, K_lp/8], s_x [M] with
+ * K_lp from ss_act_2to4_shape(). */
+ss_status ss_prune_act_2to4(const void *X, ss_in_dtype in_dtype, int64_t M, int64_t K,
+                            ss_qdtype q, void *Xv, void *Xm, float *s_x, ss_stream_t stream);
+
+/* Sparse GEMM on the sm_100a sparse tensor cores (tcgen05.mma.sp, TMEM
+ * accumulators, TMA-staged tiles), with the dequant epilogue
+ *   Y[m, n] = ((float)acc[m, n] * s_x[m]) * s_w[n]   (fp32, then bf16 RNE)
+ * sparse_operand = 0: A = weight.  Av = Wv [N, K_lp/2], Am = Wm [N, K_lp/8],
+ *                     s_a = s_w [N]; B = Xq_lift [M, K_lp], s_b = s_x [M].
+ * sparse_operand = 1: A = activation.  Av = Xv [M, K_lp/2], Am = Xm
+ *                     [M, K_lp/8], s_a = s_x [M]; B = Wq [N, K_lp] (dense),
+ *                     s_b = s_w [N].
+ * acc is exact int32 for INT8 and fp32 (tensor-core accumulation) for E4M3.
+ * K_lp must be a positive multiple of 128; M, N in [1, 2^31). */
+ss_status ss_sparse_gemm(int sparse_operand, const void *Av, const void *Am, const float *s_a,
+                         const void *B, const float *s_b, int64_t M, int64_t N, int64_t K_lp,
+                         ss_qdtype q, void *Y, ss_out_dtype out_dtype, ss_stream_t stream);
+
+/* Dense GEMM of the same construction (tcgen05.mma), the like-for-like
+ * comparison: Y = dequant(Xq [M, K_p] . Wq [N, K_p]^T) with the same
+ * epilogue; Xq from ss_quant_lift_act(dense), Wq from
+ * ss_compress_weight(dense).  K_p must be a positive multiple of 128. */
+ss_status ss_dense_gemm(const void *Xq, const float *s_x, const void *Wq, const float *s_w,
+                        int64_t M, int64_t N, int64_t K_p, ss_qdtype q, void *Y,
+                        ss_out_dtype out_dtype, ss_stream_t stream);
+
+/* Synchronises `stream`, returns the first device-side error recorded since
+ * the last call (SS_ERR_TIMEOUT, SS_ERR_DATA) or SS_OK, and clears it. */
+ss_status ss_get_device_status(ss_stream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *ss_status_string(ss_status s);
+
+/* Number of kernels this library has launched in this process. */
+int64_t ss_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SS_H_ */

@@ -506,6 +506,8 @@ int ssref_matmul_q(int qdtype, const uint8_t *X, const float *s_x, const uint8_t
                    const int64_t *m_idx, int64_t n_rows, int out_dtype, void *Y) {
     int64_t R = m_idx ? n_rows : M;
     int bad = 0;
+    double lut[256];                        /* value of every 8-bit code */
+    for (int b = 0; b < 256; b++) lut[b] = dequant_one((uint8_t)b, qdtype);
     #pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
     for (int64_t r = 0; r < R; r++) {
         int64_t m = m_idx ? m_idx[r] : r;
@@ -517,7 +519,7 @@ int ssref_matmul_q(int qdtype, const uint8_t *X, const float *s_x, const uint8_t
                 if (qdtype == SSREF_INT8)
                     acc_i += (int64_t)(int8_t)X[m * K + k] * (int64_t)(int8_t)W[n * K + k];
                 else
-                    acc_d += dequant_one(X[m * K + k], qdtype) * dequant_one(W[n * K + k], qdtype);
+                    acc_d += lut[X[m * K + k]] * lut[W[n * K + k]];
             }
             if (acc_i > INT32_MAX || acc_i < INT32_MIN) bad = 1;
             epilogue_store(acc_d, acc_i, qdtype, s_x[m], s_w[n], out_dtype, Y, r * N + n);

@@ -1,0 +1,398 @@
+// ss_api.cu -- the C ABI of libss (declared in include/ss.h): host-side
+// argument checks, TMA tensor-map construction and kernel launches.  All
+// kernels are compiled into this one translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "ss.h"
+#include "ss_common.cuh"
+#include "ss_compress.cuh"
+#include "ss_gemm.cuh"
+#include "ss_quant.cuh"
+
+namespace {
+
+std::atomic<int64_t> g_launches{0};
+
+constexpr int kMaxDevices = 64;
+int g_arch_ok[kMaxDevices];  // 0 unknown, 1 sm_100, -1 other
+int g_num_sms[kMaxDevices];
+std::mutex g_mu;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+ss_status check_device(int* dev_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SS_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return SS_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_arch_ok[dev] == 0) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return SS_ERR_CUDA;
+        g_arch_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+        g_num_sms[dev] = sms;
+    }
+    if (g_arch_ok[dev] != 1) return SS_ERR_ARCH;
+    *dev_out = dev;
+    return SS_OK;
+}
+
+ss_status launched() {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
+}
+
+bool valid_pattern(ss_pattern p) {
+    if (p.keep == 0 && p.group == 0) return true;
+    return (p.group == 4 || p.group == 6 || p.group == 8 || p.group == 10) &&
+           p.keep == p.group - 2;
+}
+
+// ---------------------------------------------------------------- tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D byte matrix [rows, cols] (row stride = cols bytes), box [box_rows, box_cols].
+bool make_map_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                 uint32_t box_rows, uint32_t box_cols, CUtensorMapSwizzle swizzle) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool kSparse, bool kInt8, bool kOutBf16>
+ss_status launch_gemm(int dev, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& e,
+                      const ss::GemmArgs& args, cudaStream_t stream) {
+    using C = ss::GemmCfg<kSparse>;
+    auto kern = ss::gemm_kernel<kSparse, kInt8, kOutBf16>;
+    static std::once_flag once[kMaxDevices];
+    static cudaError_t attr_err[kMaxDevices];
+    std::call_once(once[dev], [&] {
+        attr_err[dev] =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    });
+    if (attr_err[dev] != cudaSuccess) return SS_ERR_CUDA;
+    const int64_t tiles = static_cast<int64_t>((args.rowsA + ss::kTileA - 1) / ss::kTileA) *
+                          ((args.rowsB + args.bn - 1) / args.bn);
+    const int grid = static_cast<int>(tiles < g_num_sms[dev] ? tiles : g_num_sms[dev]);
+    kern<<<grid, ss::kGemmThreads, C::kSmemBytes, stream>>>(a, b, e, args);
+    return launched();
+}
+
+template <bool kSparse>
+ss_status dispatch_gemm(int dev, bool int8, bool bf16, const CUtensorMap& a, const CUtensorMap& b,
+                        const CUtensorMap& e, const ss::GemmArgs& args, cudaStream_t st) {
+    if (int8)
+        return bf16 ? launch_gemm<kSparse, true, true>(dev, a, b, e, args, st)
+                    : launch_gemm<kSparse, true, false>(dev, a, b, e, args, st);
+    return bf16 ? launch_gemm<kSparse, false, true>(dev, a, b, e, args, st)
+                : launch_gemm<kSparse, false, false>(dev, a, b, e, args, st);
+}
+
+// B rows per tile: the whole of a small B, else the largest width <= max.
+int choose_bn(int64_t rowsB, int bn_max) {
+    const int64_t r = round_up(rowsB, 32);
+    return static_cast<int>(r < bn_max ? r : bn_max);
+}
+
+// Opt a row kernel into more than 48 KB of dynamic shared memory when needed.
+template <typename Kern>
+ss_status set_smem(Kern kern, int /*dev*/, size_t bytes) {
+    if (bytes <= 48 * 1024) return SS_OK;
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(bytes)) == cudaSuccess
+               ? SS_OK
+               : SS_ERR_CUDA;
+}
+
+constexpr size_t kMaxRowSmem = 200 * 1024;
+
+}  // namespace
+
+extern "C" {
+
+const char* ss_status_string(ss_status s) {
+    switch (s) {
+        case SS_OK: return "SS_OK";
+        case SS_ERR_INVALID_ARG: return "SS_ERR_INVALID_ARG";
+        case SS_ERR_UNSUPPORTED: return "SS_ERR_UNSUPPORTED";
+        case SS_ERR_ALIGNMENT: return "SS_ERR_ALIGNMENT";
+        case SS_ERR_ARCH: return "SS_ERR_ARCH";
+        case SS_ERR_CUDA: return "SS_ERR_CUDA";
+        case SS_ERR_TIMEOUT: return "SS_ERR_TIMEOUT";
+        case SS_ERR_DATA: return "SS_ERR_DATA";
+    }
+    return "SS_ERR_UNKNOWN";
+}
+
+int64_t ss_kernel_launches(void) { return g_launches.load(); }
+
+ss_status ss_parse_pattern(const char* s, ss_pattern* out) {
+    if (!s || !out) return SS_ERR_INVALID_ARG;
+    if (std::strcmp(s, "dense") == 0) {
+        *out = ss_pattern{0, 0};
+        return SS_OK;
+    }
+    static const char* names[] = {"2:4", "4:6", "6:8", "8:10"};
+    for (int i = 0; i < 4; ++i)
+        if (std::strcmp(s, names[i]) == 0) {
+            *out = ss_pattern{2 * i + 2, 2 * i + 4};
+            return SS_OK;
+        }
+    return SS_ERR_INVALID_ARG;
+}
+
+ss_status ss_slide_shape(ss_pattern p, int64_t K, int64_t* K_pad, int64_t* K_lift,
+                         int64_t* K_lp) {
+    if (!valid_pattern(p) || K <= 0 || K > (int64_t{1} << 30) || !K_pad || !K_lift || !K_lp)
+        return SS_ERR_INVALID_ARG;
+    if (p.group == 0) {
+        *K_pad = K;
+        *K_lift = K;
+        *K_lp = round_up(K, 128);
+        return SS_OK;
+    }
+    const int64_t G = (K + p.group - 1) / p.group;
+    const int64_t Nh = p.group / 2;
+    *K_pad = G * p.group;
+    *K_lift = G * (Nh - 1) * 4;
+    *K_lp = round_up(*K_lift, 128);
+    return SS_OK;
+}
+
+ss_status ss_act_2to4_shape(int64_t K, int64_t* K_lp) {
+    if (K <= 0 || K > (int64_t{1} << 30) || !K_lp) return SS_ERR_INVALID_ARG;
+    *K_lp = round_up(round_up(K, 4), 128);
+    return SS_OK;
+}
+
+ss_status ss_compress_weight(const void* W, ss_in_dtype in_dtype, int64_t N, int64_t K,
+                             ss_pattern p, ss_qdtype q, void* Wv, void* Wm, float* s_w,
+                             ss_stream_t stream) {
+    int64_t K_pad, K_lift, K_lp;
+    ss_status st = ss_slide_shape(p, K, &K_pad, &K_lift, &K_lp);
+    if (st != SS_OK) return st;
+    const bool dense = p.group == 0;
+    if (!W || !Wv || !s_w || (!dense && !Wm) || N <= 0 || N > INT32_MAX) return SS_ERR_INVALID_ARG;
+    if (in_dtype != SS_IN_F32 && in_dtype != SS_IN_BF16) return SS_ERR_INVALID_ARG;
+    if (q != SS_INT8 && q != SS_FP8_E4M3) return SS_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(Wv) || !aligned16(s_w) || (!dense && !aligned16(Wm)))
+        return SS_ERR_ALIGNMENT;
+    const size_t smem = static_cast<size_t>((K_pad * 4 + 15) / 16 * 16) +
+                        (dense ? 0 : 2 * static_cast<size_t>(K_pad / p.group)) + 16;
+    if (smem > kMaxRowSmem) return SS_ERR_UNSUPPORTED;
+    int dev;
+    if ((st = check_device(&dev)) != SS_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* wv = static_cast<uint8_t*>(Wv);
+    uint8_t* wm = static_cast<uint8_t*>(Wm);
+#define SS_COMPRESS(T, I8)                                                                     \
+    do {                                                                                      \
+        auto kern = ss::compress_weight_kernel<T, I8>;                                        \
+        if ((st = set_smem(kern, dev, smem)) != SS_OK) return st;                             \
+        kern<<<static_cast<unsigned>(N), ss::kCompressThreads, smem, s>>>(                    \
+            static_cast<const T*>(W), K, p.keep, p.group, K_lift, K_lp, wv, wm, s_w);         \
+    } while (0)
+    if (in_dtype == SS_IN_BF16) {
+        if (q == SS_INT8) SS_COMPRESS(__nv_bfloat16, true);
+        else SS_COMPRESS(__nv_bfloat16, false);
+    } else {
+        if (q == SS_INT8) SS_COMPRESS(float, true);
+        else SS_COMPRESS(float, false);
+    }
+#undef SS_COMPRESS
+    return launched();
+}
+
+ss_status ss_quant_lift_act(const void* X, ss_in_dtype in_dtype, int64_t M, int64_t K,
+                            ss_pattern p, ss_qdtype q, void* Xq_lift, float* s_x,
+                            ss_stream_t stream) {
+    int64_t K_pad, K_lift, K_lp;
+    ss_status st = ss_slide_shape(p, K, &K_pad, &K_lift, &K_lp);
+    if (st != SS_OK) return st;
+    if (!X || !Xq_lift || !s_x || M <= 0 || M > INT32_MAX) return SS_ERR_INVALID_ARG;
+    if (in_dtype != SS_IN_F32 && in_dtype != SS_IN_BF16) return SS_ERR_INVALID_ARG;
+    if (q != SS_INT8 && q != SS_FP8_E4M3) return SS_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(Xq_lift) || !aligned16(s_x)) return SS_ERR_ALIGNMENT;
+    const size_t esz = in_dtype == SS_IN_BF16 ? 2 : 4;
+    const int64_t q_len = p.group == 0 ? K_lp : K_pad;
+    const size_t smem = static_cast<size_t>((K * esz + 15) / 16 * 16 + round_up(q_len, 16) + 16);
+    if (smem > kMaxRowSmem) return SS_ERR_UNSUPPORTED;
+    int dev;
+    if ((st = check_device(&dev)) != SS_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int Nh = p.group / 2;
+    uint8_t* xq = static_cast<uint8_t*>(Xq_lift);
+#define SS_QLIFT(T, I8)                                                                        \
+    do {                                                                                      \
+        auto kern = ss::quant_lift_kernel<T, I8>;                                             \
+        if ((st = set_smem(kern, dev, smem)) != SS_OK) return st;                             \
+        kern<<<static_cast<unsigned>(M), ss::kRowThreads, smem, s>>>(static_cast<const T*>(X), \
+                                                                      K, Nh, K_lift, K_lp, xq, \
+                                                                      s_x);                   \
+    } while (0)
+    if (in_dtype == SS_IN_BF16) {
+        if (q == SS_INT8) SS_QLIFT(__nv_bfloat16, true);
+        else SS_QLIFT(__nv_bfloat16, false);
+    } else {
+        if (q == SS_INT8) SS_QLIFT(float, true);
+        else SS_QLIFT(float, false);
+    }
+#undef SS_QLIFT
+    return launched();
+}
+
+ss_status ss_prune_act_2to4(const void* X, ss_in_dtype in_dtype, int64_t M, int64_t K,
+                            ss_qdtype q, void* Xv, void* Xm, float* s_x, ss_stream_t stream) {
+    int64_t K_lp;
+    ss_status st = ss_act_2to4_shape(K, &K_lp);
+    if (st != SS_OK) return st;
+    if (!X || !Xv || !Xm || !s_x || M <= 0 || M > INT32_MAX) return SS_ERR_INVALID_ARG;
+    if (in_dtype != SS_IN_F32 && in_dtype != SS_IN_BF16) return SS_ERR_INVALID_ARG;
+    if (q != SS_INT8 && q != SS_FP8_E4M3) return SS_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(Xv) || !aligned16(Xm) || !aligned16(s_x))
+        return SS_ERR_ALIGNMENT;
+    const size_t esz = in_dtype == SS_IN_BF16 ? 2 : 4;
+    const size_t smem = static_cast<size_t>((K * esz + 15) / 16 * 16 + 16);
+    if (smem > kMaxRowSmem) return SS_ERR_UNSUPPORTED;
+    int dev;
+    if ((st = check_device(&dev)) != SS_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* xv = static_cast<uint8_t*>(Xv);
+    uint8_t* xm = static_cast<uint8_t*>(Xm);
+#define SS_PRUNE(T, I8)                                                                        \
+    do {                                                                                      \
+        auto kern = ss::prune_act_kernel<T, I8>;                                              \
+        if ((st = set_smem(kern, dev, smem)) != SS_OK) return st;                             \
+        kern<<<static_cast<unsigned>(M), ss::kRowThreads, smem, s>>>(static_cast<const T*>(X), \
+                                                                      K, K_lp, xv, xm, s_x);  \
+    } while (0)
+    if (in_dtype == SS_IN_BF16) {
+        if (q == SS_INT8) SS_PRUNE(__nv_bfloat16, true);
+        else SS_PRUNE(__nv_bfloat16, false);
+    } else {
+        if (q == SS_INT8) SS_PRUNE(float, true);
+        else SS_PRUNE(float, false);
+    }
+#undef SS_PRUNE
+    return launched();
+}
+
+ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, const float* s_a,
+                         const void* B, const float* s_b, int64_t M, int64_t N, int64_t K_lp,
+                         ss_qdtype q, void* Y, ss_out_dtype out_dtype, ss_stream_t stream) {
+    if (sparse_operand != 0 && sparse_operand != 1) return SS_ERR_INVALID_ARG;
+    if (!Av || !Am || !s_a || !B || !s_b || !Y) return SS_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || M > INT32_MAX || N > INT32_MAX || K_lp <= 0 || K_lp % 128 != 0 ||
+        K_lp > (int64_t{1} << 30))
+        return SS_ERR_INVALID_ARG;
+    if (q != SS_INT8 && q != SS_FP8_E4M3) return SS_ERR_INVALID_ARG;
+    if (out_dtype != SS_OUT_F32 && out_dtype != SS_OUT_BF16) return SS_ERR_INVALID_ARG;
+    if (!aligned16(Av) || !aligned16(Am) || !aligned16(B) || !aligned16(Y)) return SS_ERR_ALIGNMENT;
+    int dev;
+    ss_status st = check_device(&dev);
+    if (st != SS_OK) return st;
+    using C = ss::GemmCfg<true>;
+    const int64_t rowsA = sparse_operand == 0 ? N : M;
+    const int64_t rowsB = sparse_operand == 0 ? M : N;
+    const int bn = choose_bn(rowsB, C::kBnMax);
+    CUtensorMap ta, tb, te;
+    if (!make_map_2d(&ta, Av, rowsA, K_lp / 2, ss::kTileA, C::kARowBytes,
+                     CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_map_2d(&tb, B, rowsB, K_lp, bn, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&te, Am, rowsA, K_lp / 8, ss::kTileA, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return SS_ERR_CUDA;
+    ss::GemmArgs args;
+    args.rowsA = static_cast<int>(rowsA);
+    args.rowsB = static_cast<int>(rowsB);
+    args.k_stages = static_cast<int>(K_lp / 128);
+    args.bn = bn;
+    args.a_is_w = sparse_operand == 0 ? 1 : 0;
+    args.ldy = static_cast<int>(N);
+    args.s_a = s_a;
+    args.s_b = s_b;
+    args.y = Y;
+    return dispatch_gemm<true>(dev, q == SS_INT8, out_dtype == SS_OUT_BF16, ta, tb, te, args,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+ss_status ss_dense_gemm(const void* Xq, const float* s_x, const void* Wq, const float* s_w,
+                        int64_t M, int64_t N, int64_t K_p, ss_qdtype q, void* Y,
+                        ss_out_dtype out_dtype, ss_stream_t stream) {
+    if (!Xq || !s_x || !Wq || !s_w || !Y) return SS_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || M > INT32_MAX || N > INT32_MAX || K_p <= 0 || K_p % 128 != 0 ||
+        K_p > (int64_t{1} << 30))
+        return SS_ERR_INVALID_ARG;
+    if (q != SS_INT8 && q != SS_FP8_E4M3) return SS_ERR_INVALID_ARG;
+    if (out_dtype != SS_OUT_F32 && out_dtype != SS_OUT_BF16) return SS_ERR_INVALID_ARG;
+    if (!aligned16(Xq) || !aligned16(Wq) || !aligned16(Y)) return SS_ERR_ALIGNMENT;
+    int dev;
+    ss_status st = check_device(&dev);
+    if (st != SS_OK) return st;
+    using C = ss::GemmCfg<false>;
+    const int bn = choose_bn(M, C::kBnMax);
+    CUtensorMap ta, tb;
+    if (!make_map_2d(&ta, Wq, N, K_p, ss::kTileA, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tb, Xq, M, K_p, bn, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+        return SS_ERR_CUDA;
+    ss::GemmArgs args;
+    args.rowsA = static_cast<int>(N);
+    args.rowsB = static_cast<int>(M);
+    args.k_stages = static_cast<int>(K_p / 128);
+    args.bn = bn;
+    args.a_is_w = 1;
+    args.ldy = static_cast<int>(N);
+    args.s_a = s_w;
+    args.s_b = s_x;
+    args.y = Y;
+    return dispatch_gemm<false>(dev, q == SS_INT8, out_dtype == SS_OUT_BF16, ta, tb, ta, args,
+                                reinterpret_cast<cudaStream_t>(stream));
+}
+
+ss_status ss_get_device_status(ss_stream_t stream) {
+    int dev;
+    ss_status st = check_device(&dev);
+    if (st != SS_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SS_ERR_CUDA;
+    int code = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(&code, ss::g_status, sizeof(int)) != cudaSuccess) return SS_ERR_CUDA;
+    if (code != 0 && cudaMemcpyToSymbol(ss::g_status, &zero, sizeof(int)) != cudaSuccess)
+        return SS_ERR_CUDA;
+    return static_cast<ss_status>(code);
+}
+
+}  // extern "C"

@@ -1,0 +1,107 @@
+"""CPU checks of the C-ABI library: it loads, exports every function that
+include/ss.h declares, and its host-only logic (pattern parsing, shapes,
+argument validation before any launch) behaves as documented.  No compute
+call runs here: there is no GPU on this machine."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+import structured_sparse_quantized_b200 as ss
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from structured_sparse_quantized_b200 import _build
+    _build.build()
+    return ss.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "ss.h"), encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ss_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ["ss_compress_weight", "ss_quant_lift_act", "ss_prune_act_2to4", "ss_sparse_gemm",
+              "ss_dense_gemm", "ss_slide_shape", "ss_parse_pattern", "ss_get_device_status"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    # same names in the Python binding
+    for name in declared_functions():
+        assert hasattr(ss, name), name
+
+
+def test_parse_pattern():
+    assert ss.ss_parse_pattern("2:4") == (2, 4)
+    assert ss.ss_parse_pattern("4:6") == (4, 6)
+    assert ss.ss_parse_pattern("6:8") == (6, 8)
+    assert ss.ss_parse_pattern("8:10") == (8, 10)
+    assert ss.ss_parse_pattern("dense") == (0, 0)
+    for bad in ["3:4", "6:9", "", "2:4:6", "10:12"]:
+        with pytest.raises(ss.SSError) as e:
+            ss.ss_parse_pattern(bad)
+        assert e.value.status == ss.SS_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("pat", ["dense", "2:4", "4:6", "6:8", "8:10"])
+def test_slide_shape_matches_oracle(pat):
+    for K in [1, 5, 64, 150, 3584, 4096, 14336, 4097]:
+        assert ss.ss_slide_shape(pat, K) == oracle.slide_shape(pat, K)
+    for K in [1, 3, 4, 130, 4096]:
+        assert ss.ss_act_2to4_shape(K) == oracle.act_2to4_k_lp(K)
+
+
+def test_status_strings():
+    assert ss.ss_status_string(ss.SS_OK) == "SS_OK"
+    assert ss.ss_status_string(ss.SS_ERR_TIMEOUT) == "SS_ERR_TIMEOUT"
+    assert ss.ss_status_string(99) == "SS_ERR_UNKNOWN"
+
+
+def test_argument_errors_return_before_any_launch(L):
+    """Validation runs before the device is touched: these return at once."""
+    vp = ctypes.c_void_p
+    good = vp(0x10000)          # never dereferenced: every call below fails first
+    odd = vp(0x10008)
+    pat = ss.ss_pattern(6, 8)
+    # GEMM: K_lp not a multiple of 128, zero sizes, NULL pointers, bad dtype
+    assert L.ss_sparse_gemm(0, good, good, good, good, good, 16, 64, 100, 0, good, 1, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_sparse_gemm(0, good, good, good, good, good, 0, 64, 128, 0, good, 1, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_sparse_gemm(2, good, good, good, good, good, 16, 64, 128, 0, good, 1, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_sparse_gemm(0, None, good, good, good, good, 16, 64, 128, 0, good, 1, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_sparse_gemm(0, good, good, good, good, good, 16, 64, 128, 5, good, 1, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_sparse_gemm(0, odd, good, good, good, good, 16, 64, 128, 0, good, 1, None) \
+        == ss.SS_ERR_ALIGNMENT
+    assert L.ss_dense_gemm(good, good, good, good, 16, 64, 96, 0, good, 1, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_dense_gemm(good, good, odd, good, 16, 64, 128, 0, good, 1, None) \
+        == ss.SS_ERR_ALIGNMENT
+    # activation kernels
+    assert L.ss_quant_lift_act(good, 1, 16, 0, pat, 0, good, good, None) == ss.SS_ERR_INVALID_ARG
+    assert L.ss_quant_lift_act(good, 3, 16, 64, pat, 0, good, good, None) == ss.SS_ERR_INVALID_ARG
+    assert L.ss_quant_lift_act(good, 1, 16, 64, ss.ss_pattern(3, 4), 0, good, good, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_quant_lift_act(odd, 1, 16, 64, pat, 0, good, good, None) == ss.SS_ERR_ALIGNMENT
+    assert L.ss_prune_act_2to4(good, 1, -1, 64, 0, good, good, good, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_prune_act_2to4(good, 1, 16, 64, 0, good, odd, good, None) == ss.SS_ERR_ALIGNMENT
+    # weight compression: Wm required unless dense; rows too long for one CTA
+    assert L.ss_compress_weight(good, 1, 64, 64, pat, 0, good, None, good, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_compress_weight(good, 1, 64, 1 << 20, pat, 0, good, good, good, None) \
+        == ss.SS_ERR_UNSUPPORTED

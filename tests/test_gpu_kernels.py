@@ -1,0 +1,175 @@
+"""GPU parity of every libss kernel against the CPU oracle on small shapes
+that span several tiles and ragged tails.  Bytes (quantised operands,
+packed values, metadata, scales) and INT8 results must be bit-exact; FP8
+results must be within the relative tolerance of 1e-2."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import structured_sparse_quantized_b200 as ss
+from structured_sparse_quantized_b200 import synth
+from _helpers import Q, assert_y_matches, dev, host
+
+pytestmark = pytest.mark.gpu
+
+PATTERNS = ["2:4", "4:6", "6:8", "8:10"]
+IN_DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+def _x(M, K, dt, seed=1, scale=1.0):
+    return synth.gaussian((M, K), std=scale, seed=seed, dtype=IN_DTYPES[dt])
+
+
+@pytest.mark.parametrize("pat", ["dense"] + PATTERNS)
+@pytest.mark.parametrize("q", ["int8", "fp8"])
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("M,K", [(1, 64), (3, 150), (129, 1000), (16, 4100)])
+def test_quant_lift_act(pat, q, dt, M, K):
+    X = _x(M, K, dt, seed=M + K)
+    Xq_ref, s_ref = oracle.quant_lift_act(X, pat, Q[q])
+    Xq, s_x = ss.quant_lift_act(dev(X), pat, q)
+    np.testing.assert_array_equal(host(s_x), s_ref)
+    np.testing.assert_array_equal(host(Xq), Xq_ref)
+
+
+@pytest.mark.parametrize("q", ["int8", "fp8"])
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("M,K", [(1, 64), (5, 150), (130, 1030), (7, 4096)])
+def test_prune_act_2to4(q, dt, M, K):
+    X = _x(M, K, dt, seed=3 * M + K)
+    Xv_ref, Xm_ref, s_ref = oracle.prune_act_2to4(X, Q[q])
+    Xv, Xm, s_x = ss.prune_act_2to4(dev(X), q)
+    np.testing.assert_array_equal(host(s_x), s_ref)
+    np.testing.assert_array_equal(host(Xm), Xm_ref)
+    np.testing.assert_array_equal(host(Xv), Xv_ref)
+
+
+@pytest.mark.parametrize("pat", ["dense"] + PATTERNS)
+@pytest.mark.parametrize("q", ["int8", "fp8"])
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("N,K", [(1, 64), (64, 150), (130, 1000)])
+def test_compress_weight(pat, q, dt, N, K):
+    W = _x(N, K, dt, seed=N * 7 + K, scale=0.02)
+    Wv_ref, Wm_ref, s_ref = oracle.compress_weight(W, pat, Q[q])
+    Wv, Wm, s_w = ss.compress_weight(dev(W), pat, q)
+    np.testing.assert_array_equal(host(s_w), s_ref)
+    np.testing.assert_array_equal(host(Wv), Wv_ref)
+    if pat != "dense":
+        np.testing.assert_array_equal(host(Wm), Wm_ref)
+    assert ss.ss_get_device_status() == ss.SS_OK
+
+
+def test_compress_weight_with_ties_and_zeros():
+    """Exact ties, zero groups and a zero row exercise the tie rule, the
+    padding of windows with fewer than two owners, and the zero scale."""
+    W = torch.tensor(np.random.default_rng(0).integers(-3, 4, (40, 96)), dtype=torch.float32)
+    W[5] = 0.0
+    for pat in PATTERNS:
+        for q in ["int8", "fp8"]:
+            Wv_ref, Wm_ref, s_ref = oracle.compress_weight(W, pat, Q[q])
+            Wv, Wm, s_w = ss.compress_weight(dev(W), pat, q)
+            np.testing.assert_array_equal(host(s_w), s_ref)
+            np.testing.assert_array_equal(host(Wv), Wv_ref)
+            np.testing.assert_array_equal(host(Wm), Wm_ref)
+
+
+def test_nan_weight_reports_data_error():
+    W = torch.randn(8, 64)
+    W[3, 10] = float("nan")
+    ss.compress_weight(dev(W), "6:8", "int8")
+    assert ss.ss_get_device_status() == ss.SS_ERR_DATA
+    assert ss.ss_get_device_status() == ss.SS_OK        # cleared by the read
+
+
+# ---------------------------------------------------------------- GEMMs
+
+GEMM_CASES = [  # M, N, K, pattern
+    (16, 64, 64, "6:8"),        # the single-linear workload shape
+    (1, 130, 300, "2:4"),       # one token, ragged channel tile
+    (37, 257, 1000, "4:6"),     # ragged both ways, K not a multiple of 6
+    (300, 200, 600, "8:10"),    # two token tiles
+    (500, 384, 2048, "6:8"),    # three token tiles, 24 K stages
+]
+
+
+@pytest.mark.parametrize("M,N,K,pat", GEMM_CASES)
+@pytest.mark.parametrize("q", ["int8", "fp8"])
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+def test_sparse_gemm_weight_sparse(M, N, K, pat, q, out):
+    W = synth.gaussian((N, K), std=0.02, seed=0, dtype=torch.bfloat16)
+    X = synth.gaussian((M, K), std=1.0, seed=1, dtype=torch.bfloat16)
+    Wv, Wm, s_w = oracle.compress_weight(W, pat, Q[q])
+    Xq, s_x = oracle.quant_lift_act(X, pat, Q[q])
+    _, _, K_lp = oracle.slide_shape(pat, K)
+    ob = out == "bf16"
+    Y_ref = oracle.sparse_gemm(0, Wv, Wm, s_w, Xq, s_x, M, N, K_lp, Q[q],
+                               oracle.OUT_BF16 if ob else oracle.OUT_F32)
+    Y = ss.sparse_gemm(0, dev(Wv), dev(Wm), dev(s_w), dev(Xq), dev(s_x), M, N, q,
+                       out_dtype=torch.bfloat16 if ob else torch.float32)
+    assert ss.ss_get_device_status() == ss.SS_OK
+    assert_y_matches(host(Y), Y_ref, q, ob)
+
+
+@pytest.mark.parametrize("M,N,K", [(130, 64, 256), (257, 300, 1024), (8, 96, 4096)])
+@pytest.mark.parametrize("q", ["int8", "fp8"])
+def test_sparse_gemm_activation_sparse(M, N, K, q):
+    W = synth.gaussian((N, K), std=0.02, seed=0, dtype=torch.bfloat16)
+    X = synth.gaussian_with_heavy_tails(M, K, seed=1)
+    Xv, Xm, s_x = oracle.prune_act_2to4(X, Q[q])
+    Wq, _, s_w = oracle.compress_weight(W, "dense", Q[q])
+    K_lp = oracle.act_2to4_k_lp(K)
+    assert Wq.shape[1] == K_lp
+    Y_ref = oracle.sparse_gemm(1, Xv, Xm, s_x, Wq, s_w, M, N, K_lp, Q[q], oracle.OUT_BF16)
+    Y = ss.sparse_gemm(1, dev(Xv), dev(Xm), dev(s_x), dev(Wq), dev(s_w), M, N, q)
+    assert ss.ss_get_device_status() == ss.SS_OK
+    assert_y_matches(host(Y), Y_ref, q, True)
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 64, 64), (1, 130, 300), (300, 257, 1000), (600, 128, 512)])
+@pytest.mark.parametrize("q", ["int8", "fp8"])
+def test_dense_gemm(M, N, K, q):
+    W = synth.gaussian((N, K), std=0.02, seed=0, dtype=torch.bfloat16)
+    X = synth.gaussian((M, K), std=1.0, seed=1, dtype=torch.bfloat16)
+    Wq, _, s_w = oracle.compress_weight(W, "dense", Q[q])
+    Xq, s_x = oracle.quant_lift_act(X, "dense", Q[q])
+    Y_ref = oracle.dense_gemm(Xq, s_x, Wq, s_w, Q[q], oracle.OUT_BF16)
+    Y = ss.dense_gemm(dev(Xq), dev(s_x), dev(Wq), dev(s_w), q)
+    assert ss.ss_get_device_status() == ss.SS_OK
+    assert_y_matches(host(Y), Y_ref, q, True)
+
+
+@pytest.mark.parametrize("pat", PATTERNS)
+@pytest.mark.parametrize("q", ["int8", "fp8"])
+def test_chained_gpu_path_matches_plain_definition(pat, q):
+    """GPU compress -> GPU quant+lift -> GPU sparse GEMM equals the oracle's
+    plain path (prune, quantise, naive matmul over the original K): the
+    lossless-decomposition identity, end to end on the device."""
+    M, N, K = 70, 200, 333
+    W = synth.gaussian((N, K), std=0.02, seed=0, dtype=torch.bfloat16)
+    X = synth.gaussian((M, K), std=1.0, seed=1, dtype=torch.bfloat16)
+    plain = oracle.plain_linear(W, X, pat, Q[q], oracle.OUT_BF16)
+    Y = ss.linear(dev(X), ss.compress_weight(dev(W), pat, q), pat, q)
+    assert_y_matches(host(Y), plain, q, True)
+
+
+def test_zero_rows_and_channels():
+    M, N, K = 20, 140, 256
+    W = synth.gaussian((N, K), std=0.02, seed=0, dtype=torch.bfloat16)
+    X = synth.gaussian((M, K), std=1.0, seed=1, dtype=torch.bfloat16)
+    W[7] = 0
+    X[3] = 0
+    for q in ["int8", "fp8"]:
+        packed = ss.compress_weight(dev(W), "6:8", q)
+        Y = host(ss.linear(dev(X), packed, "6:8", q)).view(np.uint16)
+        assert np.all(Y[3] == 0) and np.all(Y[:, 7] == 0)
+        plain = oracle.plain_linear(W, X, "6:8", Q[q], oracle.OUT_BF16)
+        assert_y_matches(Y, plain, q, True)
+
+
+def test_launch_counter_and_status():
+    before = ss.ss_kernel_launches()
+    X = synth.gaussian((4, 64), seed=2, dtype=torch.bfloat16)
+    ss.quant_lift_act(dev(X), "6:8", "int8")
+    assert ss.ss_kernel_launches() == before + 1
+    assert ss.ss_get_device_status() == ss.SS_OK
