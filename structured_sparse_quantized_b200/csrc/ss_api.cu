@@ -78,25 +78,39 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D byte matrix [rows, cols] (row stride = cols bytes), box [box_rows, box_cols].
+// 2-D row-major matrix [rows, cols] of `esz`-byte elements, box [box_rows, box_cols].
 bool make_map_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                 uint32_t box_rows, uint32_t box_cols, CUtensorMapSwizzle swizzle) {
+                 uint32_t box_rows, uint32_t box_cols, CUtensorMapSwizzle swizzle,
+                 CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_UINT8, uint32_t esz = 1) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols};
+    cuuint64_t strides[1] = {cols * esz};
     cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool kSparse, bool kInt8, bool kOutBf16>
+// Tensor map of Y [M, N] for the epilogue's TMA stores of one 32-column chunk:
+// box [32 tokens][128 channels] when A rows are channels, [128 tokens][32
+// channels] otherwise.  Returns false (direct stores instead) when the rows
+// of Y are not 16-byte aligned.
+bool make_y_map(CUtensorMap* map, void* Y, int64_t M, int64_t N, bool out_bf16, bool a_is_w) {
+    const uint32_t esz = out_bf16 ? 2 : 4;
+    if ((N * esz) % 16 != 0) return false;
+    const CUtensorMapDataType dt =
+        out_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    return a_is_w ? make_map_2d(map, Y, M, N, 32, ss::kTileA, CU_TENSOR_MAP_SWIZZLE_NONE, dt, esz)
+                  : make_map_2d(map, Y, M, N, ss::kTileA, 32, CU_TENSOR_MAP_SWIZZLE_NONE, dt, esz);
+}
+
+template <bool kSparse, bool kInt8, bool kOutBf16, int kPair>
 ss_status launch_gemm(int dev, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& e,
-                      const ss::GemmArgs& args, cudaStream_t stream) {
-    using C = ss::GemmCfg<kSparse>;
-    auto kern = ss::gemm_kernel<kSparse, kInt8, kOutBf16>;
+                      const CUtensorMap& y, const ss::GemmArgs& args, cudaStream_t stream) {
+    using C = ss::GemmCfg<kSparse, kPair>;
+    auto kern = ss::gemm_kernel<kSparse, kInt8, kOutBf16, kPair>;
     static std::once_flag once[kMaxDevices];
     static cudaError_t attr_err[kMaxDevices];
     std::call_once(once[dev], [&] {
@@ -104,21 +118,39 @@ ss_status launch_gemm(int dev, const CUtensorMap& a, const CUtensorMap& b, const
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     });
     if (attr_err[dev] != cudaSuccess) return SS_ERR_CUDA;
-    const int64_t tiles = static_cast<int64_t>((args.rowsA + ss::kTileA - 1) / ss::kTileA) *
-                          ((args.rowsB + args.bn - 1) / args.bn);
-    const int grid = static_cast<int>(tiles < g_num_sms[dev] ? tiles : g_num_sms[dev]);
-    kern<<<grid, ss::kGemmThreads, C::kSmemBytes, stream>>>(a, b, e, args);
+    const int64_t tiles =
+        static_cast<int64_t>((args.rowsA + ss::kTileA * kPair - 1) / (ss::kTileA * kPair)) *
+        ((args.rowsB + args.bn - 1) / args.bn);
+    const int64_t units = g_num_sms[dev] / kPair;
+    const int grid = static_cast<int>((tiles < units ? tiles : units) * kPair);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(ss::kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kPair;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, a, b, e, y, args) != cudaSuccess) {
+        cudaGetLastError();
+        return SS_ERR_CUDA;
+    }
     return launched();
 }
 
-template <bool kSparse>
+template <bool kSparse, int kPair>
 ss_status dispatch_gemm(int dev, bool int8, bool bf16, const CUtensorMap& a, const CUtensorMap& b,
-                        const CUtensorMap& e, const ss::GemmArgs& args, cudaStream_t st) {
+                        const CUtensorMap& e, const CUtensorMap& y, const ss::GemmArgs& args,
+                        cudaStream_t st) {
     if (int8)
-        return bf16 ? launch_gemm<kSparse, true, true>(dev, a, b, e, args, st)
-                    : launch_gemm<kSparse, true, false>(dev, a, b, e, args, st);
-    return bf16 ? launch_gemm<kSparse, false, true>(dev, a, b, e, args, st)
-                : launch_gemm<kSparse, false, false>(dev, a, b, e, args, st);
+        return bf16 ? launch_gemm<kSparse, true, true, kPair>(dev, a, b, e, y, args, st)
+                    : launch_gemm<kSparse, true, false, kPair>(dev, a, b, e, y, args, st);
+    return bf16 ? launch_gemm<kSparse, false, true, kPair>(dev, a, b, e, y, args, st)
+                : launch_gemm<kSparse, false, false, kPair>(dev, a, b, e, y, args, st);
 }
 
 // B rows per tile: the whole of a small B, else the largest width <= max.
@@ -247,7 +279,7 @@ ss_status ss_quant_lift_act(const void* X, ss_in_dtype in_dtype, int64_t M, int6
     if (q != SS_INT8 && q != SS_FP8_E4M3) return SS_ERR_INVALID_ARG;
     if (!aligned16(X) || !aligned16(Xq_lift) || !aligned16(s_x)) return SS_ERR_ALIGNMENT;
     const size_t esz = in_dtype == SS_IN_BF16 ? 2 : 4;
-    const int64_t q_len = p.group == 0 ? K_lp : K_pad;
+    const int64_t q_len = p.group <= 4 ? 0 : K_pad;  // byte row only for sliding patterns
     const size_t smem = static_cast<size_t>((K * esz + 15) / 16 * 16 + round_up(q_len, 16) + 16);
     if (smem > kMaxRowSmem) return SS_ERR_UNSUPPORTED;
     int dev;
@@ -324,14 +356,13 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
     int dev;
     ss_status st = check_device(&dev);
     if (st != SS_OK) return st;
-    using C = ss::GemmCfg<true>;
     const int64_t rowsA = sparse_operand == 0 ? N : M;
     const int64_t rowsB = sparse_operand == 0 ? M : N;
-    const int bn = choose_bn(rowsB, C::kBnMax);
+    const int pair = rowsA > ss::kTileA ? 2 : 1;
+    const int bn = choose_bn(rowsB, ss::GemmCfg<true, 1>::kBnMax);
     CUtensorMap ta, tb, te;
-    if (!make_map_2d(&ta, Av, rowsA, K_lp / 2, ss::kTileA, C::kARowBytes,
-                     CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !make_map_2d(&tb, B, rowsB, K_lp, bn, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+    if (!make_map_2d(&ta, Av, rowsA, K_lp / 2, ss::kTileA, 64, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_map_2d(&tb, B, rowsB, K_lp, bn / pair, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&te, Am, rowsA, K_lp / 8, ss::kTileA, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
         return SS_ERR_CUDA;
     ss::GemmArgs args;
@@ -344,8 +375,15 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
     args.s_a = s_a;
     args.s_b = s_b;
     args.y = Y;
-    return dispatch_gemm<true>(dev, q == SS_INT8, out_dtype == SS_OUT_BF16, ta, tb, te, args,
-                               reinterpret_cast<cudaStream_t>(stream));
+    CUtensorMap ty;
+    args.tma_store = make_y_map(&ty, Y, M, N, out_dtype == SS_OUT_BF16, args.a_is_w) ? 1 : 0;
+    if (!args.tma_store) ty = ta;  // unused
+    cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
+    return pair == 2
+               ? dispatch_gemm<true, 2>(dev, q == SS_INT8, out_dtype == SS_OUT_BF16, ta, tb, te,
+                                        ty, args, st_)
+               : dispatch_gemm<true, 1>(dev, q == SS_INT8, out_dtype == SS_OUT_BF16, ta, tb, te,
+                                        ty, args, st_);
 }
 
 ss_status ss_dense_gemm(const void* Xq, const float* s_x, const void* Wq, const float* s_w,
@@ -361,11 +399,11 @@ ss_status ss_dense_gemm(const void* Xq, const float* s_x, const void* Wq, const 
     int dev;
     ss_status st = check_device(&dev);
     if (st != SS_OK) return st;
-    using C = ss::GemmCfg<false>;
-    const int bn = choose_bn(M, C::kBnMax);
+    const int pair = N > ss::kTileA ? 2 : 1;
+    const int bn = choose_bn(M, ss::GemmCfg<false, 1>::kBnMax);
     CUtensorMap ta, tb;
     if (!make_map_2d(&ta, Wq, N, K_p, ss::kTileA, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_2d(&tb, Xq, M, K_p, bn, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+        !make_map_2d(&tb, Xq, M, K_p, bn / pair, 128, CU_TENSOR_MAP_SWIZZLE_128B))
         return SS_ERR_CUDA;
     ss::GemmArgs args;
     args.rowsA = static_cast<int>(N);
@@ -377,8 +415,15 @@ ss_status ss_dense_gemm(const void* Xq, const float* s_x, const void* Wq, const 
     args.s_a = s_w;
     args.s_b = s_x;
     args.y = Y;
-    return dispatch_gemm<false>(dev, q == SS_INT8, out_dtype == SS_OUT_BF16, ta, tb, ta, args,
-                                reinterpret_cast<cudaStream_t>(stream));
+    CUtensorMap ty;
+    args.tma_store = make_y_map(&ty, Y, M, N, out_dtype == SS_OUT_BF16, true) ? 1 : 0;
+    if (!args.tma_store) ty = ta;  // unused
+    cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
+    return pair == 2
+               ? dispatch_gemm<false, 2>(dev, q == SS_INT8, out_dtype == SS_OUT_BF16, ta, tb, ta,
+                                         ty, args, st_)
+               : dispatch_gemm<false, 1>(dev, q == SS_INT8, out_dtype == SS_OUT_BF16, ta, tb, ta,
+                                         ty, args, st_);
 }
 
 ss_status ss_get_device_status(ss_stream_t stream) {

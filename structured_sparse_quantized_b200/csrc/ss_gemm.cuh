@@ -12,21 +12,30 @@
 // sparse tensor core; SlideSparse write-up, omica.com.cn, 2.2 sparse GEMM
 // execution).  The dense variant is the like-for-like comparison.
 //
+// kPair = 2 (the default for problems with more than 128 A rows): a cluster
+// of two CTAs on two SMs issues one MMA of M = 256 (tcgen05 cta_group::2).
+// Each CTA loads its own 128 A rows and its own half of the B rows into its
+// own shared memory, so each SM moves half the B bytes per MAC of a one-SM
+// tile; D is split by A rows between the two tensor memories.  kPair = 1 is
+// the single-SM form (M = 128).
+//
 // CTA = 6 warps, one CTA per SM, persistent over output tiles:
-//   warp 0       TMA producer: A tile (128 rows), B tile (BN rows) and, for
-//                the sparse variant, the 128 x 16-byte metadata tile of each
-//                K stage, into a ring of shared-memory stages.
-//   warp 1       allocates 512 TMEM columns; one lane issues the MMAs (and
-//                the shared->tensor-memory metadata copies) into one of two
-//                accumulator buffers and commits stage / accumulator
-//                barriers.
+//   warp 0       TMA producer: A tile, B tile and, for the sparse variant, the
+//                128 x 16-byte metadata tile of each K stage, into a ring of
+//                shared-memory stages.  Both CTAs of a pair count their bytes
+//                on the leader CTA's "full" barrier.
+//   warp 1       allocates 512 TMEM columns (both CTAs); in the leader CTA one
+//                lane issues the MMAs (and the metadata copies into tensor
+//                memory) into one of two accumulator buffers and commits the
+//                stage / accumulator barriers of both CTAs.
 //   warps 2-5    epilogue: tcgen05.ld the accumulator (lane = A row, column =
-//                B row), scale, convert, store Y; release the buffer.
+//                B row), scale, convert, store Y; release the buffer on the
+//                leader's barrier.
 // Stage K is 128 logical elements: dense = 4 MMAs of K=32 (A and B 128-byte
 // rows, 128B swizzle); sparse = 2 MMAs of K=64 (A holds 64 compressed bytes
 // per row, 64B swizzle; B 128-byte rows, 128B swizzle; metadata 16 bytes per
-// A row, one tcgen05.cp of 128 lanes x 128 bits).
-// Every wait is bounded (ss_common.cuh); nothing here multicasts.
+// A row, copied to tensor memory as 128 lanes x 128 bits).
+// Every wait is bounded (ss_common.cuh); no load multicasts.
 #pragma once
 
 #include "ss_common.cuh"
@@ -34,37 +43,44 @@
 namespace ss {
 
 constexpr int kGemmThreads = 192;
-constexpr int kTileA = 128;
+constexpr int kTileA = 128;  // A rows per CTA
 constexpr int kTmemCols = 512;
 
-template <bool kSparse>
+template <bool kSparse, int kPair>
 struct GemmCfg {
     static constexpr int kStageK = 128;                    // logical K per stage
     static constexpr int kMmaK = kSparse ? 64 : 32;        // logical K per MMA
     static constexpr int kMmaPerStage = kStageK / kMmaK;   // 2 / 4
     static constexpr int kARowBytes = kSparse ? 64 : 128;  // A bytes per row per stage
     static constexpr int kABytes = kTileA * kARowBytes;
-    static constexpr int kBnMax = kSparse ? 224 : 256;     // 2 accumulators (+ metadata) in TMEM
-    static constexpr int kBBytes = kBnMax * 128;
+    static constexpr int kBnMax = kSparse ? 224 : 256;     // MMA N; 2 accumulators (+ metadata)
+    static constexpr int kBRowsMax = kBnMax / kPair;       // B rows held per CTA
+    static constexpr int kBBytes = kBRowsMax * 128;
     static constexpr int kEBytes = kSparse ? kTileA * 16 : 0;
-    static constexpr int kStageBytes = kABytes + kBBytes + kEBytes;
-    static constexpr int kStages = kSparse ? 5 : 4;
+    static constexpr int kStageRaw = kABytes + kBBytes + kEBytes;
+    static constexpr int kStageBytes = (kStageRaw + 1023) / 1024 * 1024;
+    static constexpr int kEpiBytes = 32 * kTileA * 4;      // one 32-column chunk, fp32 worst case
+    static constexpr int kStagesRaw = (196 * 1024 - 2 * kEpiBytes) / kStageBytes;
+    static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
     static constexpr int kAccStride = kBnMax;              // TMEM columns between buffers
     static constexpr int kECol = 2 * kBnMax;               // metadata columns (sparse)
     static constexpr int kESlots = 4;                      // 4 columns each
-    static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
-    static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
+    static constexpr int kEpiOffset = kStages * kStageBytes;  // 2 staging buffers for Y chunks
+    static constexpr int kSmemBytes =
+        kEpiOffset + 2 * kEpiBytes + 1024 /*align*/ + 256 /*barriers*/;
     static_assert(kABytes % 1024 == 0 && (kABytes + kBBytes) % 1024 == 0, "tile alignment");
     static_assert(!kSparse || kECol + kESlots * 4 <= kTmemCols, "TMEM budget");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
 struct GemmArgs {
-    int rowsA;        // rows of A (128-row tiles)
-    int rowsB;        // rows of B (BN-row tiles)
+    int rowsA;        // rows of A
+    int rowsB;        // rows of B
     int k_stages;     // K / 128
-    int bn;           // B rows per tile (multiple of 32, <= kBnMax)
+    int bn;           // B rows per tile (MMA N; multiple of 32 (x kPair), <= kBnMax)
     int a_is_w;       // 1: A rows are output channels (Y[b, a]); 0: Y[a, b]
     int ldy;          // leading dimension of Y (= N)
+    int tma_store;    // 1: Y written by TMA tensor stores through shared memory
     const float* s_a;
     const float* s_b;
     void* y;
@@ -90,15 +106,16 @@ __device__ __forceinline__ void store_scaled(void* y, int64_t off, uint32_t acc_
         reinterpret_cast<float*>(y)[off] = v;
 }
 
-template <bool kSparse, bool kInt8, bool kOutBf16>
+template <bool kSparse, bool kInt8, bool kOutBf16, int kPair>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                const __grid_constant__ CUtensorMap tm_e, const GemmArgs args) {
-    using C = GemmCfg<kSparse>;
+                const __grid_constant__ CUtensorMap tm_e, const __grid_constant__ CUtensorMap tm_y,
+                const GemmArgs args) {
+    using C = GemmCfg<kSparse, kPair>;
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kEpiOffset + 2 * C::kEpiBytes);
     uint64_t* empty = full + C::kStages;
     uint64_t* acc_full = empty + C::kStages;
     uint64_t* acc_empty = acc_full + 2;
@@ -109,9 +126,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int nA = (args.rowsA + kTileA - 1) / kTileA;
+    const uint32_t rank = kPair == 2 ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    const int tile_a_rows = kTileA * kPair;
+    const int b_rows_cta = args.bn / kPair;
+    const int nA = (args.rowsA + tile_a_rows - 1) / tile_a_rows;
     const int nB = (args.rowsB + args.bn - 1) / args.bn;
     const int n_tiles = nA * nB;
+    const int unit = blockIdx.x / kPair;   // cluster index
+    const int n_units = gridDim.x / kPair;
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
@@ -121,17 +144,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 4);
+            mbar_init(&acc_empty[b], 4 * kPair);
         }
         mbar_init(drain, 1);
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_base_slot, kTmemCols);
-        tmem_relinquish();
+        tmem_alloc_g<kPair>(tmem_base_slot, kTmemCols);
+        tmem_relinquish_g<kPair>();
     }
     tc_fence_before();
-    __syncthreads();
+    if constexpr (kPair == 2)
+        cluster_sync_all();  // peer barriers initialised before any remote use
+    else
+        __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_base_slot;
 
@@ -141,24 +167,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tma_prefetch_desc(&tm_a);
             tma_prefetch_desc(&tm_b);
             if (kSparse) tma_prefetch_desc(&tm_e);
-            const uint32_t tx = C::kABytes + args.bn * 128 + C::kEBytes;
+            const uint32_t tx = kPair * (C::kABytes + b_rows_cta * 128 + C::kEBytes);
             int s = 0;
             uint32_t ph = 0, armed = 0, armed_par = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-                const int a0 = (t % nA) * kTileA;
-                const int b0 = (t / nA) * args.bn;
+            for (int t = unit; t < n_tiles && ok; t += n_units) {
+                const int a0 = (t % nA) * tile_a_rows + static_cast<int>(rank) * kTileA;
+                const int b0 = (t / nA) * args.bn + static_cast<int>(rank) * b_rows_cta;
                 for (int kb = 0; kb < args.k_stages; ++kb) {
                     if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
                     uint8_t* st = smem + s * C::kStageBytes;
-                    mbar_arrive_expect_tx(&full[s], tx);
-                    tma_load_2d(st, &tm_a, &full[s], kb * C::kARowBytes, a0);
-                    tma_load_2d(st + C::kABytes, &tm_b, &full[s], kb * 128, b0);
-                    if (kSparse)
-                        tma_load_2d(st + C::kABytes + C::kBBytes, &tm_e, &full[s], kb * 16, a0);
+                    if constexpr (kPair == 2) {
+                        if (leader) mbar_arrive_expect_tx(&full[s], tx);
+                        const uint32_t fb = map_to_rank(&full[s], 0);
+                        tma_load_2d_pair(st, &tm_a, fb, kb * C::kARowBytes, a0);
+                        tma_load_2d_pair(st + C::kABytes, &tm_b, fb, kb * 128, b0);
+                        if (kSparse)
+                            tma_load_2d_pair(st + C::kABytes + C::kBBytes, &tm_e, fb, kb * 16, a0);
+                    } else {
+                        mbar_arrive_expect_tx(&full[s], tx);
+                        tma_load_2d(st, &tm_a, &full[s], kb * C::kARowBytes, a0);
+                        tma_load_2d(st + C::kABytes, &tm_b, &full[s], kb * 128, b0);
+                        if (kSparse)
+                            tma_load_2d(st + C::kABytes + C::kBBytes, &tm_e, &full[s], kb * 16,
+                                        a0);
+                    }
                     armed |= 1u << s;
                     armed_par = (armed_par & ~(1u << s)) | (ph << s);
                     if (++s == C::kStages) {
@@ -167,21 +203,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
             }
-            if (!ok) {  // let every copy already issued land before the CTA exits
-                for (int i = 0; i < C::kStages; ++i)
-                    if ((armed >> i) & 1u) mbar_drain(&full[i], (armed_par >> i) & 1u);
+            if (!ok) {  // let the copies already issued land before the CTA exits
+                if (kPair == 1 || leader) {
+                    for (int i = 0; i < C::kStages; ++i)
+                        if ((armed >> i) & 1u) mbar_drain(&full[i], (armed_par >> i) & 1u);
+                } else {  // the peer's copies count on the leader's barriers: wait 1 ms
+                    const uint64_t t0 = global_timer_ns();
+                    while (global_timer_ns() - t0 < 1000000ull) {
+                    }
+                }
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = make_idesc(kSparse, kInt8, kTileA, args.bn);
+        if (lane == 0 && leader) {
+            const uint32_t idesc = make_idesc(kSparse, kInt8, kTileA * kPair, args.bn);
             int s = 0;
             uint32_t ph = 0;
             uint32_t e_iter = 0;
             bool ok = true;
             int i = 0;
-            for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++i) {
+            for (int t = unit; t < n_tiles && ok; t += n_units, ++i) {
                 const int buf = i & 1;
                 const uint32_t aph = (i >> 1) & 1;
                 if (!mbar_wait(&acc_empty[buf], aph ^ 1u, abort_flag)) {
@@ -204,7 +246,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         ++e_iter;
                         const uint64_t e_desc =
                             smem_desc(b_addr + C::kBBytes, 128 * 16, 128, kSwizzleNone);
-                        tc_cp_128x128b(e_tmem, e_desc);
+                        tc_cp_128x128b_g<kPair>(e_tmem, e_desc);
                     }
 #pragma unroll
                     for (int j = 0; j < C::kMmaPerStage; ++j) {
@@ -214,40 +256,55 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                 smem_desc(a_addr + j * 32, 16, 8 * 64, kSwizzle64B);
                             const uint64_t b_desc =
                                 smem_desc(b_addr + j * 64, 16, 8 * 128, kSwizzle128B);
-                            mma_sparse<kInt8>(d_tmem, a_desc, b_desc, e_tmem + 2 * j, idesc, acc);
+                            mma_sparse_g<kPair, kInt8>(d_tmem, a_desc, b_desc, e_tmem + 2 * j,
+                                                       idesc, acc);
                         } else {
                             const uint64_t a_desc =
                                 smem_desc(a_addr + j * 32, 16, 8 * 128, kSwizzle128B);
                             const uint64_t b_desc =
                                 smem_desc(b_addr + j * 32, 16, 8 * 128, kSwizzle128B);
-                            mma_dense<kInt8>(d_tmem, a_desc, b_desc, idesc, acc);
+                            mma_dense_g<kPair, kInt8>(d_tmem, a_desc, b_desc, idesc, acc);
                         }
                     }
-                    tc_commit(&empty[s]);  // stage free once these MMAs have read it
+                    tc_commit_g<kPair>(&empty[s]);  // stage free in both CTAs once read
                     if (++s == C::kStages) {
                         s = 0;
                         ph ^= 1u;
                     }
                 }
                 if (!ok) break;
-                tc_commit(&acc_full[buf]);
+                tc_commit_g<kPair>(&acc_full[buf]);
             }
             if (!ok) {  // wait for every MMA already issued before TMEM is freed
-                tc_commit(drain);
+                tc_commit_g<kPair>(drain);
                 mbar_drain(drain, 0);
             }
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        // Each 32-column chunk of the accumulator is scaled, converted and
+        // written to one of two shared-memory staging buffers laid out as the
+        // chunk's box of Y, then stored by one TMA tensor store (clipped at
+        // the edges of Y).  Without TMA stores (Y rows not 16-byte aligned)
+        // the values go straight to global memory.
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const int lane_row = q * 32 + lane;
+        const bool issuer = (warp == 2 && lane == 0);
+        const uint32_t acc_empty_leader = kPair == 2 ? map_to_rank(acc_empty, 0) : 0u;
+        constexpr int kEsz = kOutBf16 ? 2 : 4;
+        uint8_t* stage_y = smem + C::kEpiOffset;
         int i = 0;
-        for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
+        uint32_t chunk_iter = 0;
+        for (int t = unit; t < n_tiles; t += n_units, ++i) {
             const int buf = i & 1;
             const uint32_t aph = (i >> 1) & 1;
-            if (!mbar_wait(&acc_full[buf], aph, abort_flag)) break;
+            // all four epilogue warps take the same decision, so none is left
+            // behind at a named barrier if the wait gives up
+            const bool got = mbar_wait(&acc_full[buf], aph, abort_flag);
+            if (!named_bar_and(1, 128, got)) break;
             tc_fence_after();
-            const int a_row = (t % nA) * kTileA + lane_row;
+            const int a_cta0 = (t % nA) * tile_a_rows + static_cast<int>(rank) * kTileA;
+            const int a_row = a_cta0 + lane_row;
             const int b0 = (t / nA) * args.bn;
             const bool row_ok = a_row < args.rowsA;
             const float sa = row_ok ? __ldg(args.s_a + a_row) : 0.0f;
@@ -257,12 +314,78 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(t_row + c, r);
                 tmem_ld_wait();
-                if (row_ok) {
+                if (c + 32 >= args.bn) {  // last read of this accumulator: release it
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if constexpr (kPair == 2)
+                            mbar_arrive_cluster(buf == 0 ? acc_empty_leader
+                                                         : acc_empty_leader + sizeof(uint64_t));
+                        else
+                            mbar_arrive(&acc_empty[buf]);
+                    }
+                }
+                const int bc = b0 + c + lane;  // this lane's B row of the chunk
+                const float sb_lane = bc < args.rowsB ? __ldg(args.s_b + bc) : 0.0f;
+                if (args.tma_store) {
+                    uint8_t* sy = stage_y + (chunk_iter & 1) * C::kEpiBytes;
+                    if (issuer) bulk_wait_read<1>();  // the store of two chunks ago has read it
+                    named_bar_sync(1, 128);
+                    if (args.a_is_w) {
+                        // box [32 B rows][128 A rows]: element (u, lane_row)
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) {
+                            const float sb = __shfl_sync(0xffffffffu, sb_lane, u);
+                            const float acc = kInt8 ? __int2float_rn(static_cast<int32_t>(r[u]))
+                                                    : __uint_as_float(r[u]);
+                            const float v = __fmul_rn(__fmul_rn(acc, sb), sa);
+                            const int off = u * kTileA + lane_row;
+                            if constexpr (kOutBf16)
+                                reinterpret_cast<__nv_bfloat16*>(sy)[off] = __float2bfloat16_rn(v);
+                            else
+                                reinterpret_cast<float*>(sy)[off] = v;
+                        }
+                    } else {
+                        // box [128 A rows][32 B rows]: this lane's row is contiguous
+                        uint32_t packed[32 * kEsz / 4];
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) {
+                            const float sb = __shfl_sync(0xffffffffu, sb_lane, u);
+                            const float acc = kInt8 ? __int2float_rn(static_cast<int32_t>(r[u]))
+                                                    : __uint_as_float(r[u]);
+                            const float v = __fmul_rn(__fmul_rn(acc, sa), sb);
+                            if constexpr (kOutBf16) {
+                                const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+                                if (u & 1)
+                                    packed[u >> 1] |= h << 16;
+                                else
+                                    packed[u >> 1] = h;
+                            } else {
+                                packed[u] = __float_as_uint(v);
+                            }
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(sy + lane_row * 32 * kEsz);
+#pragma unroll
+                        for (int w = 0; w < 32 * kEsz / 16; ++w)
+                            dst[w] = make_uint4(packed[4 * w], packed[4 * w + 1], packed[4 * w + 2],
+                                                packed[4 * w + 3]);
+                    }
+                    fence_async_shared();
+                    named_bar_sync(1, 128);
+                    if (issuer) {
+                        if (args.a_is_w)
+                            tma_store_2d(&tm_y, sy, a_cta0, b0 + c);
+                        else
+                            tma_store_2d(&tm_y, sy, b0 + c, a_cta0);
+                        bulk_commit_group();
+                    }
+                    ++chunk_iter;
+                } else {
 #pragma unroll
                     for (int u = 0; u < 32; ++u) {
                         const int b_row = b0 + c + u;
-                        if (b_row < args.rowsB) {
-                            const float sb = __ldg(args.s_b + b_row);
+                        const float sb = __shfl_sync(0xffffffffu, sb_lane, u);
+                        if (row_ok && b_row < args.rowsB) {
                             if (args.a_is_w)
                                 store_scaled<kInt8, kOutBf16>(
                                     args.y, static_cast<int64_t>(b_row) * args.ldy + a_row, r[u],
@@ -275,17 +398,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
+        if (issuer) bulk_wait_all();  // Y stores done reading shared memory
     }
 
+    __syncwarp();
     tc_fence_before();
-    __syncthreads();
+    if constexpr (kPair == 2)
+        cluster_sync_all();  // both CTAs done with barriers and tensor memory
+    else
+        __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
+        tmem_dealloc_g<kPair>(tmem_base, kTmemCols);
     }
 }
 
