@@ -99,7 +99,7 @@ bool make_map_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t col
 // of Y are not 16-byte aligned.
 bool make_y_map(CUtensorMap* map, void* Y, int64_t M, int64_t N, bool out_bf16, bool a_is_w) {
     const uint32_t esz = out_bf16 ? 2 : 4;
-    if ((N * esz) % 16 != 0) return false;
+    if (!out_bf16 || (N * esz) % 16 != 0) return false;  // fp32 Y: direct stores
     const CUtensorMapDataType dt =
         out_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     return a_is_w ? make_map_2d(map, Y, M, N, 32, ss::kTileA, CU_TENSOR_MAP_SWIZZLE_NONE, dt, esz)
@@ -361,14 +361,16 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
     const int pair = rowsA > ss::kTileA ? 2 : 1;
     const int bn = choose_bn(rowsB, ss::GemmCfg<true, 1>::kBnMax);
     CUtensorMap ta, tb, te;
-    if (!make_map_2d(&ta, Av, rowsA, K_lp / 2, ss::kTileA, 64, CU_TENSOR_MAP_SWIZZLE_64B) ||
+    if (!make_map_2d(&ta, Av, rowsA, K_lp / 2, ss::kTileA, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&tb, B, rowsB, K_lp, bn / pair, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&te, Am, rowsA, K_lp / 8, ss::kTileA, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
         return SS_ERR_CUDA;
     ss::GemmArgs args;
     args.rowsA = static_cast<int>(rowsA);
     args.rowsB = static_cast<int>(rowsB);
-    args.k_stages = static_cast<int>(K_lp / 128);
+    // a last half stage (K_lp an odd multiple of 128) reads zeros past the rows
+    args.k_stages = static_cast<int>((K_lp + ss::GemmCfg<true, 1>::kStageK - 1) /
+                                     ss::GemmCfg<true, 1>::kStageK);
     args.bn = bn;
     args.a_is_w = sparse_operand == 0 ? 1 : 0;
     args.ldy = static_cast<int>(N);

@@ -48,35 +48,44 @@ constexpr int kTmemCols = 512;
 
 template <bool kSparse, int kPair>
 struct GemmCfg {
-    static constexpr int kStageK = 128;                    // logical K per stage
-    static constexpr int kMmaK = kSparse ? 64 : 32;        // logical K per MMA
-    static constexpr int kMmaPerStage = kStageK / kMmaK;   // 2 / 4
-    static constexpr int kARowBytes = kSparse ? 64 : 128;  // A bytes per row per stage
-    static constexpr int kABytes = kTileA * kARowBytes;
+    // One pipeline stage covers kStageK logical K: dense 128 (4 MMAs of K=32),
+    // sparse 256 (4 MMAs of K=64: A holds 128 compressed bytes per row, B two
+    // 128-byte swizzle atoms per row, metadata two 16-byte chunks per A row).
+    static constexpr int kStageK = kSparse ? 256 : 128;
+    static constexpr int kMmaK = kSparse ? 64 : 32;
+    static constexpr int kMmaPerStage = kStageK / kMmaK;   // 4
+    static constexpr int kARowBytes = kSparse ? kStageK / 2 : kStageK;  // 128
+    static constexpr int kABytes = kTileA * kARowBytes;    // 16 KB
+    static constexpr int kBAtoms = kStageK / 128;          // 128-byte K atoms of B per stage
     static constexpr int kBnMax = kSparse ? 224 : 256;     // MMA N; 2 accumulators (+ metadata)
     static constexpr int kBRowsMax = kBnMax / kPair;       // B rows held per CTA
-    static constexpr int kBBytes = kBRowsMax * 128;
-    static constexpr int kEBytes = kSparse ? kTileA * 16 : 0;
+    static constexpr int kBAtomBytes = kBRowsMax * 128;
+    static constexpr int kBBytes = kBAtoms * kBAtomBytes;
+    static constexpr int kEChunks = kSparse ? kStageK / 128 : 0;  // 16-byte metadata chunks/row
+    static constexpr int kEBytes = kEChunks * kTileA * 16;
     static constexpr int kStageRaw = kABytes + kBBytes + kEBytes;
     static constexpr int kStageBytes = (kStageRaw + 1023) / 1024 * 1024;
-    static constexpr int kEpiBytes = 32 * kTileA * 4;      // one 32-column chunk, fp32 worst case
-    static constexpr int kStagesRaw = (196 * 1024 - 2 * kEpiBytes) / kStageBytes;
+    static constexpr int kEpiBytes = 32 * kTileA * 2;      // one 32-column bf16 chunk of Y
+    static constexpr int kSmemBudget = 225 * 1024 - 1024 - 256 - 2 * kEpiBytes;
+    static constexpr int kStagesRaw = kSmemBudget / kStageBytes;
     static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
     static constexpr int kAccStride = kBnMax;              // TMEM columns between buffers
     static constexpr int kECol = 2 * kBnMax;               // metadata columns (sparse)
-    static constexpr int kESlots = 4;                      // 4 columns each
+    static constexpr int kESlotCols = 4 * kEChunks;        // 8 columns per stage
+    static constexpr int kESlots = 4;
     static constexpr int kEpiOffset = kStages * kStageBytes;  // 2 staging buffers for Y chunks
     static constexpr int kSmemBytes =
         kEpiOffset + 2 * kEpiBytes + 1024 /*align*/ + 256 /*barriers*/;
-    static_assert(kABytes % 1024 == 0 && (kABytes + kBBytes) % 1024 == 0, "tile alignment");
-    static_assert(!kSparse || kECol + kESlots * 4 <= kTmemCols, "TMEM budget");
+    static_assert(kABytes % 1024 == 0 && kBAtomBytes % 1024 == 0, "tile alignment");
+    static_assert(!kSparse || kECol + kESlots * kESlotCols <= kTmemCols, "TMEM budget");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+    static_assert(kStages >= (kPair == 2 ? 3 : 2), "pipeline depth");
 };
 
 struct GemmArgs {
     int rowsA;        // rows of A
     int rowsB;        // rows of B
-    int k_stages;     // K / 128
+    int k_stages;     // ceil(K / kStageK)
     int bn;           // B rows per tile (MMA N; multiple of 32 (x kPair), <= kBnMax)
     int a_is_w;       // 1: A rows are output channels (Y[b, a]); 0: Y[a, b]
     int ldy;          // leading dimension of Y (= N)
@@ -167,7 +176,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tma_prefetch_desc(&tm_a);
             tma_prefetch_desc(&tm_b);
             if (kSparse) tma_prefetch_desc(&tm_e);
-            const uint32_t tx = kPair * (C::kABytes + b_rows_cta * 128 + C::kEBytes);
+            const uint32_t tx =
+                kPair * (C::kABytes + C::kBAtoms * b_rows_cta * 128 + C::kEBytes);
             int s = 0;
             uint32_t ph = 0, armed = 0, armed_par = 0;
             bool ok = true;
@@ -180,20 +190,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         break;
                     }
                     uint8_t* st = smem + s * C::kStageBytes;
+                    uint8_t* st_b = st + C::kABytes;
+                    uint8_t* st_e = st_b + C::kBBytes;
                     if constexpr (kPair == 2) {
                         if (leader) mbar_arrive_expect_tx(&full[s], tx);
                         const uint32_t fb = map_to_rank(&full[s], 0);
                         tma_load_2d_pair(st, &tm_a, fb, kb * C::kARowBytes, a0);
-                        tma_load_2d_pair(st + C::kABytes, &tm_b, fb, kb * 128, b0);
-                        if (kSparse)
-                            tma_load_2d_pair(st + C::kABytes + C::kBBytes, &tm_e, fb, kb * 16, a0);
+#pragma unroll
+                        for (int u = 0; u < C::kBAtoms; ++u)
+                            tma_load_2d_pair(st_b + u * C::kBAtomBytes, &tm_b, fb,
+                                             kb * C::kStageK + u * 128, b0);
+#pragma unroll
+                        for (int u = 0; u < C::kEChunks; ++u)
+                            tma_load_2d_pair(st_e + u * kTileA * 16, &tm_e, fb,
+                                             kb * C::kEChunks * 16 + u * 16, a0);
                     } else {
                         mbar_arrive_expect_tx(&full[s], tx);
                         tma_load_2d(st, &tm_a, &full[s], kb * C::kARowBytes, a0);
-                        tma_load_2d(st + C::kABytes, &tm_b, &full[s], kb * 128, b0);
-                        if (kSparse)
-                            tma_load_2d(st + C::kABytes + C::kBBytes, &tm_e, &full[s], kb * 16,
-                                        a0);
+#pragma unroll
+                        for (int u = 0; u < C::kBAtoms; ++u)
+                            tma_load_2d(st_b + u * C::kBAtomBytes, &tm_b, &full[s],
+                                        kb * C::kStageK + u * 128, b0);
+#pragma unroll
+                        for (int u = 0; u < C::kEChunks; ++u)
+                            tma_load_2d(st_e + u * kTileA * 16, &tm_e, &full[s],
+                                        kb * C::kEChunks * 16 + u * 16, a0);
                     }
                     armed |= 1u << s;
                     armed_par = (armed_par & ~(1u << s)) | (ph << s);
@@ -216,8 +237,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // Descriptors are built once; a stage or K step only adds its byte
+        // offset (>> 4) to the start-address field.
         if (lane == 0 && leader) {
             const uint32_t idesc = make_idesc(kSparse, kInt8, kTileA * kPair, args.bn);
+            const uint32_t base = smem_u32(smem);
+            const uint64_t a_desc0 = smem_desc(base, 16, 1024, kSwizzle128B);
+            const uint64_t b_desc0 = smem_desc(base + C::kABytes, 16, 1024, kSwizzle128B);
+            const uint64_t e_desc0 =
+                smem_desc(base + C::kABytes + C::kBBytes, 128 * 16, 128, kSwizzleNone);
             int s = 0;
             uint32_t ph = 0;
             uint32_t e_iter = 0;
@@ -238,32 +266,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a_addr = smem_u32(smem + s * C::kStageBytes);
-                    const uint32_t b_addr = a_addr + C::kABytes;
-                    uint32_t e_tmem = 0;
+                    const uint64_t soff = static_cast<uint64_t>((s * C::kStageBytes) >> 4);
                     if constexpr (kSparse) {
-                        e_tmem = tmem_base + C::kECol + 4 * (e_iter % C::kESlots);
+                        const uint32_t e_tmem =
+                            tmem_base + C::kECol + C::kESlotCols * (e_iter & (C::kESlots - 1));
                         ++e_iter;
-                        const uint64_t e_desc =
-                            smem_desc(b_addr + C::kBBytes, 128 * 16, 128, kSwizzleNone);
-                        tc_cp_128x128b_g<kPair>(e_tmem, e_desc);
-                    }
 #pragma unroll
-                    for (int j = 0; j < C::kMmaPerStage; ++j) {
-                        const uint32_t acc = (kb > 0 || j > 0) ? 1u : 0u;
-                        if constexpr (kSparse) {
-                            const uint64_t a_desc =
-                                smem_desc(a_addr + j * 32, 16, 8 * 64, kSwizzle64B);
+                        for (int u = 0; u < C::kEChunks; ++u)
+                            tc_cp_128x128b_g<kPair>(e_tmem + 4 * u,
+                                                    e_desc0 + soff + ((u * kTileA * 16) >> 4));
+#pragma unroll
+                        for (int j = 0; j < C::kMmaPerStage; ++j) {
+                            const uint64_t a_desc = a_desc0 + soff + ((j * 32) >> 4);
                             const uint64_t b_desc =
-                                smem_desc(b_addr + j * 64, 16, 8 * 128, kSwizzle128B);
+                                b_desc0 + soff + (((j >> 1) * C::kBAtomBytes + (j & 1) * 64) >> 4);
                             mma_sparse_g<kPair, kInt8>(d_tmem, a_desc, b_desc, e_tmem + 2 * j,
-                                                       idesc, acc);
-                        } else {
-                            const uint64_t a_desc =
-                                smem_desc(a_addr + j * 32, 16, 8 * 128, kSwizzle128B);
-                            const uint64_t b_desc =
-                                smem_desc(b_addr + j * 32, 16, 8 * 128, kSwizzle128B);
-                            mma_dense_g<kPair, kInt8>(d_tmem, a_desc, b_desc, idesc, acc);
+                                                       idesc, (kb > 0 || j > 0) ? 1u : 0u);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < C::kMmaPerStage; ++j) {
+                            const uint64_t a_desc = a_desc0 + soff + ((j * 32) >> 4);
+                            const uint64_t b_desc = b_desc0 + soff + ((j * 32) >> 4);
+                            mma_dense_g<kPair, kInt8>(d_tmem, a_desc, b_desc, idesc,
+                                                      (kb > 0 || j > 0) ? 1u : 0u);
                         }
                     }
                     tc_commit_g<kPair>(&empty[s]);  // stage free in both CTAs once read
@@ -291,7 +317,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int lane_row = q * 32 + lane;
         const bool issuer = (warp == 2 && lane == 0);
         const uint32_t acc_empty_leader = kPair == 2 ? map_to_rank(acc_empty, 0) : 0u;
-        constexpr int kEsz = kOutBf16 ? 2 : 4;
+        constexpr int kEsz = 2;  // TMA-store staging is used for bf16 output only
         uint8_t* stage_y = smem + C::kEpiOffset;
         int i = 0;
         uint32_t chunk_iter = 0;
