@@ -361,7 +361,10 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
     const int pair = rowsA > ss::kTileA ? 2 : 1;
     const int bn = choose_bn(rowsB, ss::GemmCfg<true, 1>::kBnMax);
     CUtensorMap ta, tb, te;
-    if (!make_map_2d(&ta, Av, rowsA, K_lp / 2, ss::kTileA, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+    using CS = ss::GemmCfg<true, 1>;
+    if (!make_map_2d(&ta, Av, rowsA, K_lp / 2, ss::kTileA, CS::kARowBytes,
+                     CS::kARowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                           : CU_TENSOR_MAP_SWIZZLE_64B) ||
         !make_map_2d(&tb, B, rowsB, K_lp, bn / pair, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&te, Am, rowsA, K_lp / 8, ss::kTileA, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
         return SS_ERR_CUDA;

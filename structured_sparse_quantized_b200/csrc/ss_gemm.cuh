@@ -46,15 +46,23 @@ constexpr int kGemmThreads = 192;
 constexpr int kTileA = 128;  // A rows per CTA
 constexpr int kTmemCols = 512;
 
+// Logical K of one sparse pipeline stage: 256 (A rows of 128 compressed bytes
+// in 128B swizzle, two B atoms, two metadata chunks, four MMAs) or 128 (A rows
+// of 64 bytes in 64B swizzle, one B atom, one metadata chunk, two MMAs, and
+// twice as many stages in flight).
+#ifndef SS_SPARSE_STAGE_K
+#define SS_SPARSE_STAGE_K 256
+#endif
+
 template <bool kSparse, int kPair>
 struct GemmCfg {
     // One pipeline stage covers kStageK logical K: dense 128 (4 MMAs of K=32),
-    // sparse 256 (4 MMAs of K=64: A holds 128 compressed bytes per row, B two
-    // 128-byte swizzle atoms per row, metadata two 16-byte chunks per A row).
-    static constexpr int kStageK = kSparse ? 256 : 128;
+    // sparse SS_SPARSE_STAGE_K (MMAs of K=64).
+    static constexpr int kStageK = kSparse ? SS_SPARSE_STAGE_K : 128;
     static constexpr int kMmaK = kSparse ? 64 : 32;
-    static constexpr int kMmaPerStage = kStageK / kMmaK;   // 4
-    static constexpr int kARowBytes = kSparse ? kStageK / 2 : kStageK;  // 128
+    static constexpr int kMmaPerStage = kStageK / kMmaK;
+    static constexpr int kARowBytes = kSparse ? kStageK / 2 : kStageK;  // 64 or 128
+    static constexpr uint32_t kASwizzle = kARowBytes == 128 ? kSwizzle128B : kSwizzle64B;
     static constexpr int kABytes = kTileA * kARowBytes;    // 16 KB
     static constexpr int kBAtoms = kStageK / 128;          // 128-byte K atoms of B per stage
     static constexpr int kBnMax = kSparse ? 224 : 256;     // MMA N; 2 accumulators (+ metadata)
@@ -170,40 +178,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_base_slot;
 
+    // The producer and MMA roles run as whole, converged warps: every lane
+    // takes the barrier waits (the outcome is made warp-uniform) and one
+    // elected lane issues the TMA copies / tensor-core instructions.  A lone
+    // diverged lane issuing MMAs stalls on every memory operation and leaves
+    // the tensor pipe idle between stages.
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
+        if (elect_one()) {
             tma_prefetch_desc(&tm_a);
             tma_prefetch_desc(&tm_b);
             if (kSparse) tma_prefetch_desc(&tm_e);
-            const uint32_t tx =
-                kPair * (C::kABytes + C::kBAtoms * b_rows_cta * 128 + C::kEBytes);
-            int s = 0;
-            uint32_t ph = 0, armed = 0, armed_par = 0;
-            bool ok = true;
-            for (int t = unit; t < n_tiles && ok; t += n_units) {
-                const int a0 = (t % nA) * tile_a_rows + static_cast<int>(rank) * kTileA;
-                const int b0 = (t / nA) * args.bn + static_cast<int>(rank) * b_rows_cta;
-                for (int kb = 0; kb < args.k_stages; ++kb) {
-                    if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
+        }
+        __syncwarp();
+        const uint32_t tx =
+            kPair * (C::kABytes + C::kBAtoms * b_rows_cta * 128 + C::kEBytes);
+        int s = 0;
+        uint32_t ph = 0, armed = 0, armed_par = 0;
+        bool ok = true;
+        for (int t = unit; t < n_tiles && ok; t += n_units) {
+            const int a0 = (t % nA) * tile_a_rows + static_cast<int>(rank) * kTileA;
+            const int b0 = (t / nA) * args.bn + static_cast<int>(rank) * b_rows_cta;
+            for (int kb = 0; kb < args.k_stages; ++kb) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                if (elect_one()) {
                     uint8_t* st = smem + s * C::kStageBytes;
                     uint8_t* st_b = st + C::kABytes;
                     uint8_t* st_e = st_b + C::kBBytes;
                     if constexpr (kPair == 2) {
                         if (leader) mbar_arrive_expect_tx(&full[s], tx);
                         const uint32_t fb = map_to_rank(&full[s], 0);
-                        tma_load_2d_pair(st, &tm_a, fb, kb * C::kARowBytes, a0);
+                        const uint64_t keep = l2_policy_evict_last();
+                        tma_load_2d_pair_hint(st, &tm_a, fb, kb * C::kARowBytes, a0, keep);
 #pragma unroll
                         for (int u = 0; u < C::kBAtoms; ++u)
-                            tma_load_2d_pair(st_b + u * C::kBAtomBytes, &tm_b, fb,
-                                             kb * C::kStageK + u * 128, b0);
+                            tma_load_2d_pair_hint(st_b + u * C::kBAtomBytes, &tm_b, fb,
+                                                  kb * C::kStageK + u * 128, b0, keep);
 #pragma unroll
                         for (int u = 0; u < C::kEChunks; ++u)
-                            tma_load_2d_pair(st_e + u * kTileA * 16, &tm_e, fb,
-                                             kb * C::kEChunks * 16 + u * 16, a0);
+                            tma_load_2d_pair_hint(st_e + u * kTileA * 16, &tm_e, fb,
+                                                  kb * C::kEChunks * 16 + u * 16, a0, keep);
                     } else {
                         mbar_arrive_expect_tx(&full[s], tx);
                         tma_load_2d(st, &tm_a, &full[s], kb * C::kARowBytes, a0);
@@ -216,22 +233,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             tma_load_2d(st_e + u * kTileA * 16, &tm_e, &full[s],
                                         kb * C::kEChunks * 16 + u * 16, a0);
                     }
-                    armed |= 1u << s;
-                    armed_par = (armed_par & ~(1u << s)) | (ph << s);
-                    if (++s == C::kStages) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
+                }
+                __syncwarp();
+                armed |= 1u << s;
+                armed_par = (armed_par & ~(1u << s)) | (ph << s);
+                if (++s == C::kStages) {
+                    s = 0;
+                    ph ^= 1u;
                 }
             }
-            if (!ok) {  // let the copies already issued land before the CTA exits
-                if (kPair == 1 || leader) {
-                    for (int i = 0; i < C::kStages; ++i)
-                        if ((armed >> i) & 1u) mbar_drain(&full[i], (armed_par >> i) & 1u);
-                } else {  // the peer's copies count on the leader's barriers: wait 1 ms
-                    const uint64_t t0 = global_timer_ns();
-                    while (global_timer_ns() - t0 < 1000000ull) {
-                    }
+        }
+        if (!ok && lane == 0) {  // let the copies already issued land before exiting
+            if (kPair == 1 || leader) {
+                for (int i = 0; i < C::kStages; ++i)
+                    if ((armed >> i) & 1u) mbar_drain(&full[i], (armed_par >> i) & 1u);
+            } else {  // the peer's copies count on the leader's barriers: wait 1 ms
+                const uint64_t t0 = global_timer_ns();
+                while (global_timer_ns() - t0 < 1000000ull) {
                 }
             }
         }
@@ -239,10 +257,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // ------------------------------------------------------------ MMA issuer
         // Descriptors are built once; a stage or K step only adds its byte
         // offset (>> 4) to the start-address field.
-        if (lane == 0 && leader) {
+        if (leader) {
             const uint32_t idesc = make_idesc(kSparse, kInt8, kTileA * kPair, args.bn);
             const uint32_t base = smem_u32(smem);
-            const uint64_t a_desc0 = smem_desc(base, 16, 1024, kSwizzle128B);
+            const uint64_t a_desc0 = smem_desc(base, 16, 8 * C::kARowBytes, C::kASwizzle);
             const uint64_t b_desc0 = smem_desc(base + C::kABytes, 16, 1024, kSwizzle128B);
             const uint64_t e_desc0 =
                 smem_desc(base + C::kABytes + C::kBBytes, 128 * 16, 128, kSwizzleNone);
@@ -254,56 +272,64 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int t = unit; t < n_tiles && ok; t += n_units, ++i) {
                 const int buf = i & 1;
                 const uint32_t aph = (i >> 1) & 1;
-                if (!mbar_wait(&acc_empty[buf], aph ^ 1u, abort_flag)) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&acc_empty[buf], aph ^ 1u, abort_flag))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * C::kAccStride;
                 for (int kb = 0; kb < args.k_stages; ++kb) {
-                    if (!mbar_wait(&full[s], ph, abort_flag)) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t soff = static_cast<uint64_t>((s * C::kStageBytes) >> 4);
-                    if constexpr (kSparse) {
-                        const uint32_t e_tmem =
-                            tmem_base + C::kECol + C::kESlotCols * (e_iter & (C::kESlots - 1));
-                        ++e_iter;
+                    if (elect_one()) {
+                        const uint64_t soff = static_cast<uint64_t>((s * C::kStageBytes) >> 4);
+                        if constexpr (kSparse) {
+                            const uint32_t e_tmem =
+                                tmem_base + C::kECol + C::kESlotCols * (e_iter & (C::kESlots - 1));
 #pragma unroll
-                        for (int u = 0; u < C::kEChunks; ++u)
-                            tc_cp_128x128b_g<kPair>(e_tmem + 4 * u,
-                                                    e_desc0 + soff + ((u * kTileA * 16) >> 4));
+                            for (int u = 0; u < C::kEChunks; ++u)
+                                tc_cp_128x128b_g<kPair>(e_tmem + 4 * u,
+                                                        e_desc0 + soff + ((u * kTileA * 16) >> 4));
 #pragma unroll
-                        for (int j = 0; j < C::kMmaPerStage; ++j) {
-                            const uint64_t a_desc = a_desc0 + soff + ((j * 32) >> 4);
-                            const uint64_t b_desc =
-                                b_desc0 + soff + (((j >> 1) * C::kBAtomBytes + (j & 1) * 64) >> 4);
-                            mma_sparse_g<kPair, kInt8>(d_tmem, a_desc, b_desc, e_tmem + 2 * j,
-                                                       idesc, (kb > 0 || j > 0) ? 1u : 0u);
+                            for (int j = 0; j < C::kMmaPerStage; ++j) {
+                                const uint64_t a_desc = a_desc0 + soff + ((j * 32) >> 4);
+                                const uint64_t b_desc =
+                                    b_desc0 + soff +
+                                    (((j >> 1) * C::kBAtomBytes + (j & 1) * 64) >> 4);
+                                mma_sparse_g<kPair, kInt8>(d_tmem, a_desc, b_desc, e_tmem + 2 * j,
+                                                           idesc, (kb > 0 || j > 0) ? 1u : 0u);
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < C::kMmaPerStage; ++j) {
+                                const uint64_t a_desc = a_desc0 + soff + ((j * 32) >> 4);
+                                const uint64_t b_desc = b_desc0 + soff + ((j * 32) >> 4);
+                                mma_dense_g<kPair, kInt8>(d_tmem, a_desc, b_desc, idesc,
+                                                          (kb > 0 || j > 0) ? 1u : 0u);
+                            }
                         }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < C::kMmaPerStage; ++j) {
-                            const uint64_t a_desc = a_desc0 + soff + ((j * 32) >> 4);
-                            const uint64_t b_desc = b_desc0 + soff + ((j * 32) >> 4);
-                            mma_dense_g<kPair, kInt8>(d_tmem, a_desc, b_desc, idesc,
-                                                      (kb > 0 || j > 0) ? 1u : 0u);
-                        }
+                        tc_commit_g<kPair>(&empty[s]);  // stage free in both CTAs once read
                     }
-                    tc_commit_g<kPair>(&empty[s]);  // stage free in both CTAs once read
+                    __syncwarp();
+                    ++e_iter;
                     if (++s == C::kStages) {
                         s = 0;
                         ph ^= 1u;
                     }
                 }
                 if (!ok) break;
-                tc_commit_g<kPair>(&acc_full[buf]);
+                if (elect_one()) tc_commit_g<kPair>(&acc_full[buf]);
+                __syncwarp();
             }
             if (!ok) {  // wait for every MMA already issued before TMEM is freed
-                tc_commit_g<kPair>(drain);
-                mbar_drain(drain, 0);
+                if (elect_one()) {
+                    tc_commit_g<kPair>(drain);
+                    mbar_drain(drain, 0);
+                }
+                __syncwarp();
             }
         }
     } else {
@@ -399,10 +425,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     fence_async_shared();
                     named_bar_sync(1, 128);
                     if (issuer) {
+                        const uint64_t stream = l2_policy_evict_first();
                         if (args.a_is_w)
-                            tma_store_2d(&tm_y, sy, a_cta0, b0 + c);
+                            tma_store_2d_hint(&tm_y, sy, a_cta0, b0 + c, stream);
                         else
-                            tma_store_2d(&tm_y, sy, b0 + c, a_cta0);
+                            tma_store_2d_hint(&tm_y, sy, b0 + c, a_cta0, stream);
                         bulk_commit_group();
                     }
                     ++chunk_iter;
