@@ -102,15 +102,18 @@ bool make_y_map(CUtensorMap* map, void* Y, int64_t M, int64_t N, bool out_bf16, 
     if (!out_bf16 || (N * esz) % 16 != 0) return false;  // fp32 Y: direct stores
     const CUtensorMapDataType dt =
         out_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-    return a_is_w ? make_map_2d(map, Y, M, N, 32, ss::kTileA, CU_TENSOR_MAP_SWIZZLE_NONE, dt, esz)
+    // A rows = channels: one TMA store per 64-channel half of a chunk, staged
+    // [32 tokens][64 channels] with 128B swizzle; otherwise [128 tokens][32
+    // channels] unswizzled.
+    return a_is_w ? make_map_2d(map, Y, M, N, 32, 64, CU_TENSOR_MAP_SWIZZLE_128B, dt, esz)
                   : make_map_2d(map, Y, M, N, ss::kTileA, 32, CU_TENSOR_MAP_SWIZZLE_NONE, dt, esz);
 }
 
-template <bool kSparse, bool kInt8, bool kOutBf16, int kPair>
+template <bool kSparse, bool kInt8, bool kOutBf16, int kPair, int kAT>
 ss_status launch_gemm(int dev, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& e,
                       const CUtensorMap& y, const ss::GemmArgs& args, cudaStream_t stream) {
-    using C = ss::GemmCfg<kSparse, kPair>;
-    auto kern = ss::gemm_kernel<kSparse, kInt8, kOutBf16, kPair>;
+    using C = ss::GemmCfg<kSparse, kPair, kAT>;
+    auto kern = ss::gemm_kernel<kSparse, kInt8, kOutBf16, kPair, kAT>;
     static std::once_flag once[kMaxDevices];
     static cudaError_t attr_err[kMaxDevices];
     std::call_once(once[dev], [&] {
@@ -118,9 +121,9 @@ ss_status launch_gemm(int dev, const CUtensorMap& a, const CUtensorMap& b, const
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     });
     if (attr_err[dev] != cudaSuccess) return SS_ERR_CUDA;
+    const int64_t tile_rows = static_cast<int64_t>(ss::kTileA) * kPair * kAT;
     const int64_t tiles =
-        static_cast<int64_t>((args.rowsA + ss::kTileA * kPair - 1) / (ss::kTileA * kPair)) *
-        ((args.rowsB + args.bn - 1) / args.bn);
+        ((args.rowsA + tile_rows - 1) / tile_rows) * ((args.rowsB + args.bn - 1) / args.bn);
     const int64_t units = g_num_sms[dev] / kPair;
     const int grid = static_cast<int>((tiles < units ? tiles : units) * kPair);
     cudaLaunchConfig_t cfg = {};
@@ -142,15 +145,15 @@ ss_status launch_gemm(int dev, const CUtensorMap& a, const CUtensorMap& b, const
     return launched();
 }
 
-template <bool kSparse, int kPair>
+template <bool kSparse, int kPair, int kAT>
 ss_status dispatch_gemm(int dev, bool int8, bool bf16, const CUtensorMap& a, const CUtensorMap& b,
                         const CUtensorMap& e, const CUtensorMap& y, const ss::GemmArgs& args,
                         cudaStream_t st) {
     if (int8)
-        return bf16 ? launch_gemm<kSparse, true, true, kPair>(dev, a, b, e, y, args, st)
-                    : launch_gemm<kSparse, true, false, kPair>(dev, a, b, e, y, args, st);
-    return bf16 ? launch_gemm<kSparse, false, true, kPair>(dev, a, b, e, y, args, st)
-                : launch_gemm<kSparse, false, false, kPair>(dev, a, b, e, y, args, st);
+        return bf16 ? launch_gemm<kSparse, true, true, kPair, kAT>(dev, a, b, e, y, args, st)
+                    : launch_gemm<kSparse, true, false, kPair, kAT>(dev, a, b, e, y, args, st);
+    return bf16 ? launch_gemm<kSparse, false, true, kPair, kAT>(dev, a, b, e, y, args, st)
+                : launch_gemm<kSparse, false, false, kPair, kAT>(dev, a, b, e, y, args, st);
 }
 
 // B rows per tile: the whole of a small B, else the largest width <= max.
@@ -278,24 +281,41 @@ ss_status ss_quant_lift_act(const void* X, ss_in_dtype in_dtype, int64_t M, int6
     if (in_dtype != SS_IN_F32 && in_dtype != SS_IN_BF16) return SS_ERR_INVALID_ARG;
     if (q != SS_INT8 && q != SS_FP8_E4M3) return SS_ERR_INVALID_ARG;
     if (!aligned16(X) || !aligned16(Xq_lift) || !aligned16(s_x)) return SS_ERR_ALIGNMENT;
-    const size_t esz = in_dtype == SS_IN_BF16 ? 2 : 4;
-    const int64_t q_len = p.group <= 4 ? 0 : K_pad;  // byte row only for sliding patterns
-    const size_t smem = static_cast<size_t>((K * esz + 15) / 16 * 16 + round_up(q_len, 16) + 16);
+    // one warp per token row; sliding patterns keep a quantised byte row per
+    // warp in shared memory
+    const int q_stride = p.group <= 4 ? 0 : static_cast<int>(round_up(K_pad, 16));
+    int warps = ss::kWarpRowThreads / 32;
+    if (q_stride > 0)
+        while (warps > 1 && static_cast<size_t>(warps) * q_stride > kMaxRowSmem) warps /= 2;
+    const size_t smem = static_cast<size_t>(warps) * q_stride;
     if (smem > kMaxRowSmem) return SS_ERR_UNSUPPORTED;
     int dev;
     if ((st = check_device(&dev)) != SS_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int Nh = p.group / 2;
     uint8_t* xq = static_cast<uint8_t*>(Xq_lift);
+    const unsigned grid = static_cast<unsigned>((M + warps - 1) / warps);
 #define SS_QLIFT(T, I8)                                                                        \
     do {                                                                                      \
-        auto kern = ss::quant_lift_kernel<T, I8>;                                             \
+        auto kern = ss::quant_lift_warp_kernel<T, I8>;                                        \
         if ((st = set_smem(kern, dev, smem)) != SS_OK) return st;                             \
-        kern<<<static_cast<unsigned>(M), ss::kRowThreads, smem, s>>>(static_cast<const T*>(X), \
-                                                                      K, Nh, K_lift, K_lp, xq, \
-                                                                      s_x);                   \
+        kern<<<grid, warps * 32, smem, s>>>(static_cast<const T*>(X), M, K, Nh, K_lift, K_lp,  \
+                                            q_stride, xq, s_x);                               \
     } while (0)
-    if (in_dtype == SS_IN_BF16) {
+    // bf16 rows of up to 4096 elements (K % 16 == 0) are read once, into registers
+    const bool reg_path = in_dtype == SS_IN_BF16 && K % 16 == 0 && K <= ss::kRegK;
+    if (reg_path) {
+        const auto* xb = static_cast<const __nv_bfloat16*>(X);
+        if (q == SS_INT8) {
+            auto kern = ss::quant_lift_reg_kernel<true>;
+            if ((st = set_smem(kern, dev, smem)) != SS_OK) return st;
+            kern<<<grid, warps * 32, smem, s>>>(xb, M, K, Nh, K_lift, K_lp, q_stride, xq, s_x);
+        } else {
+            auto kern = ss::quant_lift_reg_kernel<false>;
+            if ((st = set_smem(kern, dev, smem)) != SS_OK) return st;
+            kern<<<grid, warps * 32, smem, s>>>(xb, M, K, Nh, K_lift, K_lp, q_stride, xq, s_x);
+        }
+    } else if (in_dtype == SS_IN_BF16) {
         if (q == SS_INT8) SS_QLIFT(__nv_bfloat16, true);
         else SS_QLIFT(__nv_bfloat16, false);
     } else {
@@ -316,20 +336,17 @@ ss_status ss_prune_act_2to4(const void* X, ss_in_dtype in_dtype, int64_t M, int6
     if (q != SS_INT8 && q != SS_FP8_E4M3) return SS_ERR_INVALID_ARG;
     if (!aligned16(X) || !aligned16(Xv) || !aligned16(Xm) || !aligned16(s_x))
         return SS_ERR_ALIGNMENT;
-    const size_t esz = in_dtype == SS_IN_BF16 ? 2 : 4;
-    const size_t smem = static_cast<size_t>((K * esz + 15) / 16 * 16 + 16);
-    if (smem > kMaxRowSmem) return SS_ERR_UNSUPPORTED;
     int dev;
     if ((st = check_device(&dev)) != SS_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* xv = static_cast<uint8_t*>(Xv);
     uint8_t* xm = static_cast<uint8_t*>(Xm);
+    const int warps = ss::kWarpRowThreads / 32;
+    const unsigned grid = static_cast<unsigned>((M + warps - 1) / warps);
 #define SS_PRUNE(T, I8)                                                                        \
     do {                                                                                      \
-        auto kern = ss::prune_act_kernel<T, I8>;                                              \
-        if ((st = set_smem(kern, dev, smem)) != SS_OK) return st;                             \
-        kern<<<static_cast<unsigned>(M), ss::kRowThreads, smem, s>>>(static_cast<const T*>(X), \
-                                                                      K, K_lp, xv, xm, s_x);  \
+        ss::prune_act_warp_kernel<T, I8><<<grid, ss::kWarpRowThreads, 0, s>>>(               \
+            static_cast<const T*>(X), M, K, K_lp, xv, xm, s_x);                               \
     } while (0)
     if (in_dtype == SS_IN_BF16) {
         if (q == SS_INT8) SS_PRUNE(__nv_bfloat16, true);
@@ -359,9 +376,9 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
     const int64_t rowsA = sparse_operand == 0 ? N : M;
     const int64_t rowsB = sparse_operand == 0 ? M : N;
     const int pair = rowsA > ss::kTileA ? 2 : 1;
-    const int bn = choose_bn(rowsB, ss::GemmCfg<true, 1>::kBnMax);
+    const int bn = choose_bn(rowsB, ss::GemmCfg<true, 1, 1>::kBnMax);
     CUtensorMap ta, tb, te;
-    using CS = ss::GemmCfg<true, 1>;
+    using CS = ss::GemmCfg<true, 1, 1>;
     if (!make_map_2d(&ta, Av, rowsA, K_lp / 2, ss::kTileA, CS::kARowBytes,
                      CS::kARowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                            : CU_TENSOR_MAP_SWIZZLE_64B) ||
@@ -372,8 +389,7 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
     args.rowsA = static_cast<int>(rowsA);
     args.rowsB = static_cast<int>(rowsB);
     // a last half stage (K_lp an odd multiple of 128) reads zeros past the rows
-    args.k_stages = static_cast<int>((K_lp + ss::GemmCfg<true, 1>::kStageK - 1) /
-                                     ss::GemmCfg<true, 1>::kStageK);
+    args.k_stages = static_cast<int>((K_lp + CS::kStageK - 1) / CS::kStageK);
     args.bn = bn;
     args.a_is_w = sparse_operand == 0 ? 1 : 0;
     args.ldy = static_cast<int>(N);
@@ -384,11 +400,9 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
     args.tma_store = make_y_map(&ty, Y, M, N, out_dtype == SS_OUT_BF16, args.a_is_w) ? 1 : 0;
     if (!args.tma_store) ty = ta;  // unused
     cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
-    return pair == 2
-               ? dispatch_gemm<true, 2>(dev, q == SS_INT8, out_dtype == SS_OUT_BF16, ta, tb, te,
-                                        ty, args, st_)
-               : dispatch_gemm<true, 1>(dev, q == SS_INT8, out_dtype == SS_OUT_BF16, ta, tb, te,
-                                        ty, args, st_);
+    const bool i8 = q == SS_INT8, bf = out_dtype == SS_OUT_BF16;
+    if (pair == 1) return dispatch_gemm<true, 1, 1>(dev, i8, bf, ta, tb, te, ty, args, st_);
+    return dispatch_gemm<true, 2, SS_SPARSE_A_TILES>(dev, i8, bf, ta, tb, te, ty, args, st_);
 }
 
 ss_status ss_dense_gemm(const void* Xq, const float* s_x, const void* Wq, const float* s_w,
@@ -405,7 +419,7 @@ ss_status ss_dense_gemm(const void* Xq, const float* s_x, const void* Wq, const 
     ss_status st = check_device(&dev);
     if (st != SS_OK) return st;
     const int pair = N > ss::kTileA ? 2 : 1;
-    const int bn = choose_bn(M, ss::GemmCfg<false, 1>::kBnMax);
+    const int bn = choose_bn(M, ss::GemmCfg<false, 1, 1>::kBnMax);
     CUtensorMap ta, tb;
     if (!make_map_2d(&ta, Wq, N, K_p, ss::kTileA, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&tb, Xq, M, K_p, bn / pair, 128, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -424,11 +438,9 @@ ss_status ss_dense_gemm(const void* Xq, const float* s_x, const void* Wq, const 
     args.tma_store = make_y_map(&ty, Y, M, N, out_dtype == SS_OUT_BF16, true) ? 1 : 0;
     if (!args.tma_store) ty = ta;  // unused
     cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
-    return pair == 2
-               ? dispatch_gemm<false, 2>(dev, q == SS_INT8, out_dtype == SS_OUT_BF16, ta, tb, ta,
-                                         ty, args, st_)
-               : dispatch_gemm<false, 1>(dev, q == SS_INT8, out_dtype == SS_OUT_BF16, ta, tb, ta,
-                                         ty, args, st_);
+    const bool i8 = q == SS_INT8, bf = out_dtype == SS_OUT_BF16;
+    return pair == 2 ? dispatch_gemm<false, 2, 1>(dev, i8, bf, ta, tb, ta, ty, args, st_)
+                     : dispatch_gemm<false, 1, 1>(dev, i8, bf, ta, tb, ta, ty, args, st_);
 }
 
 ss_status ss_get_device_status(ss_stream_t stream) {

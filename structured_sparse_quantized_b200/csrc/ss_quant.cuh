@@ -1,28 +1,26 @@
 // ss_quant.cuh -- memory-bound activation kernels.
 //
-//  quant_lift_kernel   fused per-token absmax, quantisation and activation
-//                      lifting (SlideSparse, 66bd.net: lifting is an index map
-//                      fused into the per-token quant kernel; SlideSparse
-//                      write-up, omica.com.cn, 3.2: one pass computes the
-//                      absmax, the scale, the clamped quantised values, the
-//                      window remap and the packed 32-bit stores, iterating
-//                      over output windows).
-//  prune_act_kernel    online 2:4 prune + compress of an activation ("add 2:4
-//                      or drop a precision tier?", paper-daily 2610.28947,
-//                      sections 1 and 2.3).
+//  quant_lift_warp_kernel  fused per-token absmax, quantisation and activation
+//                          lifting (SlideSparse, 66bd.net: lifting is an index
+//                          map fused into the per-token quant kernel;
+//                          SlideSparse write-up, omica.com.cn, 3.2: one kernel
+//                          computes the absmax, the scale, the clamped
+//                          quantised values, the window remap and the packed
+//                          stores, iterating over output windows).
+//  prune_act_warp_kernel   online 2:4 prune + compress of an activation ("add
+//                          2:4 or drop a precision tier?", paper-daily
+//                          2610.28947, sections 1 and 2.3).
 //
-// One CTA per token row.  The row is read from HBM once into shared memory
-// (16-byte loads), the absmax is reduced there, and the output is produced in
-// 16-byte stores: four lifted windows (or sixteen identity bytes) per store
-// for the lift, eight 2:4 groups (16 value bytes + one 32-bit nibble word)
-// per step for the prune.
+// One warp per token row, no block-wide barrier on the path: pass 1 streams
+// the row with 16-byte loads for its absmax, pass 2 streams it again (from
+// L2) and quantises; outputs leave in 16-byte stores -- four lifted windows
+// (or sixteen identity bytes) per store for the lift, eight 2:4 groups (16
+// value bytes + one 32-bit nibble word) per step for the prune.
 #pragma once
 
 #include "ss_common.cuh"
 
 namespace ss {
-
-constexpr int kRowThreads = 256;
 
 // Largest |v| over the eight values of a 16-byte chunk.
 template <typename T>
@@ -43,103 +41,15 @@ __device__ __forceinline__ float chunk_absmax<float>(const uint4& v) {
                  fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w))));
 }
 
-// Stage one row of X into shared memory as raw input elements and return the
-// row absmax (block-wide).  Rows are read once, 16 bytes per load.
-template <typename T>
-__device__ __forceinline__ float stage_row_absmax(const T* __restrict__ x, int64_t K64, T* srow,
-                                                  float* red) {
-    const int K = static_cast<int>(K64);
-    float a = 0.0f;
-    constexpr int kVec = 16 / sizeof(T);
-    const bool vec_ok = (K % kVec == 0) && ((reinterpret_cast<uintptr_t>(x) & 15) == 0);
-    if (vec_ok) {
-        const int nv = K / kVec;
-        const uint4* xv = reinterpret_cast<const uint4*>(x);
-        uint4* sv = reinterpret_cast<uint4*>(srow);
-        int i = threadIdx.x;
-        for (; i + 3 * static_cast<int>(blockDim.x) < nv; i += 4 * blockDim.x) {
-            uint4 v[4];  // four loads in flight per thread
-#pragma unroll
-            for (int u = 0; u < 4; ++u) v[u] = __ldcs(xv + i + u * blockDim.x);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                sv[i + u * blockDim.x] = v[u];
-                a = fmaxf(a, chunk_absmax<T>(v[u]));
-            }
-        }
-        for (; i < nv; i += blockDim.x) {
-            const uint4 v = __ldcs(xv + i);
-            sv[i] = v;
-            a = fmaxf(a, chunk_absmax<T>(v));
-        }
-    } else {
-        for (int i = threadIdx.x; i < K; i += blockDim.x) {
-            T v = x[i];
-            srow[i] = v;
-            a = fmaxf(a, fabsf(to_f32<T>(v)));
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane == 0) red[warp] = a;
-    __syncthreads();
-    if (warp == 0) {
-        a = lane < static_cast<int>(blockDim.x >> 5) ? red[lane] : 0.0f;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-        if (lane == 0) red[0] = a;
-    }
-    __syncthreads();
-    return red[0];
-}
-
-template <typename T>
-__device__ __forceinline__ float row_at(const T* srow, int64_t k, int64_t K) {
-    return k < K ? to_f32<T>(srow[k]) : 0.0f;
-}
-
-// Sixteen consecutive inputs of the staged row (zero past K) as floats.
-template <typename T>
-__device__ __forceinline__ void load16(const T* srow, int k0, int K, float (&f)[16]) {
-    if (k0 + 16 <= K) {
-        if constexpr (sizeof(T) == 2) {
-            const uint4* p = reinterpret_cast<const uint4*>(srow + k0);  // 16-byte aligned
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint4 v = p[h];
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    f[8 * h + 2 * j] = __uint_as_float(w[j] << 16);         // bf16 -> f32 (exact)
-                    f[8 * h + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-                }
-            }
-        } else {
-            const float4* p = reinterpret_cast<const float4*>(srow + k0);
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                const float4 v = p[h];
-                f[4 * h] = v.x;
-                f[4 * h + 1] = v.y;
-                f[4 * h + 2] = v.z;
-                f[4 * h + 3] = v.w;
-            }
-        }
-    } else {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) f[j] = (k0 + j < K) ? to_f32<T>(srow[k0 + j]) : 0.0f;
-    }
-}
-
 // INT8 code of x * inv as the low byte of a 32-bit word: the product is
-// rounded to fp32, clamped to [-127, 127], and rounded to the nearest integer
-// (ties to even) by adding 1.5 * 2^23, after which the integer sits in the
-// low mantissa bits.  This is the IEEE round-to-nearest-even of the fp32
-// product, without the low-throughput float-to-int conversion unit.
+// rounded to fp32 and then to the nearest integer (ties to even) by adding
+// 1.5 * 2^23, after which the integer sits in the low mantissa bits -- the
+// IEEE round-to-nearest-even of the fp32 product, without the low-throughput
+// float-to-int conversion unit.  No clamp is needed: |x| <= a and
+// inv = RN(127 / a) give |x * inv| <= 127 (1 + 2^-24), which rounds into
+// [-127, 127].
 __device__ __forceinline__ uint32_t int8_code(float x, float inv) {
-    const float p = fminf(fmaxf(__fmul_rn(x, inv), -127.0f), 127.0f);
-    return __float_as_uint(__fadd_rn(p, 12582912.0f));  // low byte = code
+    return __float_as_uint(__fadd_rn(__fmul_rn(x, inv), 12582912.0f));  // low byte = code
 }
 
 // Quantise sixteen values into sixteen bytes (byte j = value j).
@@ -163,76 +73,6 @@ __device__ __forceinline__ uint4 quant16(const float (&f)[16], float inv) {
         }
     }
     return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-// Xq[m, :] for pattern with half-group Nh (Nh = 0: dense identity map).
-// Pass 1 stages the row and reduces the absmax.  Identity maps (dense and
-// 2:4, whose single window per group is the group itself) then quantise
-// sixteen inputs into one 16-byte store each.  Sliding patterns quantise
-// every input once into a byte row in shared memory and build the lifted
-// windows from it: each window starts at an even position, so it is two
-// 16-bit shared loads, and four windows make one 16-byte store.
-template <typename T, bool kInt8>
-__global__ void __launch_bounds__(kRowThreads) quant_lift_kernel(
-    const T* __restrict__ X, int64_t K64, int Nh, int64_t K_lift64, int64_t K_lp64,
-    uint8_t* __restrict__ Xq, float* __restrict__ s_x) {
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    __shared__ float red[32];
-    const int K = static_cast<int>(K64);
-    const int K_lift = static_cast<int>(K_lift64);
-    const int K_lp = static_cast<int>(K_lp64);
-    T* srow = reinterpret_cast<T*>(smem_raw);
-    const int row_bytes = (K * static_cast<int>(sizeof(T)) + 15) / 16 * 16;
-    const int64_t m = blockIdx.x;
-    const float a = stage_row_absmax<T>(X + m * K64, K64, srow, red);
-    float inv, s;
-    scale_from_absmax<kInt8>(a, inv, s);
-    if (threadIdx.x == 0) s_x[m] = s;
-
-    uint4* out = reinterpret_cast<uint4*>(Xq + m * K_lp64);
-    const int n_chunks = K_lp / 16;  // 16 output bytes
-    if (Nh <= 2) {                   // identity map
-        for (int c = threadIdx.x; c < n_chunks; c += blockDim.x) {
-            float f[16];
-            load16<T>(srow, c * 16, K, f);
-            __stcs(out + c, quant16<kInt8>(f, inv));
-        }
-        return;
-    }
-    // quantised byte row covering K_pad = (K_lift / (4 (Nh-1))) * 2Nh positions
-    uint4* qrow = reinterpret_cast<uint4*>(smem_raw + row_bytes);
-    const int q_chunks = ((K_lift / (4 * (Nh - 1))) * 2 * Nh + 15) / 16;
-    for (int c = threadIdx.x; c < q_chunks; c += blockDim.x) {
-        float f[16];
-        load16<T>(srow, c * 16, K, f);
-        qrow[c] = quant16<kInt8>(f, inv);
-    }
-    __syncthreads();
-    const uint16_t* q16 = reinterpret_cast<const uint16_t*>(qrow);
-    const uint32_t n_win = static_cast<uint32_t>(K_lift / 4);
-    const uint32_t per_group = static_cast<uint32_t>(Nh - 1);
-    for (int c = threadIdx.x; c < n_chunks; c += blockDim.x) {
-        uint32_t win = static_cast<uint32_t>(c) * 4u;
-        uint32_t g = win / per_group;
-        uint32_t j = win - g * per_group;
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint32_t word = 0;
-            if (win < n_win) {
-                const uint32_t half = Nh * g + j;  // base / 2, base = 2Nh g + 2j
-                word = static_cast<uint32_t>(q16[half]) |
-                       (static_cast<uint32_t>(q16[half + 1]) << 16);
-            }
-            w[i] = word;  // byte t of the window at ascending address
-            ++win;
-            if (++j == per_group) {
-                j = 0;
-                ++g;
-            }
-        }
-        __stcs(out + c, make_uint4(w[0], w[1], w[2], w[3]));
-    }
 }
 
 // Keep the two largest |v| of a group of four (ties keep the lower index);
@@ -267,29 +107,176 @@ __device__ __forceinline__ uint32_t quantize_pair(float x0, float x1, float inv)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Warp-per-row kernels.  One warp owns one token row; no block-wide barrier
+// is on the path, so many rows are in flight per SM.  Pass 1 streams the row
+// (16-byte loads, four in flight per lane) for its absmax; pass 2 streams it
+// again -- the row was just read, so this comes from L2 -- and quantises.
+// ---------------------------------------------------------------------------
+constexpr int kWarpRowThreads = 256;  // 8 rows per CTA
+
+// Sixteen inputs at k0 straight from global memory (zero past K); `vec`
+// means the row is 16-byte aligned with K * sizeof(T) a multiple of 16.
+template <typename T>
+__device__ __forceinline__ void gload16(const T* __restrict__ x, int k0, int K, bool vec,
+                                        float (&f)[16]) {
+    if (vec && k0 + 16 <= K) {
+        if constexpr (sizeof(T) == 2) {
+            const uint4* p = reinterpret_cast<const uint4*>(x + k0);
+            const uint4 v0 = __ldg(p), v1 = __ldg(p + 1);
+            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                f[2 * j] = __uint_as_float(w[j] << 16);
+                f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+            }
+        } else {
+            const float4* p = reinterpret_cast<const float4*>(x + k0);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const float4 v = __ldg(p + h);
+                f[4 * h] = v.x;
+                f[4 * h + 1] = v.y;
+                f[4 * h + 2] = v.z;
+                f[4 * h + 3] = v.w;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) f[j] = (k0 + j < K) ? to_f32<T>(x[k0 + j]) : 0.0f;
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ float warp_row_absmax(const T* __restrict__ x, int K, bool vec,
+                                                 int lane) {
+    float a = 0.0f;
+    if (vec) {
+        constexpr int kVec = 16 / sizeof(T);
+        const int nv = K / kVec;
+        const uint4* xv = reinterpret_cast<const uint4*>(x);
+        int i = lane;
+        for (; i + 96 < nv; i += 128) {
+            const uint4 v0 = __ldg(xv + i), v1 = __ldg(xv + i + 32);
+            const uint4 v2 = __ldg(xv + i + 64), v3 = __ldg(xv + i + 96);
+            a = fmaxf(a, fmaxf(fmaxf(chunk_absmax<T>(v0), chunk_absmax<T>(v1)),
+                               fmaxf(chunk_absmax<T>(v2), chunk_absmax<T>(v3))));
+        }
+        for (; i < nv; i += 32) a = fmaxf(a, chunk_absmax<T>(__ldg(xv + i)));
+    } else {
+        for (int k = lane; k < K; k += 32) a = fmaxf(a, fabsf(to_f32<T>(x[k])));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    return a;
+}
+
 template <typename T, bool kInt8>
-__global__ void __launch_bounds__(kRowThreads) prune_act_kernel(
-    const T* __restrict__ X, int64_t K64, int64_t K_lp64, uint8_t* __restrict__ Xv,
-    uint8_t* __restrict__ Xm, float* __restrict__ s_x) {
+__global__ void __launch_bounds__(kWarpRowThreads) quant_lift_warp_kernel(
+    const T* __restrict__ X, int64_t M, int64_t K64, int Nh, int64_t K_lift64, int64_t K_lp64,
+    int q_stride, uint8_t* __restrict__ Xq, float* __restrict__ s_x) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    __shared__ float red[32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t m = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
+    if (m >= M) return;
     const int K = static_cast<int>(K64);
+    const int K_lift = static_cast<int>(K_lift64);
     const int K_lp = static_cast<int>(K_lp64);
-    T* srow = reinterpret_cast<T*>(smem_raw);
-    const int64_t m = blockIdx.x;
-    const float a = stage_row_absmax<T>(X + m * K64, K64, srow, red);
+    const T* x = X + m * K64;
+    const bool vec = (K * static_cast<int>(sizeof(T))) % 16 == 0 &&
+                     (reinterpret_cast<uintptr_t>(X) & 15) == 0;
+    const float a = warp_row_absmax<T>(x, K, vec, lane);
     float inv, s;
     scale_from_absmax<kInt8>(a, inv, s);
-    if (threadIdx.x == 0) s_x[m] = s;
+    if (lane == 0) s_x[m] = s;
+    uint4* out = reinterpret_cast<uint4*>(Xq + m * K_lp64);
+    const int n_chunks = K_lp / 16;  // 16 output bytes per chunk
+    if (Nh <= 2) {                   // identity map (dense, 2:4)
+        int c = lane;
+        for (; c + 32 < n_chunks; c += 64) {  // two chunks of loads in flight
+            float f0[16], f1[16];
+            gload16<T>(x, c * 16, K, vec, f0);
+            gload16<T>(x, (c + 32) * 16, K, vec, f1);
+            __stcs(out + c, quant16<kInt8>(f0, inv));
+            __stcs(out + c + 32, quant16<kInt8>(f1, inv));
+        }
+        if (c < n_chunks) {
+            float f[16];
+            gload16<T>(x, c * 16, K, vec, f);
+            __stcs(out + c, quant16<kInt8>(f, inv));
+        }
+        return;
+    }
+    // sliding patterns: quantised byte row of this warp, then window gather
+    uint4* qrow = reinterpret_cast<uint4*>(smem_raw + warp * q_stride);
+    const int q_chunks = ((K_lift / (4 * (Nh - 1))) * 2 * Nh + 15) / 16;
+    {
+        int c = lane;
+        for (; c + 32 < q_chunks; c += 64) {  // two chunks of loads in flight
+            float f0[16], f1[16];
+            gload16<T>(x, c * 16, K, vec, f0);
+            gload16<T>(x, (c + 32) * 16, K, vec, f1);
+            qrow[c] = quant16<kInt8>(f0, inv);
+            qrow[c + 32] = quant16<kInt8>(f1, inv);
+        }
+        if (c < q_chunks) {
+            float f[16];
+            gload16<T>(x, c * 16, K, vec, f);
+            qrow[c] = quant16<kInt8>(f, inv);
+        }
+    }
+    __syncwarp();
+    const uint16_t* q16 = reinterpret_cast<const uint16_t*>(qrow);
+    const uint32_t n_win = static_cast<uint32_t>(K_lift / 4);
+    const uint32_t per_group = static_cast<uint32_t>(Nh - 1);
+    for (int c = lane; c < n_chunks; c += 32) {
+        uint32_t win = static_cast<uint32_t>(c) * 4u;
+        uint32_t g = win / per_group;
+        uint32_t j = win - g * per_group;
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t word = 0;
+            if (win < n_win) {
+                const uint32_t half = Nh * g + j;  // base / 2, base = 2Nh g + 2j
+                word = static_cast<uint32_t>(q16[half]) |
+                       (static_cast<uint32_t>(q16[half + 1]) << 16);
+            }
+            w[i] = word;
+            ++win;
+            if (++j == per_group) {
+                j = 0;
+                ++g;
+            }
+        }
+        __stcs(out + c, make_uint4(w[0], w[1], w[2], w[3]));
+    }
+}
 
+template <typename T, bool kInt8>
+__global__ void __launch_bounds__(kWarpRowThreads) prune_act_warp_kernel(
+    const T* __restrict__ X, int64_t M, int64_t K64, int64_t K_lp64, uint8_t* __restrict__ Xv,
+    uint8_t* __restrict__ Xm, float* __restrict__ s_x) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t m = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
+    if (m >= M) return;
+    const int K = static_cast<int>(K64);
+    const int K_lp = static_cast<int>(K_lp64);
+    const T* x = X + m * K64;
+    const bool vec = (K * static_cast<int>(sizeof(T))) % 16 == 0 &&
+                     (reinterpret_cast<uintptr_t>(X) & 15) == 0;
+    const float a = warp_row_absmax<T>(x, K, vec, lane);
+    float inv, s;
+    scale_from_absmax<kInt8>(a, inv, s);
+    if (lane == 0) s_x[m] = s;
     // One step = 8 groups of 4 = 32 inputs -> 16 value bytes + 4 nibble bytes.
     uint4* vout = reinterpret_cast<uint4*>(Xv + m * (K_lp64 / 2));
     uint32_t* mout = reinterpret_cast<uint32_t*>(Xm + m * (K_lp64 / 8));
     const int n_steps = K_lp / 32;
-    for (int st = threadIdx.x; st < n_steps; st += blockDim.x) {
+    for (int st = lane; st < n_steps; st += 32) {
         float f[32];
-        load16<T>(srow, st * 32, K, *reinterpret_cast<float(*)[16]>(f));
-        load16<T>(srow, st * 32 + 16, K, *reinterpret_cast<float(*)[16]>(f + 16));
+        gload16<T>(x, st * 32, K, vec, *reinterpret_cast<float(*)[16]>(f));
+        gload16<T>(x, st * 32 + 16, K, vec, *reinterpret_cast<float(*)[16]>(f + 16));
         uint32_t vals[4];
         uint32_t nibs = 0;
 #pragma unroll
@@ -306,6 +293,111 @@ __global__ void __launch_bounds__(kRowThreads) prune_act_kernel(
         }
         __stcs(vout + st, make_uint4(vals[0], vals[1], vals[2], vals[3]));
         __stcs(mout + st, nibs);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Single-pass variants for bf16 rows of up to kRegK elements: the whole row
+// sits in registers (16 bytes x 2 x 8 per lane), so X is read from HBM once.
+// ---------------------------------------------------------------------------
+constexpr int kRegChunks = 8;                 // 16-element chunks per lane
+constexpr int kRegK = 32 * 16 * kRegChunks;   // 4096 elements
+
+__device__ __forceinline__ void bf16x16_to_f32(const uint4& a, const uint4& b, float (&f)[16]) {
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        f[2 * j] = __uint_as_float(w[j] << 16);
+        f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+}
+
+// Requires K % 16 == 0, K <= kRegK and a 16-byte aligned X.
+template <bool kInt8>
+__global__ void __launch_bounds__(kWarpRowThreads) quant_lift_reg_kernel(
+    const __nv_bfloat16* __restrict__ X, int64_t M, int64_t K64, int Nh, int64_t K_lift64,
+    int64_t K_lp64, int q_stride, uint8_t* __restrict__ Xq, float* __restrict__ s_x) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t m = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
+    if (m >= M) return;
+    const int K = static_cast<int>(K64);
+    const int K_lift = static_cast<int>(K_lift64);
+    const int K_lp = static_cast<int>(K_lp64);
+    const uint4* xv = reinterpret_cast<const uint4*>(X + m * K64);
+    const int n16 = K / 16;
+    uint4 v[2 * kRegChunks];
+#pragma unroll
+    for (int i = 0; i < kRegChunks; ++i) {
+        const int c = lane + 32 * i;
+        if (c < n16) {
+            v[2 * i] = __ldcs(xv + 2 * c);
+            v[2 * i + 1] = __ldcs(xv + 2 * c + 1);
+        } else {
+            v[2 * i] = make_uint4(0, 0, 0, 0);
+            v[2 * i + 1] = make_uint4(0, 0, 0, 0);
+        }
+    }
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 2 * kRegChunks; ++i) a = fmaxf(a, chunk_absmax<__nv_bfloat16>(v[i]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    float inv, s;
+    scale_from_absmax<kInt8>(a, inv, s);
+    if (lane == 0) s_x[m] = s;
+    uint4* out = reinterpret_cast<uint4*>(Xq + m * K_lp64);
+    const int n_chunks = K_lp / 16;
+    if (Nh <= 2) {  // identity map: chunk c of the output is chunk c of the input
+#pragma unroll
+        for (int i = 0; i < kRegChunks; ++i) {
+            const int c = lane + 32 * i;
+            if (c < n16) {
+                float f[16];
+                bf16x16_to_f32(v[2 * i], v[2 * i + 1], f);
+                __stcs(out + c, quant16<kInt8>(f, inv));
+            }
+        }
+        for (int c = n16 + lane; c < n_chunks; c += 32) __stcs(out + c, make_uint4(0, 0, 0, 0));
+        return;
+    }
+    uint4* qrow = reinterpret_cast<uint4*>(smem_raw + warp * q_stride);
+    const int q_chunks = ((K_lift / (4 * (Nh - 1))) * 2 * Nh + 15) / 16;
+#pragma unroll
+    for (int i = 0; i < kRegChunks; ++i) {
+        const int c = lane + 32 * i;
+        if (c < n16) {
+            float f[16];
+            bf16x16_to_f32(v[2 * i], v[2 * i + 1], f);
+            qrow[c] = quant16<kInt8>(f, inv);
+        }
+    }
+    for (int c = n16 + lane; c < q_chunks; c += 32) qrow[c] = make_uint4(0, 0, 0, 0);
+    __syncwarp();
+    const uint16_t* q16 = reinterpret_cast<const uint16_t*>(qrow);
+    const uint32_t n_win = static_cast<uint32_t>(K_lift / 4);
+    const uint32_t per_group = static_cast<uint32_t>(Nh - 1);
+    for (int c = lane; c < n_chunks; c += 32) {
+        uint32_t win = static_cast<uint32_t>(c) * 4u;
+        uint32_t g = win / per_group;
+        uint32_t j = win - g * per_group;
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t word = 0;
+            if (win < n_win) {
+                const uint32_t half = Nh * g + j;  // base / 2, base = 2Nh g + 2j
+                word = static_cast<uint32_t>(q16[half]) |
+                       (static_cast<uint32_t>(q16[half + 1]) << 16);
+            }
+            w[i] = word;
+            ++win;
+            if (++j == per_group) {
+                j = 0;
+                ++g;
+            }
+        }
+        __stcs(out + c, make_uint4(w[0], w[1], w[2], w[3]));
     }
 }
 
