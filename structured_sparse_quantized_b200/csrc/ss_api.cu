@@ -13,6 +13,7 @@
 #include "ss_common.cuh"
 #include "ss_compress.cuh"
 #include "ss_gemm.cuh"
+#include "ss_gemm_wide.cuh"
 #include "ss_quant.cuh"
 
 namespace {
@@ -154,6 +155,63 @@ ss_status dispatch_gemm(int dev, bool int8, bool bf16, const CUtensorMap& a, con
                     : launch_gemm<kSparse, true, false, kPair, kAT>(dev, a, b, e, y, args, st);
     return bf16 ? launch_gemm<kSparse, false, true, kPair, kAT>(dev, a, b, e, y, args, st)
                 : launch_gemm<kSparse, false, false, kPair, kAT>(dev, a, b, e, y, args, st);
+}
+
+template <bool kInt8>
+ss_status launch_gemm_wide(int dev, const CUtensorMap& a, const CUtensorMap& b,
+                           const CUtensorMap& e, const CUtensorMap& y, const ss::GemmArgs& args,
+                           cudaStream_t stream) {
+    using C = ss::WideCfg;
+    auto kern = ss::gemm_sparse_wide_kernel<kInt8>;
+    static std::once_flag once[kMaxDevices];
+    static cudaError_t attr_err[kMaxDevices];
+    std::call_once(once[dev], [&] {
+        attr_err[dev] =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    });
+    if (attr_err[dev] != cudaSuccess) return SS_ERR_CUDA;
+    const int64_t tile_b = static_cast<int64_t>(ss::kWideBT) * args.bn;
+    const int64_t tiles = ((args.rowsA + 2 * ss::kTileA - 1) / (2 * ss::kTileA)) *
+                          ((args.rowsB + tile_b - 1) / tile_b);
+    const int64_t units = g_num_sms[dev] / 2;
+    const int grid = static_cast<int>((tiles < units ? tiles : units) * 2);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(ss::kWideThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, a, b, e, y, args) != cudaSuccess) {
+        cudaGetLastError();
+        return SS_ERR_CUDA;
+    }
+    return launched();
+}
+
+// B-tile width of the wide sparse GEMM: the multiple of 32 (<= 224) that
+// minimises waves x per-tile time, the per-tile time taken as proportional to
+// the bytes a K step brings into each SM (A and metadata 5 KB shared by the
+// two B tiles, plus 32 bytes per B row), which is what bounds the mainloop.
+int choose_bn_wide(int64_t rowsA, int64_t rowsB, int units) {
+    const int64_t nA = (rowsA + 2 * ss::kTileA - 1) / (2 * ss::kTileA);
+    int best = ss::WideCfg::kBnMax;
+    double best_cost = 0.0;
+    for (int bn = ss::WideCfg::kBnMax; bn >= 64; bn -= 32) {
+        const int64_t tiles = nA * ((rowsB + 2 * bn - 1) / (2 * bn));
+        const int64_t waves = (tiles + units - 1) / units;
+        const double cost = static_cast<double>(waves) * (5120.0 / 2 + 32.0 * bn);
+        if (bn == ss::WideCfg::kBnMax || cost < best_cost * 0.999) {
+            best = bn;
+            best_cost = cost;
+        }
+    }
+    return best;
 }
 
 // B rows per tile: the whole of a small B, else the largest width <= max.
@@ -401,6 +459,23 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
     if (!args.tma_store) ty = ta;  // unused
     cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
     const bool i8 = q == SS_INT8, bf = out_dtype == SS_OUT_BF16;
+#if SS_SPARSE_WIDE
+    // Large problems with channel rows and bf16 Y: two B tiles per output tile.
+    if (pair == 2 && args.a_is_w && args.tma_store && rowsB > 2 * ss::WideCfg::kBnMax) {
+        using CW = ss::WideCfg;
+        const int bnw = choose_bn_wide(rowsA, rowsB, g_num_sms[dev] / 2);
+        CUtensorMap wa, wb;
+        if (!make_map_2d(&wa, Av, rowsA, K_lp / 2, ss::kTileA, CW::kARowBytes,
+                         CU_TENSOR_MAP_SWIZZLE_64B) ||
+            !make_map_2d(&wb, B, rowsB, K_lp, bnw / 2, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+            return SS_ERR_CUDA;
+        ss::GemmArgs wargs = args;
+        wargs.bn = bnw;
+        wargs.k_stages = static_cast<int>(K_lp / CW::kStageK);
+        return i8 ? launch_gemm_wide<true>(dev, wa, wb, te, ty, wargs, st_)
+                  : launch_gemm_wide<false>(dev, wa, wb, te, ty, wargs, st_);
+    }
+#endif
     if (pair == 1) return dispatch_gemm<true, 1, 1>(dev, i8, bf, ta, tb, te, ty, args, st_);
     return dispatch_gemm<true, 2, SS_SPARSE_A_TILES>(dev, i8, bf, ta, tb, te, ty, args, st_);
 }

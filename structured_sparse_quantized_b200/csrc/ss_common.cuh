@@ -473,6 +473,41 @@ __device__ __forceinline__ void mma_sparse_g(uint32_t d_tmem, uint64_t a_desc, u
     }
 }
 
+// Two fp32 products in one instruction (mul.rn.f32x2): (a0 * b0, a1 * b1),
+// each rounded to nearest even as __fmul_rn would.
+__device__ __forceinline__ void mul_rn_f32x2(float a0, float a1, float b0, float b1, float& r0,
+                                             float& r1) {
+    uint64_t a, b, r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b0), "f"(b1));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r0), "=f"(r1) : "l"(r));
+}
+
+// Pair sparse MMA that keeps its A operand in the tensor core's collector
+// buffer: kUse = 0 reads A from shared memory and keeps it (fill), kUse = 1
+// takes A from the collector and releases it (lastuse).  Two MMAs that share
+// one A tile then read it from shared memory once.
+template <bool kInt8, int kUse>
+__device__ __forceinline__ void mma_sparse_pair_coll(uint32_t d_tmem, uint64_t a_desc,
+                                                     uint64_t b_desc, uint32_t e_tmem,
+                                                     uint32_t idesc, uint32_t accumulate) {
+#define SS_MMA_SP_COLL(KIND, USE)                                                             \
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %5, 0;\n\t"                         \
+                 "tcgen05.mma.sp.cta_group::2.kind::" KIND ".collector::a::" USE             \
+                 " [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),                          \
+                 "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)          \
+                 : "memory")
+    if constexpr (kInt8) {
+        if constexpr (kUse == 0) SS_MMA_SP_COLL("i8", "fill");
+        else SS_MMA_SP_COLL("i8", "lastuse");
+    } else {
+        if constexpr (kUse == 0) SS_MMA_SP_COLL("f8f6f4", "fill");
+        else SS_MMA_SP_COLL("f8f6f4", "lastuse");
+    }
+#undef SS_MMA_SP_COLL
+}
+
 template <int kPair>
 __device__ __forceinline__ void tc_cp_128x128b_g(uint32_t taddr, uint64_t src_desc) {
     if constexpr (kPair == 2)

@@ -111,6 +111,36 @@ def test_sparse_gemm_weight_sparse(M, N, K, pat, q, out):
     assert_y_matches(host(Y), Y_ref, q, ob)
 
 
+# Shapes with more than two 224-token tiles and more than 128 channels take
+# the two-B-tile kernel (single-buffered accumulators, collector-reused A):
+# several tiles per CTA pair, ragged channels and tokens, odd stage counts and
+# the narrower B tiles the wave balancing picks.
+WIDE_CASES = [  # M, N, K, pattern, sampled token rows (None = all)
+    (1000, 520, 1024, "2:4", None),    # ragged both ways, 8 stages
+    (2000, 300, 768, "6:8", None),     # 9 stages (odd against the 5-stage ring)
+    (4500, 1100, 640, "4:6", None),    # 192-token B tiles, ragged channel tile
+    (8192, 2048, 256, "2:4", 384),     # 160-token B tiles, 3 tiles per pair
+    (3000, 4096, 512, "8:10", 256),    # 16 channel tiles, 2 tiles per pair
+    (8192, 14336, 128, "2:4", 256),    # full 224-token B tiles, one stage, 15 waves
+]
+
+
+@pytest.mark.parametrize("M,N,K,pat,nrows", WIDE_CASES)
+@pytest.mark.parametrize("q", ["int8", "fp8"])
+def test_sparse_gemm_wide_tiles(M, N, K, pat, nrows, q):
+    W = synth.gaussian((N, K), std=0.02, seed=0, dtype=torch.bfloat16)
+    X = synth.gaussian((M, K), std=1.0, seed=1, dtype=torch.bfloat16)
+    Wv, Wm, s_w = oracle.compress_weight(W, pat, Q[q])
+    Xq, s_x = oracle.quant_lift_act(X, pat, Q[q])
+    _, _, K_lp = oracle.slide_shape(pat, K)
+    rows = None if nrows is None else synth.sample_rows(M, seed=5, middle=nrows)
+    Y_ref = oracle.sparse_gemm(0, Wv, Wm, s_w, Xq, s_x, M, N, K_lp, Q[q], oracle.OUT_BF16,
+                               m_idx=rows)
+    Y = host(ss.sparse_gemm(0, dev(Wv), dev(Wm), dev(s_w), dev(Xq), dev(s_x), M, N, q))
+    assert ss.ss_get_device_status() == ss.SS_OK
+    assert_y_matches(Y if rows is None else Y[rows], Y_ref, q, True)
+
+
 @pytest.mark.parametrize("M,N,K", [(130, 64, 256), (257, 300, 1024), (8, 96, 4096)])
 @pytest.mark.parametrize("q", ["int8", "fp8"])
 def test_sparse_gemm_activation_sparse(M, N, K, q):
