@@ -46,9 +46,12 @@ ALSO_WORKLOAD = ("qwen_gateup_6of8_fp8", 8192)  # the SlideSparse 6:8 headline s
 FLUSH_BYTES = 256 << 20
 IDEAL = {"2:4": 2.0, "4:6": 1.5, "6:8": 4.0 / 3.0, "8:10": 1.25}
 
-# DRAM bytes per launch of the dominant kernel from an ncu capture of the
-# same kernel build (profiles/); None when not captured for this build.
-TRAFFIC = {}
+# DRAM bytes per launch of the dominant kernel (dram__bytes_read.sum +
+# dram__bytes_write.sum of one sparse-GEMM launch) from one ncu capture of the
+# same kernel build; absent when not captured for this build.
+TRAFFIC = {
+    ("llama_q_2of4_int8", 8192): 44.19e6 + 17.82e6,
+}
 
 
 def load_peaks():
@@ -106,7 +109,7 @@ class ClockSampler:
     REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40,
                "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
 
-    def __init__(self, index: int, period_s: float = 0.02):
+    def __init__(self, index: int, period_s: float = 0.002):
         self.samples, self.reasons, self.ok = [], set(), False
         self.max_mhz = None
         try:
@@ -415,7 +418,7 @@ def run_reference(args, dist: Dist):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ss", choices=["ss", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))

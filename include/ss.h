@@ -72,6 +72,16 @@ ss_status ss_slide_shape(ss_pattern p, int64_t K, int64_t *K_pad, int64_t *K_lif
 /* K_lp of an online-pruned 2:4 activation: K rounded up to 4, then to 128. */
 ss_status ss_act_2to4_shape(int64_t K, int64_t *K_lp);
 
+/* Size in bytes of a metadata buffer (Wm, Xm) for `rows` rows of K_lp
+ * lifted elements.  Metadata is stored tile-major so that the 2:4 selectors
+ * of 128 rows x 128 K (the unit the GEMM stages) are one contiguous 2 KB
+ * block, which the tensor-memory copy takes as is:
+ *   byte b of row r (its nibbles as in the row layout [rows, K_lp/8]) is at
+ *   ((r / 128) * (K_lp / 128) + b / 16) * 2048 + (r % 128) * 16 + b % 16.
+ * Rows are padded to a multiple of 128; padding rows are zero.
+ * Returns 0 for rows < 1 or K_lp not a positive multiple of 128. */
+int64_t ss_meta_bytes(int64_t rows, int64_t K_lp);
+
 /* Offline weight compression (SlideSparse write-up, omica.com.cn, 2.2 weight
  * preprocessing and 3.1; LLM-Compressor W8A8 rows: channel-wise weights).
  * Per row of W[N, K] (f32 or bf16):
@@ -86,7 +96,8 @@ ss_status ss_act_2to4_shape(int64_t K, int64_t *K_lp);
  *      idx0 | idx1 << 2.
  * Outputs (pattern != dense):
  *   Wv  [N, K_lp/2] bytes   stored values, window w at bytes 2w, 2w+1
- *   Wm  [N, K_lp/8] bytes   nibbles, window w in byte w/2, low nibble = even w
+ *   Wm  ss_meta_bytes(N, K_lp) bytes, tile-major (see ss_meta_bytes): row n's
+ *       nibbles, window w in its byte w/2, low nibble = even w
  *   s_w [N] fp32
  * Dense: Wv is [N, K_lp] (per-channel quantised W, zero padded), Wm unused
  * (may be NULL).  A NaN/Inf weight sets SS_ERR_DATA in the device status. */
@@ -110,21 +121,25 @@ ss_status ss_quant_lift_act(const void *X, ss_in_dtype in_dtype, int64_t M, int6
  * the fly must be pruned and compressed before every matmul).  Per token m:
  * in each group of 4 along K keep the two largest |x| (ties keep the lower
  * index), s_x[m] = row absmax / Q, quantise the kept values, pack as in
- * ss_compress_weight.  Outputs Xv [M, K_lp/2], Xm [M, K_lp/8], s_x [M] with
- * K_lp from ss_act_2to4_shape(). */
+ * ss_compress_weight.  Outputs Xv [M, K_lp/2], Xm (ss_meta_bytes(M, K_lp)
+ * bytes, tile-major), s_x [M] with K_lp from ss_act_2to4_shape(). */
 ss_status ss_prune_act_2to4(const void *X, ss_in_dtype in_dtype, int64_t M, int64_t K,
                             ss_qdtype q, void *Xv, void *Xm, float *s_x, ss_stream_t stream);
 
 /* Sparse GEMM on the sm_100a sparse tensor cores (tcgen05.mma.sp, TMEM
  * accumulators, TMA-staged tiles), with the dequant epilogue
  *   Y[m, n] = ((float)acc[m, n] * s_x[m]) * s_w[n]   (fp32, then bf16 RNE)
- * sparse_operand = 0: A = weight.  Av = Wv [N, K_lp/2], Am = Wm [N, K_lp/8],
+ * sparse_operand = 0: A = weight.  Av = Wv [N, K_lp/2], Am = Wm (tile-major),
  *                     s_a = s_w [N]; B = Xq_lift [M, K_lp], s_b = s_x [M].
  * sparse_operand = 1: A = activation.  Av = Xv [M, K_lp/2], Am = Xm
- *                     [M, K_lp/8], s_a = s_x [M]; B = Wq [N, K_lp] (dense),
+ *                     (tile-major), s_a = s_x [M]; B = Wq [N, K_lp] (dense),
  *                     s_b = s_w [N].
  * acc is exact int32 for INT8 and fp32 (tensor-core accumulation) for E4M3.
- * K_lp must be a positive multiple of 128; M, N in [1, 2^31). */
+ * K_lp must be a positive multiple of 128; M, N in [1, 2^31).
+ * Kernel shape: with more than 128 weight rows and bf16 Y, large problems
+ * run output tiles of 256 channels x 2 token tiles (one A slice feeds two
+ * MMAs), the rest 256 x 1.  The choice follows the wave count; the
+ * environment variable SS_SPARSE_KERNEL=narrow|wide pins it (same results). */
 ss_status ss_sparse_gemm(int sparse_operand, const void *Av, const void *Am, const float *s_a,
                          const void *B, const float *s_b, int64_t M, int64_t N, int64_t K_lp,
                          ss_qdtype q, void *Y, ss_out_dtype out_dtype, ss_stream_t stream);

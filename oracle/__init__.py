@@ -302,3 +302,29 @@ def plain_linear(W, X, p: str, qdtype: int, out_dtype: int, m_idx=None):
 
 def bf16_bits_to_float(y: np.ndarray) -> np.ndarray:
     return (np.asarray(y, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+# ------------------------------------------------------------------ storage layout
+
+def meta_to_tiles(Am: np.ndarray, K_lp: int) -> np.ndarray:
+    """Row-layout selectors [rows, K_lp/8] -> the library's tile-major storage
+    [ceil(rows/128), K_lp/128, 128, 16]: block (row tile, K tile) holds the 16
+    selector bytes of 128 lifted K for each of the tile's 128 rows; padding
+    rows are zero.  A pure relabelling of bytes (no arithmetic), used to hand
+    oracle metadata to the GPU and to compare the GPU's metadata with it."""
+    Am = np.ascontiguousarray(Am, dtype=np.uint8)
+    rows, nb = Am.shape
+    assert nb == K_lp // 8 and K_lp % 128 == 0
+    rt = (rows + 127) // 128
+    padded = np.zeros((rt * 128, nb), dtype=np.uint8)
+    padded[:rows] = Am
+    # [row tile, row in tile, K tile, byte in K tile] -> [row tile, K tile, row, byte]
+    return np.ascontiguousarray(padded.reshape(rt, 128, K_lp // 128, 16).transpose(0, 2, 1, 3))
+
+
+def meta_from_tiles(At: np.ndarray, rows: int, K_lp: int) -> np.ndarray:
+    """Inverse of meta_to_tiles: tile-major storage -> [rows, K_lp/8]."""
+    At = np.ascontiguousarray(At, dtype=np.uint8)
+    rt = (rows + 127) // 128
+    At = At.reshape(rt, K_lp // 128, 128, 16)
+    return np.ascontiguousarray(At.transpose(0, 2, 1, 3).reshape(rt * 128, K_lp // 8)[:rows])

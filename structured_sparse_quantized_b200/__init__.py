@@ -88,6 +88,8 @@ def lib() -> ctypes.CDLL:
     L.ss_status_string.restype = ctypes.c_char_p
     L.ss_kernel_launches.argtypes = []
     L.ss_kernel_launches.restype = i64
+    L.ss_meta_bytes.argtypes = [i64, i64]
+    L.ss_meta_bytes.restype = i64
     del f
     _lib = L
     return L
@@ -174,6 +176,16 @@ def ss_act_2to4_shape(K: int) -> int:
     return a.value
 
 
+def ss_meta_bytes(rows: int, K_lp: int) -> int:
+    return int(lib().ss_meta_bytes(int(rows), int(K_lp)))
+
+
+def meta_shape(rows: int, K_lp: int) -> tuple:
+    """Shape of a tile-major metadata buffer: [row tiles, K tiles, 128, 16]
+    (one 2 KB block of 2:4 selectors per 128 rows x 128 lifted K)."""
+    return ((rows + 127) // 128, K_lp // 128, 128, 16)
+
+
 def ss_compress_weight(W, pattern, q, Wv, Wm, s_w, stream=None) -> None:
     N, K = W.shape
     _check(lib().ss_compress_weight(_dev(W, "W"), _in_dtype(W), N, K, _pattern(pattern),
@@ -226,7 +238,7 @@ def compress_weight(W: torch.Tensor, pattern, q, stream=None):
         Wm = None
     else:
         Wv = torch.empty((N, K_lp // 2), dtype=torch.uint8, device=dev)
-        Wm = torch.empty((N, K_lp // 8), dtype=torch.uint8, device=dev)
+        Wm = torch.empty(meta_shape(N, K_lp), dtype=torch.uint8, device=dev)
     s_w = torch.empty(N, dtype=torch.float32, device=dev)
     ss_compress_weight(W, p, q, Wv, Wm, s_w, stream)
     return Wv, Wm, s_w
@@ -248,7 +260,7 @@ def prune_act_2to4(X: torch.Tensor, q, stream=None, out=None):
     K_lp = ss_act_2to4_shape(K)
     if out is None:
         out = (torch.empty((M, K_lp // 2), dtype=torch.uint8, device=X.device),
-               torch.empty((M, K_lp // 8), dtype=torch.uint8, device=X.device),
+               torch.empty(meta_shape(M, K_lp), dtype=torch.uint8, device=X.device),
                torch.empty(M, dtype=torch.float32, device=X.device))
     ss_prune_act_2to4(X, q, out[0], out[1], out[2], stream)
     return out

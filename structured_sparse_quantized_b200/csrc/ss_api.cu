@@ -6,8 +6,11 @@
 
 #include <atomic>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "ss.h"
 #include "ss_common.cuh"
@@ -194,24 +197,56 @@ ss_status launch_gemm_wide(int dev, const CUtensorMap& a, const CUtensorMap& b,
     return launched();
 }
 
-// B-tile width of the wide sparse GEMM: the multiple of 32 (<= 224) that
-// minimises waves x per-tile time, the per-tile time taken as proportional to
-// the bytes a K step brings into each SM (A and metadata 5 KB shared by the
-// two B tiles, plus 32 bytes per B row), which is what bounds the mainloop.
+// B-tile width of the wide sparse GEMM: the multiple of 32 (<= 224) whose
+// tile schedule (persistent pairs, snake order) finishes first.  A tile's time
+// is taken as proportional to the bytes a K step brings into each SM (A and
+// metadata 5 KB shared by the two B tiles, plus 32 bytes per token of the
+// tile), which is what bounds the mainloop.
 int choose_bn_wide(int64_t rowsA, int64_t rowsB, int units) {
     const int64_t nA = (rowsA + 2 * ss::kTileA - 1) / (2 * ss::kTileA);
     int best = ss::WideCfg::kBnMax;
     double best_cost = 0.0;
+    std::vector<double> load(static_cast<size_t>(units));
     for (int bn = ss::WideCfg::kBnMax; bn >= 64; bn -= 32) {
-        const int64_t tiles = nA * ((rowsB + 2 * bn - 1) / (2 * bn));
-        const int64_t waves = (tiles + units - 1) / units;
-        const double cost = static_cast<double>(waves) * (5120.0 / 2 + 32.0 * bn);
-        if (bn == ss::WideCfg::kBnMax || cost < best_cost * 0.999) {
+        const int64_t nB = (rowsB + 2 * bn - 1) / (2 * bn);
+        const int64_t tiles = nA * nB;
+        std::fill(load.begin(), load.end(), 0.0);
+        for (int64_t t = 0; t < tiles; ++t) {
+            const int64_t k = t / units, r = t % units;
+            const int64_t u = (k & 1) ? units - 1 - r : r;
+            const int64_t tok = std::min<int64_t>(2 * bn, rowsB - (t / nA) * 2 * bn);
+            load[static_cast<size_t>(u)] += 5120.0 + 32.0 * static_cast<double>(tok);
+        }
+        const double cost = *std::max_element(load.begin(), load.end());
+        if (bn == ss::WideCfg::kBnMax || cost < best_cost * 0.98) {
             best = bn;
             best_cost = cost;
         }
     }
     return best;
+}
+
+// SS_SPARSE_KERNEL=narrow|wide pins the sparse GEMM shape where both apply
+// (for tests and measurements); unset or anything else: chosen per problem.
+int forced_sparse_kernel() {
+    const char* v = std::getenv("SS_SPARSE_KERNEL");
+    if (!v) return 0;
+    if (std::strcmp(v, "narrow") == 0) return 1;
+    if (std::strcmp(v, "wide") == 0) return 2;
+    return 0;
+}
+
+// Wide or narrow sparse GEMM: compare the waves each needs, a wide tile
+// (256 channels x 448 tokens) counting as 1.8 narrow ones (256 x 224).  The
+// factor is measured on B200 (Qwen2.5-7B gate/up and Llama-3.1-8B q_proj
+// shapes at 8192 tokens): a wide K step moves 19 KB into each SM against
+// 2 x 12 KB, but its accumulators drain with the tensor pipe idle.
+bool prefer_wide(int64_t rowsA, int64_t rowsB, int bn_narrow, int units) {
+    const int64_t nA = (rowsA + 2 * ss::kTileA - 1) / (2 * ss::kTileA);
+    const int64_t waves_n = (nA * ((rowsB + bn_narrow - 1) / bn_narrow) + units - 1) / units;
+    const int64_t tile_w = 2 * ss::WideCfg::kBnMax;
+    const int64_t waves_w = (nA * ((rowsB + tile_w - 1) / tile_w) + units - 1) / units;
+    return 1.8 * static_cast<double>(waves_w) < static_cast<double>(waves_n);
 }
 
 // B rows per tile: the whole of a small B, else the largest width <= max.
@@ -291,6 +326,12 @@ ss_status ss_act_2to4_shape(int64_t K, int64_t* K_lp) {
     return SS_OK;
 }
 
+int64_t ss_meta_bytes(int64_t rows, int64_t K_lp) {
+    if (rows < 1 || rows > INT32_MAX || K_lp <= 0 || K_lp % 128 != 0 || K_lp > (int64_t{1} << 30))
+        return 0;
+    return (rows + 127) / 128 * 128 * (K_lp / 8);
+}
+
 ss_status ss_compress_weight(const void* W, ss_in_dtype in_dtype, int64_t N, int64_t K,
                              ss_pattern p, ss_qdtype q, void* Wv, void* Wm, float* s_w,
                              ss_stream_t stream) {
@@ -311,12 +352,14 @@ ss_status ss_compress_weight(const void* W, ss_in_dtype in_dtype, int64_t N, int
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* wv = static_cast<uint8_t*>(Wv);
     uint8_t* wm = static_cast<uint8_t*>(Wm);
+    // sparse: one more CTA per padding row of the last 128-row metadata tile
+    const int64_t rows_grid = dense ? N : (N + 127) / 128 * 128;
 #define SS_COMPRESS(T, I8)                                                                     \
     do {                                                                                      \
         auto kern = ss::compress_weight_kernel<T, I8>;                                        \
         if ((st = set_smem(kern, dev, smem)) != SS_OK) return st;                             \
-        kern<<<static_cast<unsigned>(N), ss::kCompressThreads, smem, s>>>(                    \
-            static_cast<const T*>(W), K, p.keep, p.group, K_lift, K_lp, wv, wm, s_w);         \
+        kern<<<static_cast<unsigned>(rows_grid), ss::kCompressThreads, smem, s>>>(            \
+            static_cast<const T*>(W), N, K, p.keep, p.group, K_lift, K_lp, wv, wm, s_w);      \
     } while (0)
     if (in_dtype == SS_IN_BF16) {
         if (q == SS_INT8) SS_COMPRESS(__nv_bfloat16, true);
@@ -400,7 +443,8 @@ ss_status ss_prune_act_2to4(const void* X, ss_in_dtype in_dtype, int64_t M, int6
     uint8_t* xv = static_cast<uint8_t*>(Xv);
     uint8_t* xm = static_cast<uint8_t*>(Xm);
     const int warps = ss::kWarpRowThreads / 32;
-    const unsigned grid = static_cast<unsigned>((M + warps - 1) / warps);
+    // warps past M zero the padding rows of the last 128-row metadata tile
+    const unsigned grid = static_cast<unsigned>(((M + 127) / 128 * 128 + warps - 1) / warps);
 #define SS_PRUNE(T, I8)                                                                        \
     do {                                                                                      \
         ss::prune_act_warp_kernel<T, I8><<<grid, ss::kWarpRowThreads, 0, s>>>(               \
@@ -441,7 +485,8 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
                      CS::kARowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                            : CU_TENSOR_MAP_SWIZZLE_64B) ||
         !make_map_2d(&tb, B, rowsB, K_lp, bn / pair, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_2d(&te, Am, rowsA, K_lp / 8, ss::kTileA, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
+        !make_map_2d(&te, Am, (rowsA + 127) / 128 * (K_lp / 128) * 16, 128, 16, 128,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
         return SS_ERR_CUDA;
     ss::GemmArgs args;
     args.rowsA = static_cast<int>(rowsA);
@@ -451,6 +496,7 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
     args.bn = bn;
     args.a_is_w = sparse_operand == 0 ? 1 : 0;
     args.ldy = static_cast<int>(N);
+    args.e_chunks = static_cast<int>(K_lp / 128);
     args.s_a = s_a;
     args.s_b = s_b;
     args.y = Y;
@@ -460,8 +506,12 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
     cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
     const bool i8 = q == SS_INT8, bf = out_dtype == SS_OUT_BF16;
 #if SS_SPARSE_WIDE
-    // Large problems with channel rows and bf16 Y: two B tiles per output tile.
-    if (pair == 2 && args.a_is_w && args.tma_store && rowsB > 2 * ss::WideCfg::kBnMax) {
+    // Large problems with channel rows and bf16 Y may take two B tiles per
+    // output tile: fewer bytes per MMA, but single-buffered accumulators.
+    const int forced = forced_sparse_kernel();
+    if (pair == 2 && args.a_is_w && args.tma_store && forced != 1 &&
+        (forced == 2 || (rowsB > 2 * ss::WideCfg::kBnMax &&
+                         prefer_wide(rowsA, rowsB, bn, g_num_sms[dev] / 2)))) {
         using CW = ss::WideCfg;
         const int bnw = choose_bn_wide(rowsA, rowsB, g_num_sms[dev] / 2);
         CUtensorMap wa, wb;

@@ -90,6 +90,13 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  : "memory");
 }
 
+// Tile-major metadata: byte b of row r of a [rows, K_lp/8] selector matrix is
+// stored at this offset, so the selectors of 128 rows x 128 K (one GEMM
+// stage's metadata tile) form one contiguous 2 KB block ([128 rows][16 B]).
+__host__ __device__ __forceinline__ int64_t meta_offset(int64_t r, int64_t b, int64_t K_lp) {
+    return ((r >> 7) * (K_lp >> 7) + (b >> 4)) * 2048 + (r & 127) * 16 + (b & 15);
+}
+
 // ---------------------------------------------------------------------------
 // TMA (no multicast anywhere in this library).
 // ---------------------------------------------------------------------------

@@ -74,12 +74,16 @@ __device__ __forceinline__ void window_indices(uint32_t own, int& i0, int& i1) {
 
 template <typename T, bool kInt8>
 __global__ void __launch_bounds__(kCompressThreads) compress_weight_kernel(
-    const T* __restrict__ W, int64_t K, int keep, int group, int64_t K_lift, int64_t K_lp,
-    uint8_t* __restrict__ Wv, uint8_t* __restrict__ Wm, float* __restrict__ s_w) {
+    const T* __restrict__ W, int64_t N, int64_t K, int keep, int group, int64_t K_lift,
+    int64_t K_lp, uint8_t* __restrict__ Wv, uint8_t* __restrict__ Wm, float* __restrict__ s_w) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     __shared__ float red[32];
     __shared__ int bad;
     const int64_t n = blockIdx.x;
+    if (n >= N) {  // padding row of the last 128-row metadata tile
+        for (int64_t b = threadIdx.x; b < K_lp / 8; b += blockDim.x) Wm[meta_offset(n, b, K_lp)] = 0;
+        return;
+    }
     const T* w = W + n * K;
     float* srow = reinterpret_cast<float*>(smem_raw);  // K_pad floats
     const bool dense = (group == 0);
@@ -133,7 +137,6 @@ __global__ void __launch_bounds__(kCompressThreads) compress_weight_kernel(
     const int Nh = group / 2;
     const int64_t n_win = K_lift / 4;
     uint8_t* vrow = Wv + n * (K_lp / 2);
-    uint8_t* mrow = Wm + n * (K_lp / 8);
     const uint8_t* kept_hi = kept + K_pad / group;
     for (int64_t pr = threadIdx.x; pr < K_lp / 8; pr += blockDim.x) {
         uint32_t vals = 0;
@@ -157,7 +160,7 @@ __global__ void __launch_bounds__(kCompressThreads) compress_weight_kernel(
             meta |= static_cast<uint32_t>(i0 | (i1 << 2)) << (4 * h);
         }
         reinterpret_cast<uint32_t*>(vrow)[pr] = vals;  // 4 value bytes
-        mrow[pr] = static_cast<uint8_t>(meta);
+        Wm[meta_offset(n, pr, K_lp)] = static_cast<uint8_t>(meta);
     }
 }
 

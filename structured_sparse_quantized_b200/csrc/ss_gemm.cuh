@@ -116,6 +116,7 @@ struct GemmArgs {
     int ldy;          // leading dimension of Y (= N)
     int tma_store;    // 1: Y written by TMA tensor stores through shared memory
                       //    (A rows = channels: 128B-swizzled [32][64] halves)
+    int e_chunks;     // K_lp / 128: 2 KB metadata tiles per 128 rows (tile-major)
     const float* s_a;
     const float* s_b;
     void* y;
@@ -243,7 +244,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             for (int u = 0; u < C::kEChunks; ++u)
                                 tma_load_2d_pair_hint(
                                     st + C::kEOffset + at * C::kEBytes + u * kTileA * 16, &tm_e,
-                                    fb, kb * C::kEChunks * 16 + u * 16, a0 + at * pair_rows, keep);
+                                    fb, 0,
+                                    (((a0 + at * pair_rows) >> 7) * args.e_chunks +
+                                     kb * C::kEChunks + u) * 16,
+                                    keep);
                     } else {
                         mbar_arrive_expect_tx(&full[s], tx);
                         tma_load_2d(st, &tm_a, &full[s], kb * C::kARowBytes, a0);
@@ -253,8 +257,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                         kb * C::kStageK + u * 128, b0);
 #pragma unroll
                         for (int u = 0; u < C::kEChunks; ++u)
-                            tma_load_2d(st + C::kEOffset + u * kTileA * 16, &tm_e, &full[s],
-                                        kb * C::kEChunks * 16 + u * 16, a0);
+                            tma_load_2d(st + C::kEOffset + u * kTileA * 16, &tm_e, &full[s], 0,
+                                        ((a0 >> 7) * args.e_chunks + kb * C::kEChunks + u) * 16);
                     }
                 }
                 __syncwarp();

@@ -75,6 +75,13 @@ struct WideCfg {
                   "stage alignment");
 };
 
+// Tile of pair `unit` in wave k.  Waves alternate direction, so the short
+// tiles at the end of the list (the last, partial token tile of every channel
+// tile) go to the pairs that took fewer full tiles in the wave before.
+__device__ __forceinline__ int snake_tile(int k, int unit, int n_units) {
+    return k * n_units + ((k & 1) ? (n_units - 1 - unit) : unit);
+}
+
 template <bool kInt8>
 __global__ void __launch_bounds__(kWideThreads, 1)
     gemm_sparse_wide_kernel(const __grid_constant__ CUtensorMap tm_a,
@@ -139,7 +146,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         int s = 0;
         uint32_t ph = 0, armed = 0, armed_par = 0;
         bool ok = true;
-        for (int t = unit; t < n_tiles && ok; t += n_units) {
+        for (int k = 0, t = snake_tile(0, unit, n_units); t < n_tiles && ok;
+             ++k, t = snake_tile(k, unit, n_units)) {
             const int a0 = (t % nA) * kPairRows + static_cast<int>(rank) * kTileA;
             const int b0 = (t / nA) * tile_b_rows + static_cast<int>(rank) * b_rows_cta;
             for (int kb = 0; kb < args.k_stages; ++kb) {
@@ -157,7 +165,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                     for (int u = 0; u < kWideBT; ++u)
                         tma_load_2d_pair_hint(st + C::kBOffset + u * C::kBTileBytes, &tm_b, fb,
                                               kb * C::kStageK, b0 + u * args.bn, keep);
-                    tma_load_2d_pair_hint(st + C::kEOffset, &tm_e, fb, kb * 16, a0, keep);
+                    tma_load_2d_pair_hint(st + C::kEOffset, &tm_e, fb, 0,
+                                          ((a0 >> 7) * args.e_chunks + kb) * 16, keep);
                 }
                 __syncwarp();
                 armed |= 1u << s;
@@ -193,7 +202,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
             uint32_t ph = 0;
             bool ok = true;
             int i = 0;
-            for (int t = unit; t < n_tiles && ok; t += n_units, ++i) {
+            for (int t = snake_tile(0, unit, n_units); t < n_tiles && ok;
+                 ++i, t = snake_tile(i, unit, n_units)) {
                 if (!__all_sync(0xffffffffu, mbar_wait(acc_empty, (i & 1) ^ 1u, abort_flag))) {
                     ok = false;
                     break;
@@ -269,7 +279,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         const int mi = lane >> 3, mj = lane & 7;  // this thread's stmatrix matrix / row
         int i = 0;
         uint32_t chunk_iter = 0;
-        for (int t = unit; t < n_tiles; t += n_units, ++i) {
+        for (int t = snake_tile(0, unit, n_units); t < n_tiles;
+             ++i, t = snake_tile(i, unit, n_units)) {
             const int a_cta0 = (t % nA) * kPairRows + static_cast<int>(rank) * kTileA;
             const int tile_tok0 = (t / nA) * tile_b_rows;
             const int tok0 = tile_tok0 + bt * args.bn;

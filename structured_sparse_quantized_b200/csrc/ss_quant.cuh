@@ -259,7 +259,13 @@ __global__ void __launch_bounds__(kWarpRowThreads) prune_act_warp_kernel(
     uint8_t* __restrict__ Xm, float* __restrict__ s_x) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t m = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
-    if (m >= M) return;
+    const int64_t M_pad = (M + 127) / 128 * 128;
+    if (m >= M_pad) return;
+    if (m >= M) {  // padding row of the last 128-row metadata tile
+        for (int64_t st = lane; st < K_lp64 / 32; st += 32)
+            *reinterpret_cast<uint32_t*>(Xm + meta_offset(m, 4 * st, K_lp64)) = 0u;
+        return;
+    }
     const int K = static_cast<int>(K64);
     const int K_lp = static_cast<int>(K_lp64);
     const T* x = X + m * K64;
@@ -271,7 +277,6 @@ __global__ void __launch_bounds__(kWarpRowThreads) prune_act_warp_kernel(
     if (lane == 0) s_x[m] = s;
     // One step = 8 groups of 4 = 32 inputs -> 16 value bytes + 4 nibble bytes.
     uint4* vout = reinterpret_cast<uint4*>(Xv + m * (K_lp64 / 2));
-    uint32_t* mout = reinterpret_cast<uint32_t*>(Xm + m * (K_lp64 / 8));
     const int n_steps = K_lp / 32;
     for (int st = lane; st < n_steps; st += 32) {
         float f[32];
@@ -292,7 +297,7 @@ __global__ void __launch_bounds__(kWarpRowThreads) prune_act_warp_kernel(
             nibs |= static_cast<uint32_t>(i0 | (i1 << 2)) << (4 * gi);
         }
         __stcs(vout + st, make_uint4(vals[0], vals[1], vals[2], vals[3]));
-        __stcs(mout + st, nibs);
+        __stcs(reinterpret_cast<uint32_t*>(Xm + meta_offset(m, 4 * st, K_lp64)), nibs);
     }
 }
 

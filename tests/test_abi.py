@@ -6,6 +6,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 import oracle
@@ -105,3 +106,28 @@ def test_argument_errors_return_before_any_launch(L):
         == ss.SS_ERR_INVALID_ARG
     assert L.ss_compress_weight(good, 1, 64, 1 << 20, pat, 0, good, good, good, None) \
         == ss.SS_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("rows,K_lp", [(1, 128), (130, 384), (256, 1024), (300, 128)])
+def test_metadata_storage_layout(L, rows, K_lp):
+    """Tile-major selector storage: every byte sits where ss.h's formula puts
+    it, padding rows are zero, and the buffer size is ss_meta_bytes()."""
+    rng = np.random.default_rng(rows + K_lp)
+    Am = rng.integers(0, 256, (rows, K_lp // 8), dtype=np.uint8)
+    At = oracle.meta_to_tiles(Am, K_lp)
+    assert At.shape == ss.meta_shape(rows, K_lp)
+    assert At.size == ss.ss_meta_bytes(rows, K_lp)
+    flat = At.reshape(-1)
+    r, b = np.meshgrid(np.arange(rows), np.arange(K_lp // 8), indexing="ij")
+    off = ((r // 128) * (K_lp // 128) + b // 16) * 2048 + (r % 128) * 16 + b % 16
+    np.testing.assert_array_equal(flat[off], Am)
+    mask = np.ones(flat.size, dtype=bool)
+    mask[off.reshape(-1)] = False
+    assert not flat[mask].any()                          # padding rows
+    np.testing.assert_array_equal(oracle.meta_from_tiles(At, rows, K_lp), Am)
+
+
+def test_meta_bytes_rejects_bad_shapes(L):
+    assert ss.ss_meta_bytes(0, 128) == 0
+    assert ss.ss_meta_bytes(5, 100) == 0
+    assert ss.ss_meta_bytes(5, 0) == 0

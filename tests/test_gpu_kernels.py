@@ -41,7 +41,8 @@ def test_prune_act_2to4(q, dt, M, K):
     Xv_ref, Xm_ref, s_ref = oracle.prune_act_2to4(X, Q[q])
     Xv, Xm, s_x = ss.prune_act_2to4(dev(X), q)
     np.testing.assert_array_equal(host(s_x), s_ref)
-    np.testing.assert_array_equal(host(Xm), Xm_ref)
+    K_lp = Xv_ref.shape[1] * 2
+    np.testing.assert_array_equal(host(Xm), oracle.meta_to_tiles(Xm_ref, K_lp))
     np.testing.assert_array_equal(host(Xv), Xv_ref)
 
 
@@ -56,7 +57,7 @@ def test_compress_weight(pat, q, dt, N, K):
     np.testing.assert_array_equal(host(s_w), s_ref)
     np.testing.assert_array_equal(host(Wv), Wv_ref)
     if pat != "dense":
-        np.testing.assert_array_equal(host(Wm), Wm_ref)
+        np.testing.assert_array_equal(host(Wm), oracle.meta_to_tiles(Wm_ref, Wv_ref.shape[1] * 2))
     assert ss.ss_get_device_status() == ss.SS_OK
 
 
@@ -71,7 +72,8 @@ def test_compress_weight_with_ties_and_zeros():
             Wv, Wm, s_w = ss.compress_weight(dev(W), pat, q)
             np.testing.assert_array_equal(host(s_w), s_ref)
             np.testing.assert_array_equal(host(Wv), Wv_ref)
-            np.testing.assert_array_equal(host(Wm), Wm_ref)
+            np.testing.assert_array_equal(host(Wm),
+                                          oracle.meta_to_tiles(Wm_ref, Wv_ref.shape[1] * 2))
 
 
 def test_nan_weight_reports_data_error():
@@ -105,16 +107,16 @@ def test_sparse_gemm_weight_sparse(M, N, K, pat, q, out):
     ob = out == "bf16"
     Y_ref = oracle.sparse_gemm(0, Wv, Wm, s_w, Xq, s_x, M, N, K_lp, Q[q],
                                oracle.OUT_BF16 if ob else oracle.OUT_F32)
-    Y = ss.sparse_gemm(0, dev(Wv), dev(Wm), dev(s_w), dev(Xq), dev(s_x), M, N, q,
-                       out_dtype=torch.bfloat16 if ob else torch.float32)
+    Y = ss.sparse_gemm(0, dev(Wv), dev(oracle.meta_to_tiles(Wm, K_lp)), dev(s_w), dev(Xq),
+                       dev(s_x), M, N, q, out_dtype=torch.bfloat16 if ob else torch.float32)
     assert ss.ss_get_device_status() == ss.SS_OK
     assert_y_matches(host(Y), Y_ref, q, ob)
 
 
-# Shapes with more than two 224-token tiles and more than 128 channels take
-# the two-B-tile kernel (single-buffered accumulators, collector-reused A):
-# several tiles per CTA pair, ragged channels and tokens, odd stage counts and
-# the narrower B tiles the wave balancing picks.
+# Shapes run by both sparse kernel shapes (pinned with SS_SPARSE_KERNEL): the
+# two-B-tile one (single-buffered accumulators, collector-reused A) and the
+# one-B-tile one.  Several tiles per CTA pair, ragged channels and tokens, odd
+# stage counts and the narrower B tiles the wave balancing picks.
 WIDE_CASES = [  # M, N, K, pattern, sampled token rows (None = all)
     (1000, 520, 1024, "2:4", None),    # ragged both ways, 8 stages
     (2000, 300, 768, "6:8", None),     # 9 stages (odd against the 5-stage ring)
@@ -127,7 +129,9 @@ WIDE_CASES = [  # M, N, K, pattern, sampled token rows (None = all)
 
 @pytest.mark.parametrize("M,N,K,pat,nrows", WIDE_CASES)
 @pytest.mark.parametrize("q", ["int8", "fp8"])
-def test_sparse_gemm_wide_tiles(M, N, K, pat, nrows, q):
+@pytest.mark.parametrize("kernel", ["wide", "narrow"])
+def test_sparse_gemm_wide_tiles(M, N, K, pat, nrows, q, kernel, monkeypatch):
+    monkeypatch.setenv("SS_SPARSE_KERNEL", kernel)
     W = synth.gaussian((N, K), std=0.02, seed=0, dtype=torch.bfloat16)
     X = synth.gaussian((M, K), std=1.0, seed=1, dtype=torch.bfloat16)
     Wv, Wm, s_w = oracle.compress_weight(W, pat, Q[q])
@@ -136,7 +140,8 @@ def test_sparse_gemm_wide_tiles(M, N, K, pat, nrows, q):
     rows = None if nrows is None else synth.sample_rows(M, seed=5, middle=nrows)
     Y_ref = oracle.sparse_gemm(0, Wv, Wm, s_w, Xq, s_x, M, N, K_lp, Q[q], oracle.OUT_BF16,
                                m_idx=rows)
-    Y = host(ss.sparse_gemm(0, dev(Wv), dev(Wm), dev(s_w), dev(Xq), dev(s_x), M, N, q))
+    Y = host(ss.sparse_gemm(0, dev(Wv), dev(oracle.meta_to_tiles(Wm, K_lp)), dev(s_w), dev(Xq),
+                            dev(s_x), M, N, q))
     assert ss.ss_get_device_status() == ss.SS_OK
     assert_y_matches(Y if rows is None else Y[rows], Y_ref, q, True)
 
@@ -151,7 +156,8 @@ def test_sparse_gemm_activation_sparse(M, N, K, q):
     K_lp = oracle.act_2to4_k_lp(K)
     assert Wq.shape[1] == K_lp
     Y_ref = oracle.sparse_gemm(1, Xv, Xm, s_x, Wq, s_w, M, N, K_lp, Q[q], oracle.OUT_BF16)
-    Y = ss.sparse_gemm(1, dev(Xv), dev(Xm), dev(s_x), dev(Wq), dev(s_w), M, N, q)
+    Y = ss.sparse_gemm(1, dev(Xv), dev(oracle.meta_to_tiles(Xm, K_lp)), dev(s_x), dev(Wq),
+                       dev(s_w), M, N, q)
     assert ss.ss_get_device_status() == ss.SS_OK
     assert_y_matches(host(Y), Y_ref, q, True)
 
