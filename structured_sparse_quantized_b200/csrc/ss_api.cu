@@ -406,16 +406,29 @@ ss_status ss_quant_lift_act(const void* X, ss_in_dtype in_dtype, int64_t M, int6
     // bf16 rows of up to 4096 elements (K % 16 == 0) are read once, into registers
     const bool reg_path = in_dtype == SS_IN_BF16 && K % 16 == 0 && K <= ss::kRegK;
     if (reg_path) {
+        // registers for the row: just enough 16-element chunks per lane for K
+        const int chunks = static_cast<int>((K + 511) / 512);
         const auto* xb = static_cast<const __nv_bfloat16*>(X);
-        if (q == SS_INT8) {
-            auto kern = ss::quant_lift_reg_kernel<true>;
-            if ((st = set_smem(kern, dev, smem)) != SS_OK) return st;
-            kern<<<grid, warps * 32, smem, s>>>(xb, M, K, Nh, K_lift, K_lp, q_stride, xq, s_x);
-        } else {
-            auto kern = ss::quant_lift_reg_kernel<false>;
-            if ((st = set_smem(kern, dev, smem)) != SS_OK) return st;
-            kern<<<grid, warps * 32, smem, s>>>(xb, M, K, Nh, K_lift, K_lp, q_stride, xq, s_x);
-        }
+        // 6:8 lifts in registers (no shared-memory row)
+        const size_t rsmem = Nh == 4 ? 0 : smem;
+#define SS_QREG(I8, C)                                                                         \
+    do {                                                                                      \
+        auto kern = ss::quant_lift_reg_kernel<I8, C>;                                         \
+        if ((st = set_smem(kern, dev, rsmem)) != SS_OK) return st;                            \
+        kern<<<grid, warps * 32, rsmem, s>>>(xb, M, K, Nh, K_lift, K_lp, q_stride, xq, s_x);  \
+    } while (0)
+#define SS_QREG_C(I8)                                                                          \
+    do {                                                                                      \
+        if (chunks <= 2) SS_QREG(I8, 2);                                                      \
+        else if (chunks <= 4) SS_QREG(I8, 4);                                                 \
+        else if (chunks <= 6) SS_QREG(I8, 6);                                                 \
+        else if (chunks <= 7) SS_QREG(I8, 7);                                                 \
+        else SS_QREG(I8, 8);                                                                  \
+    } while (0)
+        if (q == SS_INT8) SS_QREG_C(true);
+        else SS_QREG_C(false);
+#undef SS_QREG_C
+#undef SS_QREG
     } else if (in_dtype == SS_IN_BF16) {
         if (q == SS_INT8) SS_QLIFT(__nv_bfloat16, true);
         else SS_QLIFT(__nv_bfloat16, false);

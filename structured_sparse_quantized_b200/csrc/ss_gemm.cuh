@@ -122,14 +122,6 @@ struct GemmArgs {
     void* y;
 };
 
-__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
-    const uint32_t b = smem_u32(bar);
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(b, parity))
-        if (global_timer_ns() - t0 > 100000000ull) return false;  // 100 ms
-    return true;
-}
-
 template <bool kInt8, bool kOutBf16>
 __device__ __forceinline__ void store_scaled(void* y, int64_t off, uint32_t acc_bits, float sx,
                                              float sw) {

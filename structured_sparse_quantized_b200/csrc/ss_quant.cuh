@@ -317,8 +317,9 @@ __device__ __forceinline__ void bf16x16_to_f32(const uint4& a, const uint4& b, f
     }
 }
 
-// Requires K % 16 == 0, K <= kRegK and a 16-byte aligned X.
-template <bool kInt8>
+// Requires K % 16 == 0, K <= 512 * kChunks and a 16-byte aligned X.
+// kChunks = 16-element chunks per lane (rows of up to 512 kChunks values).
+template <bool kInt8, int kChunks>
 __global__ void __launch_bounds__(kWarpRowThreads) quant_lift_reg_kernel(
     const __nv_bfloat16* __restrict__ X, int64_t M, int64_t K64, int Nh, int64_t K_lift64,
     int64_t K_lp64, int q_stride, uint8_t* __restrict__ Xq, float* __restrict__ s_x) {
@@ -331,9 +332,9 @@ __global__ void __launch_bounds__(kWarpRowThreads) quant_lift_reg_kernel(
     const int K_lp = static_cast<int>(K_lp64);
     const uint4* xv = reinterpret_cast<const uint4*>(X + m * K64);
     const int n16 = K / 16;
-    uint4 v[2 * kRegChunks];
+    uint4 v[2 * kChunks];
 #pragma unroll
-    for (int i = 0; i < kRegChunks; ++i) {
+    for (int i = 0; i < kChunks; ++i) {
         const int c = lane + 32 * i;
         if (c < n16) {
             v[2 * i] = __ldcs(xv + 2 * c);
@@ -345,7 +346,7 @@ __global__ void __launch_bounds__(kWarpRowThreads) quant_lift_reg_kernel(
     }
     float a = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 2 * kRegChunks; ++i) a = fmaxf(a, chunk_absmax<__nv_bfloat16>(v[i]));
+    for (int i = 0; i < 2 * kChunks; ++i) a = fmaxf(a, chunk_absmax<__nv_bfloat16>(v[i]));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
     float inv, s;
@@ -355,7 +356,7 @@ __global__ void __launch_bounds__(kWarpRowThreads) quant_lift_reg_kernel(
     const int n_chunks = K_lp / 16;
     if (Nh <= 2) {  // identity map: chunk c of the output is chunk c of the input
 #pragma unroll
-        for (int i = 0; i < kRegChunks; ++i) {
+        for (int i = 0; i < kChunks; ++i) {
             const int c = lane + 32 * i;
             if (c < n16) {
                 float f[16];
@@ -366,10 +367,32 @@ __global__ void __launch_bounds__(kWarpRowThreads) quant_lift_reg_kernel(
         for (int c = n16 + lane; c < n_chunks; c += 32) __stcs(out + c, make_uint4(0, 0, 0, 0));
         return;
     }
+    if (Nh == 4) {
+        // 6:8: a 16-element chunk is exactly two groups of 8, and its six
+        // windows (elements 0-3, 2-5, 4-7 of each group) are made of its own
+        // codes: 24 lifted bytes at 24c, no other lane's data involved.
+#pragma unroll
+        for (int i = 0; i < kChunks; ++i) {
+            const int c = lane + 32 * i;
+            if (c < n16) {
+                float f[16];
+                bf16x16_to_f32(v[2 * i], v[2 * i + 1], f);
+                const uint4 w = quant16<kInt8>(f, inv);
+                uint2* o = reinterpret_cast<uint2*>(Xq + m * K_lp64 + 24 * static_cast<int64_t>(c));
+                __stcs(o, make_uint2(w.x, __byte_perm(w.x, w.y, 0x5432)));
+                __stcs(o + 1, make_uint2(w.y, w.z));
+                __stcs(o + 2, make_uint2(__byte_perm(w.z, w.w, 0x5432), w.w));
+            }
+        }
+        // zero windows past the last group up to K_lp (8-byte aligned: K_lift = 24 K / 16)
+        uint2* z = reinterpret_cast<uint2*>(Xq + m * K_lp64);
+        for (int c8 = K_lift / 8 + lane; c8 < K_lp / 8; c8 += 32) __stcs(z + c8, make_uint2(0, 0));
+        return;
+    }
     uint4* qrow = reinterpret_cast<uint4*>(smem_raw + warp * q_stride);
     const int q_chunks = ((K_lift / (4 * (Nh - 1))) * 2 * Nh + 15) / 16;
 #pragma unroll
-    for (int i = 0; i < kRegChunks; ++i) {
+    for (int i = 0; i < kChunks; ++i) {
         const int c = lane + 32 * i;
         if (c < n16) {
             float f[16];

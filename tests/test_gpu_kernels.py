@@ -46,6 +46,32 @@ def test_prune_act_2to4(q, dt, M, K):
     np.testing.assert_array_equal(host(Xv), Xv_ref)
 
 
+# Many bf16 rows (several CTAs per SM, many warps per row stream) at the K
+# values of each register-resident variant (up to 2, 4, 6, 7 and 8 sixteen-
+# element chunks per lane), the 6:8 in-register lift with and without a zero
+# tail up to K_lp, and a K that takes the two-pass kernel.
+@pytest.mark.parametrize("pat", ["dense"] + PATTERNS)
+@pytest.mark.parametrize("q", ["int8", "fp8"])
+@pytest.mark.parametrize("K", [4096, 3584, 3072, 2048, 1040, 1032, 512])
+def test_quant_lift_act_many_rows(pat, q, K):
+    X = _x(3000, K, "bf16", seed=K)
+    Xq_ref, s_ref = oracle.quant_lift_act(X, pat, Q[q])
+    Xq, s_x = ss.quant_lift_act(dev(X), pat, q)
+    np.testing.assert_array_equal(host(s_x), s_ref)
+    np.testing.assert_array_equal(host(Xq), Xq_ref)
+
+
+@pytest.mark.parametrize("q", ["int8", "fp8"])
+@pytest.mark.parametrize("M,K", [(5000, 4096), (3001, 2056)])
+def test_prune_act_2to4_many_rows(q, M, K):
+    X = synth.gaussian_with_heavy_tails(M, K, seed=M)
+    Xv_ref, Xm_ref, s_ref = oracle.prune_act_2to4(X, Q[q])
+    Xv, Xm, s_x = ss.prune_act_2to4(dev(X), q)
+    np.testing.assert_array_equal(host(s_x), s_ref)
+    np.testing.assert_array_equal(host(Xm), oracle.meta_to_tiles(Xm_ref, Xv_ref.shape[1] * 2))
+    np.testing.assert_array_equal(host(Xv), Xv_ref)
+
+
 @pytest.mark.parametrize("pat", ["dense"] + PATTERNS)
 @pytest.mark.parametrize("q", ["int8", "fp8"])
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
