@@ -62,7 +62,7 @@ def test_quant_lift_act_many_rows(pat, q, K):
 
 
 @pytest.mark.parametrize("q", ["int8", "fp8"])
-@pytest.mark.parametrize("M,K", [(5000, 4096), (3001, 2056)])
+@pytest.mark.parametrize("M,K", [(5000, 4096), (3001, 4000), (3001, 2056), (700, 1024)])
 def test_prune_act_2to4_many_rows(q, M, K):
     X = synth.gaussian_with_heavy_tails(M, K, seed=M)
     Xv_ref, Xm_ref, s_ref = oracle.prune_act_2to4(X, Q[q])
