@@ -96,7 +96,9 @@ struct GemmCfg {
     static constexpr int kAccStride = kBnMax;              // TMEM columns between accumulators
     static constexpr int kECol = 2 * kBnMax;               // metadata columns (sparse)
     static constexpr int kESlotCols = 4 * kEChunks * kAT;  // columns one stage's metadata takes
-    static constexpr int kESlots = kAT == 1 ? 4 : 2;
+    // one metadata slot per stage: a slot is rewritten only after its stage's
+    // "empty" commit, i.e. after the MMAs that read it completed
+    static constexpr int kESlots = kStages;
     static constexpr int kEpiOffset = kStages * kStageBytes;  // 2 staging buffers for Y chunks
     static constexpr int kSmemBytes =
         kEpiOffset + 2 * kEpiBytes + 1024 /*align*/ + 256 /*barriers*/;
@@ -105,6 +107,7 @@ struct GemmCfg {
     static_assert(!kSparse || kECol + kESlots * kESlotCols <= kTmemCols, "TMEM budget");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
     static_assert(kStages >= (kPair == 2 ? 3 : 2), "pipeline depth");
+    static_assert((2 * kStages + 5) * 8 + 4 <= 256, "barrier area");
 };
 
 struct GemmArgs {
@@ -285,7 +288,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 smem_desc(base + C::kEOffset, 128 * 16, 128, kSwizzleNone);
             int s = 0;
             uint32_t ph = 0;
-            uint32_t e_iter = 0;
             bool ok = true;
             int i = 0;
             for (int t = unit; t < n_tiles && ok; t += n_units, ++i) {
@@ -306,7 +308,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tc_fence_after();
                     const uint64_t soff = static_cast<uint64_t>((s * C::kStageBytes) >> 4);
                     const uint32_t e_tmem =
-                        tmem_base + C::kECol + C::kESlotCols * (e_iter & (C::kESlots - 1));
+                        tmem_base + C::kECol + C::kESlotCols * s;
 #pragma unroll
                     for (int at = 0; at < kAT; ++at) {
                         if (kAT == 2 && at == 1 && kb == 0) {  // A tile 1's accumulator drained?
@@ -351,7 +353,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     if (!ok) break;
                     if (elect_one()) tc_commit_g<kPair>(&empty[s]);  // stage free in both CTAs
                     __syncwarp();
-                    ++e_iter;
                     if (++s == C::kStages) {
                         s = 0;
                         ph ^= 1u;
