@@ -426,7 +426,16 @@ def main():
     ap.add_argument("--no-also", action="store_true", help="skip the 6:8 FP8 side measurement")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--ref-budget", type=float, default=6.0)
+    ap.add_argument("--pattern", default=None, choices=["2:4", "4:6", "6:8", "8:10"],
+                    help="override the workload's pattern (the Llama-layer sweep)")
+    ap.add_argument("--qdtype", default=None, choices=["int8", "fp8"],
+                    help="override the workload's quantised type")
     args = ap.parse_args()
+    if args.pattern or args.qdtype:
+        w = dict(synth.WORKLOADS[args.workload])
+        w["pattern"] = args.pattern or w["pattern"]
+        w["qdtype"] = args.qdtype or w["qdtype"]
+        synth.WORKLOADS[args.workload] = w
     if args.m is None:
         args.m = DEFAULT_M if args.workload != "linear_6of8_int8_m16" else 16
     args.warmup = max(args.warmup, 3)

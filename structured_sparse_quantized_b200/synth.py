@@ -76,6 +76,13 @@ WORKLOADS = {
 LLAMA_LAYER = {"q_o": (4096, 4096), "k_v": (1024, 4096), "gate_up": (14336, 4096),
                "down": (4096, 14336)}
 
+# The sweep's workloads (one per projection; pattern and qdtype are varied on
+# the bench command line): Gaussian W std 0.02, Gaussian X, bf16 out.
+for _proj, (_n, _k) in LLAMA_LAYER.items():
+    WORKLOADS[f"llama_layer_{_proj}"] = dict(M=16384, K=_k, N=_n, pattern="6:8", qdtype="int8",
+                                            in_dtype="bf16", w_std=0.02, out="bf16",
+                                            x_kind="gauss")
+
 
 def make_weight(N: int, K: int, std: float, in_dtype: str, seed: int = 0) -> torch.Tensor:
     return gaussian((N, K), std=std, seed=seed,
