@@ -406,24 +406,39 @@ ss_status ss_quant_lift_act(const void* X, ss_in_dtype in_dtype, int64_t M, int6
     // bf16 rows of up to 4096 elements (K % 16 == 0) are read once, into registers
     const bool reg_path = in_dtype == SS_IN_BF16 && K % 16 == 0 && K <= ss::kRegK;
     if (reg_path) {
-        // registers for the row: just enough 16-element chunks per lane for K
-        const int chunks = static_cast<int>((K + 511) / 512);
+        // registers for the row: 1, 2 or 4 warps per row, each lane holding
+        // just enough 16-element chunks
+        const int wpr = K <= 4096 ? 1 : (K <= 8192 ? 2 : 4);
+        const int chunks = static_cast<int>((K + 512 * wpr - 1) / (512 * wpr));
+        const int rows_per_cta = (ss::kWarpRowThreads / 32) / wpr;
+        const unsigned rgrid = static_cast<unsigned>((M + rows_per_cta - 1) / rows_per_cta);
         const auto* xb = static_cast<const __nv_bfloat16*>(X);
-        // 6:8 lifts in registers (no shared-memory row)
-        const size_t rsmem = Nh == 4 ? 0 : smem;
-#define SS_QREG(I8, C)                                                                         \
+        // 6:8 lifts in registers; 4:6 and 8:10 keep one code row per row slot
+        const size_t rsmem = Nh == 4 ? 0 : static_cast<size_t>(rows_per_cta) * q_stride;
+#define SS_QREG(I8, C, W)                                                                      \
     do {                                                                                      \
-        auto kern = ss::quant_lift_reg_kernel<I8, C>;                                         \
+        auto kern = ss::quant_lift_reg_kernel<I8, C, W>;                                      \
         if ((st = set_smem(kern, dev, rsmem)) != SS_OK) return st;                            \
-        kern<<<grid, warps * 32, rsmem, s>>>(xb, M, K, Nh, K_lift, K_lp, q_stride, xq, s_x);  \
+        kern<<<rgrid, ss::kWarpRowThreads, rsmem, s>>>(xb, M, K, Nh, K_lift, K_lp, q_stride,  \
+                                                       xq, s_x);                              \
     } while (0)
 #define SS_QREG_C(I8)                                                                          \
     do {                                                                                      \
-        if (chunks <= 2) SS_QREG(I8, 2);                                                      \
-        else if (chunks <= 4) SS_QREG(I8, 4);                                                 \
-        else if (chunks <= 6) SS_QREG(I8, 6);                                                 \
-        else if (chunks <= 7) SS_QREG(I8, 7);                                                 \
-        else SS_QREG(I8, 8);                                                                  \
+        if (wpr == 1) {                                                                       \
+            if (chunks <= 2) SS_QREG(I8, 2, 1);                                               \
+            else if (chunks <= 4) SS_QREG(I8, 4, 1);                                          \
+            else if (chunks <= 6) SS_QREG(I8, 6, 1);                                          \
+            else if (chunks <= 7) SS_QREG(I8, 7, 1);                                          \
+            else SS_QREG(I8, 8, 1);                                                           \
+        } else if (wpr == 2) {                                                                \
+            if (chunks <= 6) SS_QREG(I8, 6, 2);                                               \
+            else if (chunks <= 7) SS_QREG(I8, 7, 2);                                          \
+            else SS_QREG(I8, 8, 2);                                                           \
+        } else {                                                                              \
+            if (chunks <= 6) SS_QREG(I8, 6, 4);                                               \
+            else if (chunks <= 7) SS_QREG(I8, 7, 4);                                          \
+            else SS_QREG(I8, 8, 4);                                                           \
+        }                                                                                     \
     } while (0)
         if (q == SS_INT8) SS_QREG_C(true);
         else SS_QREG_C(false);

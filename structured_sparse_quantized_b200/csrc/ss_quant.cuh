@@ -305,8 +305,8 @@ __global__ void __launch_bounds__(kWarpRowThreads) prune_act_warp_kernel(
 // Single-pass variants for bf16 rows of up to kRegK elements: the whole row
 // sits in registers (16 bytes x 2 x 8 per lane), so X is read from HBM once.
 // ---------------------------------------------------------------------------
-constexpr int kRegChunks = 8;                 // 16-element chunks per lane
-constexpr int kRegK = 32 * 16 * kRegChunks;   // 4096 elements
+constexpr int kRegChunks = 8;                     // 16-element chunks per lane, at most
+constexpr int kRegK = 4 * 32 * 16 * kRegChunks;   // 16384 elements (4 warps per row)
 
 __device__ __forceinline__ void bf16x16_to_f32(const uint4& a, const uint4& b, float (&f)[16]) {
     const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
@@ -317,25 +317,36 @@ __device__ __forceinline__ void bf16x16_to_f32(const uint4& a, const uint4& b, f
     }
 }
 
-// Requires K % 16 == 0, K <= 512 * kChunks and a 16-byte aligned X.
-// kChunks = 16-element chunks per lane (rows of up to 512 kChunks values).
-template <bool kInt8, int kChunks>
+// Requires K % 16 == 0, K <= 512 * kChunks * kWpr and a 16-byte aligned X.
+// A row is held by kWpr warps (kWpr = 1, 2 or 4), each lane keeping kChunks
+// 16-element chunks: chunk c of the row sits with warp c / (32 kChunks), lane
+// c % 32.  The warps of a row combine their absmax through shared memory;
+// 256 / (32 kWpr) rows per CTA.
+template <bool kInt8, int kChunks, int kWpr = 1>
 __global__ void __launch_bounds__(kWarpRowThreads) quant_lift_reg_kernel(
     const __nv_bfloat16* __restrict__ X, int64_t M, int64_t K64, int Nh, int64_t K_lift64,
     int64_t K_lp64, int q_stride, uint8_t* __restrict__ Xq, float* __restrict__ s_x) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
+    constexpr int kRowsPerCta = kWarpRowThreads / (32 * kWpr);
+    __shared__ float part[kRowsPerCta][kWpr];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t m = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
+    const int slot = warp / kWpr;            // row slot of this CTA
+    const int sub = warp % kWpr;             // part of the row this warp holds
+    const int rt = sub * 32 + lane;          // thread index within the row
+    constexpr int kRowThreads = 32 * kWpr;
+    const int64_t m = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + slot;
+    // rows are whole per warp group, so a group leaves (or stays) together
     if (m >= M) return;
     const int K = static_cast<int>(K64);
     const int K_lift = static_cast<int>(K_lift64);
     const int K_lp = static_cast<int>(K_lp64);
     const uint4* xv = reinterpret_cast<const uint4*>(X + m * K64);
     const int n16 = K / 16;
+    const int c0 = sub * 32 * kChunks + lane;  // this lane's first chunk
     uint4 v[2 * kChunks];
 #pragma unroll
     for (int i = 0; i < kChunks; ++i) {
-        const int c = lane + 32 * i;
+        const int c = c0 + 32 * i;
         if (c < n16) {
             v[2 * i] = __ldcs(xv + 2 * c);
             v[2 * i + 1] = __ldcs(xv + 2 * c + 1);
@@ -349,22 +360,28 @@ __global__ void __launch_bounds__(kWarpRowThreads) quant_lift_reg_kernel(
     for (int i = 0; i < 2 * kChunks; ++i) a = fmaxf(a, chunk_absmax<__nv_bfloat16>(v[i]));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if constexpr (kWpr > 1) {
+        if (lane == 0) part[slot][sub] = a;
+        named_bar_sync(1 + slot, kRowThreads);
+#pragma unroll
+        for (int w = 0; w < kWpr; ++w) a = fmaxf(a, part[slot][w]);
+    }
     float inv, s;
     scale_from_absmax<kInt8>(a, inv, s);
-    if (lane == 0) s_x[m] = s;
+    if (rt == 0) s_x[m] = s;
     uint4* out = reinterpret_cast<uint4*>(Xq + m * K_lp64);
     const int n_chunks = K_lp / 16;
     if (Nh <= 2) {  // identity map: chunk c of the output is chunk c of the input
 #pragma unroll
         for (int i = 0; i < kChunks; ++i) {
-            const int c = lane + 32 * i;
+            const int c = c0 + 32 * i;
             if (c < n16) {
                 float f[16];
                 bf16x16_to_f32(v[2 * i], v[2 * i + 1], f);
                 __stcs(out + c, quant16<kInt8>(f, inv));
             }
         }
-        for (int c = n16 + lane; c < n_chunks; c += 32) __stcs(out + c, make_uint4(0, 0, 0, 0));
+        for (int c = n16 + rt; c < n_chunks; c += kRowThreads) __stcs(out + c, make_uint4(0, 0, 0, 0));
         return;
     }
     if (Nh == 4) {
@@ -373,7 +390,7 @@ __global__ void __launch_bounds__(kWarpRowThreads) quant_lift_reg_kernel(
         // codes: 24 lifted bytes at 24c, no other lane's data involved.
 #pragma unroll
         for (int i = 0; i < kChunks; ++i) {
-            const int c = lane + 32 * i;
+            const int c = c0 + 32 * i;
             if (c < n16) {
                 float f[16];
                 bf16x16_to_f32(v[2 * i], v[2 * i + 1], f);
@@ -386,26 +403,32 @@ __global__ void __launch_bounds__(kWarpRowThreads) quant_lift_reg_kernel(
         }
         // zero windows past the last group up to K_lp (8-byte aligned: K_lift = 24 K / 16)
         uint2* z = reinterpret_cast<uint2*>(Xq + m * K_lp64);
-        for (int c8 = K_lift / 8 + lane; c8 < K_lp / 8; c8 += 32) __stcs(z + c8, make_uint2(0, 0));
+        for (int c8 = K_lift / 8 + rt; c8 < K_lp / 8; c8 += kRowThreads)
+            __stcs(z + c8, make_uint2(0, 0));
         return;
     }
-    uint4* qrow = reinterpret_cast<uint4*>(smem_raw + warp * q_stride);
+    // 4:6, 8:10: the row's codes go to a shared-memory row, then each 16-byte
+    // output word gathers four windows from it
+    uint4* qrow = reinterpret_cast<uint4*>(smem_raw + slot * q_stride);
     const int q_chunks = ((K_lift / (4 * (Nh - 1))) * 2 * Nh + 15) / 16;
 #pragma unroll
     for (int i = 0; i < kChunks; ++i) {
-        const int c = lane + 32 * i;
+        const int c = c0 + 32 * i;
         if (c < n16) {
             float f[16];
             bf16x16_to_f32(v[2 * i], v[2 * i + 1], f);
             qrow[c] = quant16<kInt8>(f, inv);
         }
     }
-    for (int c = n16 + lane; c < q_chunks; c += 32) qrow[c] = make_uint4(0, 0, 0, 0);
-    __syncwarp();
+    for (int c = n16 + rt; c < q_chunks; c += kRowThreads) qrow[c] = make_uint4(0, 0, 0, 0);
+    if constexpr (kWpr > 1)
+        named_bar_sync(1 + slot, kRowThreads);
+    else
+        __syncwarp();
     const uint16_t* q16 = reinterpret_cast<const uint16_t*>(qrow);
     const uint32_t n_win = static_cast<uint32_t>(K_lift / 4);
     const uint32_t per_group = static_cast<uint32_t>(Nh - 1);
-    for (int c = lane; c < n_chunks; c += 32) {
+    for (int c = rt; c < n_chunks; c += kRowThreads) {
         uint32_t win = static_cast<uint32_t>(c) * 4u;
         uint32_t g = win / per_group;
         uint32_t j = win - g * per_group;

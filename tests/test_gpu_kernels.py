@@ -46,15 +46,18 @@ def test_prune_act_2to4(q, dt, M, K):
     np.testing.assert_array_equal(host(Xv), Xv_ref)
 
 
-# Many bf16 rows (several CTAs per SM, many warps per row stream) at the K
-# values of each register-resident variant (up to 2, 4, 6, 7 and 8 sixteen-
-# element chunks per lane), the 6:8 in-register lift with and without a zero
-# tail up to K_lp, and a K that takes the two-pass kernel.
+# Many bf16 rows (several CTAs per SM) at the K values of each register-
+# resident variant: 1 warp per row with up to 2, 4, 6, 7 and 8 sixteen-element
+# chunks per lane, 2 and 4 warps per row (K up to 16384) with 6, 7 and 8; the
+# 6:8 in-register lift with and without a zero tail up to K_lp; and a K that
+# takes the two-pass kernel.
 @pytest.mark.parametrize("pat", ["dense"] + PATTERNS)
 @pytest.mark.parametrize("q", ["int8", "fp8"])
-@pytest.mark.parametrize("K", [4096, 3584, 3072, 2048, 1040, 1032, 512])
-def test_quant_lift_act_many_rows(pat, q, K):
-    X = _x(3000, K, "bf16", seed=K)
+@pytest.mark.parametrize("M,K", [(1200, 16384), (1200, 14336), (1500, 8192), (1500, 5120),
+                                 (3000, 4096), (3000, 3584), (3000, 3072), (3000, 2048),
+                                 (3000, 1040), (3000, 1032), (3000, 512)])
+def test_quant_lift_act_many_rows(pat, q, M, K):
+    X = _x(M, K, "bf16", seed=K)
     Xq_ref, s_ref = oracle.quant_lift_act(X, pat, Q[q])
     Xq, s_x = ss.quant_lift_act(dev(X), pat, q)
     np.testing.assert_array_equal(host(s_x), s_ref)
