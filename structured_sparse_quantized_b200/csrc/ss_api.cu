@@ -160,12 +160,12 @@ ss_status dispatch_gemm(int dev, bool int8, bool bf16, const CUtensorMap& a, con
                 : launch_gemm<kSparse, false, false, kPair, kAT>(dev, a, b, e, y, args, st);
 }
 
-template <bool kInt8>
+template <bool kInt8, bool kAIsW>
 ss_status launch_gemm_wide(int dev, const CUtensorMap& a, const CUtensorMap& b,
                            const CUtensorMap& e, const CUtensorMap& y, const ss::GemmArgs& args,
                            cudaStream_t stream) {
     using C = ss::WideCfg;
-    auto kern = ss::gemm_sparse_wide_kernel<kInt8>;
+    auto kern = ss::gemm_sparse_wide_kernel<kInt8, kAIsW>;
     static std::once_flag once[kMaxDevices];
     static cudaError_t attr_err[kMaxDevices];
     std::call_once(once[dev], [&] {
@@ -534,10 +534,10 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
     cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
     const bool i8 = q == SS_INT8, bf = out_dtype == SS_OUT_BF16;
 #if SS_SPARSE_WIDE
-    // Large problems with channel rows and bf16 Y may take two B tiles per
-    // output tile: fewer bytes per MMA, but single-buffered accumulators.
+    // Large problems with bf16 Y may take two B tiles per output tile: fewer
+    // bytes per MMA, but single-buffered accumulators.
     const int forced = forced_sparse_kernel();
-    if (pair == 2 && args.a_is_w && args.tma_store && forced != 1 &&
+    if (pair == 2 && args.tma_store && forced != 1 &&
         (forced == 2 || (rowsB > 2 * ss::WideCfg::kBnMax &&
                          prefer_wide(rowsA, rowsB, bn, g_num_sms[dev] / 2)))) {
         using CW = ss::WideCfg;
@@ -550,8 +550,11 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
         ss::GemmArgs wargs = args;
         wargs.bn = bnw;
         wargs.k_stages = static_cast<int>(K_lp / CW::kStageK);
-        return i8 ? launch_gemm_wide<true>(dev, wa, wb, te, ty, wargs, st_)
-                  : launch_gemm_wide<false>(dev, wa, wb, te, ty, wargs, st_);
+        if (args.a_is_w)
+            return i8 ? launch_gemm_wide<true, true>(dev, wa, wb, te, ty, wargs, st_)
+                      : launch_gemm_wide<false, true>(dev, wa, wb, te, ty, wargs, st_);
+        return i8 ? launch_gemm_wide<true, false>(dev, wa, wb, te, ty, wargs, st_)
+                  : launch_gemm_wide<false, false>(dev, wa, wb, te, ty, wargs, st_);
     }
 #endif
     if (pair == 1) return dispatch_gemm<true, 1, 1>(dev, i8, bf, ta, tb, te, ty, args, st_);

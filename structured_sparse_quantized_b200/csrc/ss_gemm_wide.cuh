@@ -1,8 +1,10 @@
 // ss_gemm_wide.cuh -- the sparse GEMM of ss_gemm.cuh with output tiles two
-// B tiles wide, for large problems whose A rows are output channels.
+// B tiles wide, for large problems.
 //
 // Same operation, same operands, same epilogue arithmetic as gemm_kernel:
-//   D[a, b] = sum_k A[a, k] * B[b, k],  Y[b, a] = bf16(((float)D * s_b) * s_a)
+//   D[a, b] = sum_k A[a, k] * B[b, k]
+//   A = weight (rows = channels):   Y[b, a] = bf16(((float)D * s_b) * s_a)
+//   A = activation (rows = tokens): Y[a, b] = bf16(((float)D * s_a) * s_b)
 // (the sparse matmul after the sliding-window decomposition: SlideSparse
 // write-up, omica.com.cn, 2.2 sparse GEMM execution).
 //
@@ -82,7 +84,9 @@ __device__ __forceinline__ int snake_tile(int k, int unit, int n_units) {
     return k * n_units + ((k & 1) ? (n_units - 1 - unit) : unit);
 }
 
-template <bool kInt8>
+// kAIsW: A rows are output channels (weight-sparse, Y[b, a]); otherwise A
+// rows are tokens (activation-sparse, Y[a, b]).
+template <bool kInt8, bool kAIsW>
 __global__ void __launch_bounds__(kWideThreads, 1)
     gemm_sparse_wide_kernel(const __grid_constant__ CUtensorMap tm_a,
                             const __grid_constant__ CUtensorMap tm_b,
@@ -256,15 +260,18 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         // Warp w (2..9) drains TMEM lane quarter w % 4 of accumulator (w - 2) / 4,
-        // i.e. 32 channels x up to 224 tokens.  The tile's scales are fetched
-        // before its accumulators are ready (token scales through shared
+        // i.e. 32 A rows x up to 224 B rows.  The tile's scales are fetched
+        // before its accumulators are ready (B-row scales through shared
         // memory), so the drain itself only reads tensor and shared memory.
-        // Phase 1 reads every 32-token chunk as m8n8 fragments (tcgen05.ld
-        // 16x256b), scales, and keeps the packed bf16 pairs in registers; then
-        // the accumulator is released.  Phase 2 writes each chunk with
-        // stmatrix.trans into a 128B-swizzled [32 tokens][64 channels] pair of
-        // halves shared by the four warps of the B tile, stored by two TMA
-        // stores, while the next tile's MMAs run.
+        // Phase 1 reads every 32-column chunk, scales, and keeps the packed
+        // bf16 pairs in registers; then the accumulator is released.  Phase 2
+        // writes each chunk through shared memory with TMA stores while the
+        // next tile's MMAs run:
+        //   A = weight: m8n8 fragments (tcgen05.ld 16x256b) go through
+        //     stmatrix.trans into a 128B-swizzled [32 tokens][64 channels]
+        //     pair of halves shared by the four warps of the B tile;
+        //   A = activation: each thread's own token row (tcgen05.ld 32x32b)
+        //     goes to a [128 tokens][32 channels] box.
         constexpr int kChunks = C::kBnMax / 32;
         const int ew = warp - 2;
         const int et = ew * 32 + lane;  // 0..255
@@ -292,14 +299,22 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                 const int tok = tile_tok0 + j;
                 sb_pre[u] = (j < tile_b_rows && tok < args.rowsB) ? __ldg(args.s_b + tok) : 0.0f;
             }
+            // A-row scales: channel-row path, the m8n8 fragment rows of this
+            // thread; token-row path, this thread's own row
             float sa2[2][2];
+            float sa_row = 0.0f;
+            if constexpr (kAIsW) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+                for (int h = 0; h < 2; ++h)
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int ch = a_cta0 + q * 32 + 16 * h + t4 + 8 * e;
-                    sa2[h][e] = ch < args.rowsA ? __ldg(args.s_a + ch) : 0.0f;
-                }
+                    for (int e = 0; e < 2; ++e) {
+                        const int ch = a_cta0 + q * 32 + 16 * h + t4 + 8 * e;
+                        sa2[h][e] = ch < args.rowsA ? __ldg(args.s_a + ch) : 0.0f;
+                    }
+            } else {
+                const int ar = a_cta0 + q * 32 + lane;
+                sa_row = ar < args.rowsA ? __ldg(args.s_a + ar) : 0.0f;
+            }
             // all eight epilogue warps take the same decision, so none is left
             // behind at a named barrier if the wait gives up; passing it also
             // means every warp is done with the previous tile's token scales
@@ -313,38 +328,71 @@ __global__ void __launch_bounds__(kWideThreads, 1)
             const float* sb_tile = sb_smem + bt * args.bn;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    static_cast<uint32_t>(bt * C::kAccStride);
-            uint32_t pk[kChunks][2][8];  // [chunk][half][token group r * 2 + channel block]
+            uint32_t pk[kChunks][2][8];  // 16 packed bf16 pairs per chunk
+            if constexpr (kAIsW) {
+                // [chunk][half][token group r * 2 + channel block]
 #pragma unroll
-            for (int c = 0; c < kChunks; ++c) {
-                if (c * 32 < args.bn) {
-                    uint32_t v[2][16];
-                    tmem_ld_16x256b_x4(t_row + c * 32, v[0]);
-                    tmem_ld_16x256b_x4(t_row + (16u << 16) + c * 32, v[1]);
-                    // token scales of the chunk: tokens 8r + 2tm + {0, 1}
-                    float2 sb[4];
-#pragma unroll
-                    for (int r = 0; r < 4; ++r)
-                        sb[r] = *reinterpret_cast<const float2*>(sb_tile + c * 32 + 8 * r + 2 * tm);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
+                for (int c = 0; c < kChunks; ++c) {
+                    if (c * 32 < args.bn) {
+                        uint32_t v[2][16];
+                        tmem_ld_16x256b_x4(t_row + c * 32, v[0]);
+                        tmem_ld_16x256b_x4(t_row + (16u << 16) + c * 32, v[1]);
+                        // token scales of the chunk: tokens 8r + 2tm + {0, 1}
+                        float2 sb[4];
 #pragma unroll
                         for (int r = 0; r < 4; ++r)
+                            sb[r] =
+                                *reinterpret_cast<const float2*>(sb_tile + c * 32 + 8 * r + 2 * tm);
+                        tmem_ld_wait();
 #pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const uint32_t b0 = v[h][4 * r + 2 * e];
-                                const uint32_t b1 = v[h][4 * r + 2 * e + 1];
-                                const float x0 =
-                                    kInt8 ? __int2float_rn(static_cast<int32_t>(b0)) : __uint_as_float(b0);
-                                const float x1 =
-                                    kInt8 ? __int2float_rn(static_cast<int32_t>(b1)) : __uint_as_float(b1);
-                                // ((acc * s_b) * s_a), both products rounded to fp32
-                                float y0, y1;
-                                mul_rn_f32x2(x0, x1, sb[r].x, sb[r].y, y0, y1);
-                                mul_rn_f32x2(y0, y1, sa2[h][e], sa2[h][e], y0, y1);
-                                const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
-                                pk[c][h][2 * r + e] = *reinterpret_cast<const uint32_t*>(&b2);
-                            }
+                        for (int h = 0; h < 2; ++h)
+#pragma unroll
+                            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                                for (int e = 0; e < 2; ++e) {
+                                    const uint32_t b0 = v[h][4 * r + 2 * e];
+                                    const uint32_t b1 = v[h][4 * r + 2 * e + 1];
+                                    const float x0 = kInt8 ? __int2float_rn(static_cast<int32_t>(b0))
+                                                           : __uint_as_float(b0);
+                                    const float x1 = kInt8 ? __int2float_rn(static_cast<int32_t>(b1))
+                                                           : __uint_as_float(b1);
+                                    // ((acc * s_b) * s_a), both products rounded to fp32
+                                    float y0, y1;
+                                    mul_rn_f32x2(x0, x1, sb[r].x, sb[r].y, y0, y1);
+                                    mul_rn_f32x2(y0, y1, sa2[h][e], sa2[h][e], y0, y1);
+                                    const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
+                                    pk[c][h][2 * r + e] = *reinterpret_cast<const uint32_t*>(&b2);
+                                }
+                    }
+                }
+            } else {
+                // this thread's token row, 32 channels per chunk: [chunk][k / 8][k % 8]
+#pragma unroll
+                for (int c = 0; c < kChunks; ++c) {
+                    if (c * 32 < args.bn) {
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(t_row + c * 32, r);
+                        float4 sb[8];  // channel scales of the chunk
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            sb[k] = *reinterpret_cast<const float4*>(sb_tile + c * 32 + 4 * k);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {
+                            const float x0 = kInt8 ? __int2float_rn(static_cast<int32_t>(r[2 * k]))
+                                                   : __uint_as_float(r[2 * k]);
+                            const float x1 = kInt8 ? __int2float_rn(static_cast<int32_t>(r[2 * k + 1]))
+                                                   : __uint_as_float(r[2 * k + 1]);
+                            const float s0 = (k & 1) ? sb[k >> 1].z : sb[k >> 1].x;
+                            const float s1 = (k & 1) ? sb[k >> 1].w : sb[k >> 1].y;
+                            // ((acc * s_a) * s_b), both products rounded to fp32
+                            float y0, y1;
+                            mul_rn_f32x2(x0, x1, sa_row, sa_row, y0, y1);
+                            mul_rn_f32x2(y0, y1, s0, s1, y0, y1);
+                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
+                            pk[c][k >> 3][k & 7] = *reinterpret_cast<const uint32_t*>(&b2);
+                        }
+                    }
                 }
             }
             tc_fence_before();
@@ -357,29 +405,43 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                     if (issuer) bulk_wait_read<1>();  // the stores of two chunks ago have read it
                     named_bar_sync(grp_bar, 128);
                     const uint32_t sy_u32 = smem_u32(sy);
+                    if constexpr (kAIsW) {
 #pragma unroll
-                    for (int h = 0; h < 2; ++h)
+                        for (int h = 0; h < 2; ++h)
 #pragma unroll
-                        for (int rp = 0; rp < 2; ++rp) {
-                            // matrices: (r = 2rp, e = 0), (2rp, 1), (2rp+1, 0), (2rp+1, 1)
-                            const int r = 2 * rp + (mi >> 1);
-                            const int e = mi & 1;
-                            const int tok = 8 * r + mj;              // row of the chunk
-                            const int ch = q * 32 + 16 * h + 8 * e;  // 8-channel block
-                            const int half = ch >> 6;
-                            const int blk = (ch & 63) >> 3;
-                            const uint32_t addr =
-                                sy_u32 + half * (32 * 128) + tok * 128 + ((blk ^ (tok & 7)) << 4);
-                            stmatrix_x4_trans(addr, pk[c][h][4 * rp + 0], pk[c][h][4 * rp + 1],
-                                              pk[c][h][4 * rp + 2], pk[c][h][4 * rp + 3]);
-                        }
+                            for (int rp = 0; rp < 2; ++rp) {
+                                // matrices: (r = 2rp, e = 0), (2rp, 1), (2rp+1, 0), (2rp+1, 1)
+                                const int r = 2 * rp + (mi >> 1);
+                                const int e = mi & 1;
+                                const int tok = 8 * r + mj;              // row of the chunk
+                                const int ch = q * 32 + 16 * h + 8 * e;  // 8-channel block
+                                const int half = ch >> 6;
+                                const int blk = (ch & 63) >> 3;
+                                const uint32_t addr = sy_u32 + half * (32 * 128) + tok * 128 +
+                                                      ((blk ^ (tok & 7)) << 4);
+                                stmatrix_x4_trans(addr, pk[c][h][4 * rp + 0], pk[c][h][4 * rp + 1],
+                                                  pk[c][h][4 * rp + 2], pk[c][h][4 * rp + 3]);
+                            }
+                    } else {
+                        // [128 token rows][32 channels]: this thread's row is 64 bytes
+                        uint4* dst = reinterpret_cast<uint4*>(sy + (q * 32 + lane) * 64);
+#pragma unroll
+                        for (int w = 0; w < 4; ++w)
+                            dst[w] = make_uint4(pk[c][w >> 1][4 * (w & 1)], pk[c][w >> 1][4 * (w & 1) + 1],
+                                                pk[c][w >> 1][4 * (w & 1) + 2],
+                                                pk[c][w >> 1][4 * (w & 1) + 3]);
+                    }
                     fence_async_shared();
                     named_bar_sync(grp_bar, 128);
                     if (issuer) {
                         const uint64_t stream = l2_policy_evict_first();
-                        tma_store_2d_hint(&tm_y, sy, a_cta0, tok0 + c * 32, stream);
-                        tma_store_2d_hint(&tm_y, sy + 32 * 128, a_cta0 + 64, tok0 + c * 32,
-                                          stream);
+                        if constexpr (kAIsW) {
+                            tma_store_2d_hint(&tm_y, sy, a_cta0, tok0 + c * 32, stream);
+                            tma_store_2d_hint(&tm_y, sy + 32 * 128, a_cta0 + 64, tok0 + c * 32,
+                                              stream);
+                        } else {
+                            tma_store_2d_hint(&tm_y, sy, tok0 + c * 32, a_cta0, stream);
+                        }
                         bulk_commit_group();
                     }
                     ++chunk_iter;

@@ -175,6 +175,27 @@ def test_sparse_gemm_wide_tiles(M, N, K, pat, nrows, q, kernel, monkeypatch):
     assert_y_matches(Y if rows is None else Y[rows], Y_ref, q, True)
 
 
+# Activation-sparse shapes (A = pruned X, token rows) on both kernel shapes.
+@pytest.mark.parametrize("M,N,K", [(1000, 520, 1024), (300, 2000, 768), (2049, 4096, 512),
+                                   (8192, 1400, 256)])
+@pytest.mark.parametrize("q", ["int8", "fp8"])
+@pytest.mark.parametrize("kernel", ["wide", "narrow"])
+def test_sparse_gemm_activation_sparse_tiles(M, N, K, q, kernel, monkeypatch):
+    monkeypatch.setenv("SS_SPARSE_KERNEL", kernel)
+    W = synth.gaussian((N, K), std=0.02, seed=0, dtype=torch.bfloat16)
+    X = synth.gaussian_with_heavy_tails(M, K, seed=1)
+    Xv, Xm, s_x = oracle.prune_act_2to4(X, Q[q])
+    Wq, _, s_w = oracle.compress_weight(W, "dense", Q[q])
+    K_lp = oracle.act_2to4_k_lp(K)
+    rows = synth.sample_rows(M, seed=3, middle=200)
+    Y_ref = oracle.sparse_gemm(1, Xv, Xm, s_x, Wq, s_w, M, N, K_lp, Q[q], oracle.OUT_BF16,
+                               m_idx=rows)
+    Y = host(ss.sparse_gemm(1, dev(Xv), dev(oracle.meta_to_tiles(Xm, K_lp)), dev(s_x), dev(Wq),
+                            dev(s_w), M, N, q))
+    assert ss.ss_get_device_status() == ss.SS_OK
+    assert_y_matches(Y[rows], Y_ref, q, True)
+
+
 @pytest.mark.parametrize("M,N,K", [(130, 64, 256), (257, 300, 1024), (8, 96, 4096)])
 @pytest.mark.parametrize("q", ["int8", "fp8"])
 def test_sparse_gemm_activation_sparse(M, N, K, q):
