@@ -113,11 +113,11 @@ bool make_y_map(CUtensorMap* map, void* Y, int64_t M, int64_t N, bool out_bf16, 
                   : make_map_2d(map, Y, M, N, ss::kTileA, 32, CU_TENSOR_MAP_SWIZZLE_NONE, dt, esz);
 }
 
-template <bool kSparse, bool kInt8, bool kOutBf16, int kPair, int kAT>
+template <bool kSparse, bool kInt8, bool kOutBf16, int kPair>
 ss_status launch_gemm(int dev, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& e,
                       const CUtensorMap& y, const ss::GemmArgs& args, cudaStream_t stream) {
-    using C = ss::GemmCfg<kSparse, kPair, kAT>;
-    auto kern = ss::gemm_kernel<kSparse, kInt8, kOutBf16, kPair, kAT>;
+    using C = ss::GemmCfg<kSparse, kPair>;
+    auto kern = ss::gemm_kernel<kSparse, kInt8, kOutBf16, kPair>;
     static std::once_flag once[kMaxDevices];
     static cudaError_t attr_err[kMaxDevices];
     std::call_once(once[dev], [&] {
@@ -125,7 +125,7 @@ ss_status launch_gemm(int dev, const CUtensorMap& a, const CUtensorMap& b, const
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     });
     if (attr_err[dev] != cudaSuccess) return SS_ERR_CUDA;
-    const int64_t tile_rows = static_cast<int64_t>(ss::kTileA) * kPair * kAT;
+    const int64_t tile_rows = static_cast<int64_t>(ss::kTileA) * kPair;
     const int64_t tiles =
         ((args.rowsA + tile_rows - 1) / tile_rows) * ((args.rowsB + args.bn - 1) / args.bn);
     const int64_t units = g_num_sms[dev] / kPair;
@@ -149,15 +149,15 @@ ss_status launch_gemm(int dev, const CUtensorMap& a, const CUtensorMap& b, const
     return launched();
 }
 
-template <bool kSparse, int kPair, int kAT>
+template <bool kSparse, int kPair>
 ss_status dispatch_gemm(int dev, bool int8, bool bf16, const CUtensorMap& a, const CUtensorMap& b,
                         const CUtensorMap& e, const CUtensorMap& y, const ss::GemmArgs& args,
                         cudaStream_t st) {
     if (int8)
-        return bf16 ? launch_gemm<kSparse, true, true, kPair, kAT>(dev, a, b, e, y, args, st)
-                    : launch_gemm<kSparse, true, false, kPair, kAT>(dev, a, b, e, y, args, st);
-    return bf16 ? launch_gemm<kSparse, false, true, kPair, kAT>(dev, a, b, e, y, args, st)
-                : launch_gemm<kSparse, false, false, kPair, kAT>(dev, a, b, e, y, args, st);
+        return bf16 ? launch_gemm<kSparse, true, true, kPair>(dev, a, b, e, y, args, st)
+                    : launch_gemm<kSparse, true, false, kPair>(dev, a, b, e, y, args, st);
+    return bf16 ? launch_gemm<kSparse, false, true, kPair>(dev, a, b, e, y, args, st)
+                : launch_gemm<kSparse, false, false, kPair>(dev, a, b, e, y, args, st);
 }
 
 template <bool kInt8, bool kAIsW>
@@ -506,12 +506,11 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
     const int64_t rowsA = sparse_operand == 0 ? N : M;
     const int64_t rowsB = sparse_operand == 0 ? M : N;
     const int pair = rowsA > ss::kTileA ? 2 : 1;
-    const int bn = choose_bn(rowsB, ss::GemmCfg<true, 1, 1>::kBnMax);
+    const int bn = choose_bn(rowsB, ss::GemmCfg<true, 1>::kBnMax);
     CUtensorMap ta, tb, te;
-    using CS = ss::GemmCfg<true, 1, 1>;
+    using CS = ss::GemmCfg<true, 1>;
     if (!make_map_2d(&ta, Av, rowsA, K_lp / 2, ss::kTileA, CS::kARowBytes,
-                     CS::kARowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
-                                           : CU_TENSOR_MAP_SWIZZLE_64B) ||
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&tb, B, rowsB, K_lp, bn / pair, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&te, Am, (rowsA + 127) / 128 * (K_lp / 128) * 16, 128, 16, 128,
                      CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -557,8 +556,8 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
                   : launch_gemm_wide<false, false>(dev, wa, wb, te, ty, wargs, st_);
     }
 #endif
-    if (pair == 1) return dispatch_gemm<true, 1, 1>(dev, i8, bf, ta, tb, te, ty, args, st_);
-    return dispatch_gemm<true, 2, SS_SPARSE_A_TILES>(dev, i8, bf, ta, tb, te, ty, args, st_);
+    if (pair == 1) return dispatch_gemm<true, 1>(dev, i8, bf, ta, tb, te, ty, args, st_);
+    return dispatch_gemm<true, 2>(dev, i8, bf, ta, tb, te, ty, args, st_);
 }
 
 ss_status ss_dense_gemm(const void* Xq, const float* s_x, const void* Wq, const float* s_w,
@@ -575,7 +574,7 @@ ss_status ss_dense_gemm(const void* Xq, const float* s_x, const void* Wq, const 
     ss_status st = check_device(&dev);
     if (st != SS_OK) return st;
     const int pair = N > ss::kTileA ? 2 : 1;
-    const int bn = choose_bn(M, ss::GemmCfg<false, 1, 1>::kBnMax);
+    const int bn = choose_bn(M, ss::GemmCfg<false, 1>::kBnMax);
     CUtensorMap ta, tb;
     if (!make_map_2d(&ta, Wq, N, K_p, ss::kTileA, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&tb, Xq, M, K_p, bn / pair, 128, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -595,8 +594,8 @@ ss_status ss_dense_gemm(const void* Xq, const float* s_x, const void* Wq, const 
     if (!args.tma_store) ty = ta;  // unused
     cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
     const bool i8 = q == SS_INT8, bf = out_dtype == SS_OUT_BF16;
-    return pair == 2 ? dispatch_gemm<false, 2, 1>(dev, i8, bf, ta, tb, ta, ty, args, st_)
-                     : dispatch_gemm<false, 1, 1>(dev, i8, bf, ta, tb, ta, ty, args, st_);
+    return pair == 2 ? dispatch_gemm<false, 2>(dev, i8, bf, ta, tb, ta, ty, args, st_)
+                     : dispatch_gemm<false, 1>(dev, i8, bf, ta, tb, ta, ty, args, st_);
 }
 
 ss_status ss_get_device_status(ss_stream_t stream) {

@@ -19,13 +19,9 @@
 // the sparse MMA run at twice the dense rate.  D is split by A rows between
 // the two tensor memories.  kPair = 1 is the single-SM form (M = 128).
 //
-// kAT = number of 256-row A tiles a pair covers per output tile (sparse
-// only).  With kAT = 2 every B stage feeds two A tiles, so the bytes a stage
-// must bring in per MAC fall by ~1.4x -- the sparse mainloop is bound by the
-// bytes in flight that shared memory can hold.  The two A tiles' accumulators
-// then fill tensor memory, so they are single-buffered: the epilogue drains
-// accumulator 0 first and the next tile's A-tile-0 MMAs start as soon as it
-// is free.  kAT = 1 double-buffers one accumulator.
+// The accumulator is double-buffered in tensor memory: the epilogue drains
+// one tile while the MMAs of the next fill the other buffer.  (For large
+// problems the sparse GEMM also has a two-B-tile shape, ss_gemm_wide.cuh.)
 //
 // CTA = 6 warps, one CTA per SM, persistent over output tiles:
 //   warp 0       TMA producer (whole warp, one elected lane issues): A tiles,
@@ -52,31 +48,16 @@ constexpr int kGemmThreads = 192;
 constexpr int kTileA = 128;  // A rows per CTA per A tile
 constexpr int kTmemCols = 512;
 
-// Logical K of one sparse pipeline stage: 256 (A rows of 128 compressed bytes
-// in 128B swizzle, two B atoms, two metadata chunks, four MMAs per A tile) or
-// 128 (A rows of 64 bytes in 64B swizzle, one B atom, one metadata chunk, two
-// MMAs per A tile, twice as many stages in flight).
-#ifndef SS_SPARSE_STAGE_K
-#define SS_SPARSE_STAGE_K 256
-#endif
-
-// 256-row A tiles per sparse output tile (1 or 2).  Two halve the B bytes per
-// MAC but single-buffer the accumulators; measured on B200 the exposed
-// epilogue costs more than the bandwidth saves, so one is the default.
-#ifndef SS_SPARSE_A_TILES
-#define SS_SPARSE_A_TILES 1
-#endif
-
-template <bool kSparse, int kPair, int kAT = 1>
+template <bool kSparse, int kPair>
 struct GemmCfg {
     // One pipeline stage covers kStageK logical K: dense 128 (4 MMAs of K=32),
-    // sparse SS_SPARSE_STAGE_K (MMAs of K=64).
-    static constexpr int kStageK = kSparse ? SS_SPARSE_STAGE_K : 128;
+    // sparse 256 (4 MMAs of K=64).  Either way an A row holds 128 bytes of the
+    // stage (128B swizzle).
+    static constexpr int kStageK = kSparse ? 256 : 128;
     static constexpr int kMmaK = kSparse ? 64 : 32;
-    static constexpr int kMmaPerStage = kStageK / kMmaK;   // per A tile
-    static constexpr int kARowBytes = kSparse ? kStageK / 2 : kStageK;  // 64 or 128
-    static constexpr uint32_t kASwizzle = kARowBytes == 128 ? kSwizzle128B : kSwizzle64B;
-    static constexpr int kABytes = kTileA * kARowBytes;    // one A tile, 16 KB (or 8 KB)
+    static constexpr int kMmaPerStage = kStageK / kMmaK;
+    static constexpr int kARowBytes = kSparse ? kStageK / 2 : kStageK;  // 128
+    static constexpr int kABytes = kTileA * kARowBytes;    // one A tile, 16 KB
     static constexpr int kBAtoms = kStageK / 128;          // 128-byte K atoms of B per stage
     static constexpr int kBnMax = kSparse ? 224 : 256;     // MMA N; accumulators + metadata
     static constexpr int kBRowsMax = kBnMax / kPair;       // B rows held per CTA
@@ -84,10 +65,10 @@ struct GemmCfg {
     static constexpr int kBBytes = kBAtoms * kBAtomBytes;
     static constexpr int kEChunks = kSparse ? kStageK / 128 : 0;  // 16-byte chunks per A row
     static constexpr int kEBytes = kEChunks * kTileA * 16;  // one A tile
-    // stage layout: [A tile 0 .. A tile kAT-1 | B atoms | E tile 0 .. kAT-1]
-    static constexpr int kBOffset = kAT * kABytes;
+    // stage layout: [A tile | B atoms | E chunks]
+    static constexpr int kBOffset = kABytes;
     static constexpr int kEOffset = kBOffset + kBBytes;
-    static constexpr int kStageRaw = kEOffset + kAT * kEBytes;
+    static constexpr int kStageRaw = kEOffset + kEBytes;
     static constexpr int kStageBytes = (kStageRaw + 1023) / 1024 * 1024;
     static constexpr int kEpiBytes = 32 * kTileA * 2;      // one 32-column bf16 chunk of Y
     static constexpr int kSmemBudget = 225 * 1024 - 1024 - 256 - 2 * kEpiBytes;
@@ -95,14 +76,13 @@ struct GemmCfg {
     static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
     static constexpr int kAccStride = kBnMax;              // TMEM columns between accumulators
     static constexpr int kECol = 2 * kBnMax;               // metadata columns (sparse)
-    static constexpr int kESlotCols = 4 * kEChunks * kAT;  // columns one stage's metadata takes
+    static constexpr int kESlotCols = 4 * kEChunks;        // columns one stage's metadata takes
     // one metadata slot per stage: a slot is rewritten only after its stage's
     // "empty" commit, i.e. after the MMAs that read it completed
     static constexpr int kESlots = kStages;
     static constexpr int kEpiOffset = kStages * kStageBytes;  // 2 staging buffers for Y chunks
     static constexpr int kSmemBytes =
         kEpiOffset + 2 * kEpiBytes + 1024 /*align*/ + 256 /*barriers*/;
-    static_assert(kAT == 1 || (kSparse && kPair == 2), "two A tiles: sparse pair form only");
     static_assert(kABytes % 1024 == 0 && kBAtomBytes % 1024 == 0, "tile alignment");
     static_assert(!kSparse || kECol + kESlots * kESlotCols <= kTmemCols, "TMEM budget");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -137,18 +117,18 @@ __device__ __forceinline__ void store_scaled(void* y, int64_t off, uint32_t acc_
         reinterpret_cast<float*>(y)[off] = v;
 }
 
-template <bool kSparse, bool kInt8, bool kOutBf16, int kPair, int kAT>
+template <bool kSparse, bool kInt8, bool kOutBf16, int kPair>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_e, const __grid_constant__ CUtensorMap tm_y,
                 const GemmArgs args) {
-    using C = GemmCfg<kSparse, kPair, kAT>;
+    using C = GemmCfg<kSparse, kPair>;
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kEpiOffset + 2 * C::kEpiBytes);
     uint64_t* empty = full + C::kStages;
-    uint64_t* acc_full = empty + C::kStages;  // [2]: buffers (kAT = 1) or A tiles (kAT = 2)
+    uint64_t* acc_full = empty + C::kStages;  // [2]: one per accumulator buffer
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drain = acc_empty + 2;
     uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -160,7 +140,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t rank = kPair == 2 ? cluster_ctarank() : 0u;
     const bool leader = rank == 0;
     const int pair_rows = kTileA * kPair;     // A rows one MMA covers
-    const int tile_a_rows = pair_rows * kAT;  // A rows of one output tile
+    const int tile_a_rows = pair_rows;        // A rows of one output tile
     const int b_rows_cta = args.bn / kPair;
     const int nA = (args.rowsA + tile_a_rows - 1) / tile_a_rows;
     const int nB = (args.rowsB + args.bn - 1) / args.bn;
@@ -207,7 +187,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         __syncwarp();
         const uint32_t tx =
-            kPair * (kAT * (C::kABytes + C::kEBytes) + C::kBAtoms * b_rows_cta * 128);
+            kPair * (C::kABytes + C::kEBytes + C::kBAtoms * b_rows_cta * 128);
         int s = 0;
         uint32_t ph = 0, armed = 0, armed_par = 0;
         bool ok = true;
@@ -225,24 +205,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         if (leader) mbar_arrive_expect_tx(&full[s], tx);
                         const uint32_t fb = map_to_rank(&full[s], 0);
                         const uint64_t keep = l2_policy_evict_last();
-#pragma unroll
-                        for (int at = 0; at < kAT; ++at)
-                            tma_load_2d_pair_hint(st + at * C::kABytes, &tm_a, fb,
-                                                  kb * C::kARowBytes, a0 + at * pair_rows, keep);
+                        tma_load_2d_pair_hint(st, &tm_a, fb, kb * C::kARowBytes, a0, keep);
 #pragma unroll
                         for (int u = 0; u < C::kBAtoms; ++u)
                             tma_load_2d_pair_hint(st + C::kBOffset + u * C::kBAtomBytes, &tm_b,
                                                   fb, kb * C::kStageK + u * 128, b0, keep);
 #pragma unroll
-                        for (int at = 0; at < kAT; ++at)
-#pragma unroll
-                            for (int u = 0; u < C::kEChunks; ++u)
-                                tma_load_2d_pair_hint(
-                                    st + C::kEOffset + at * C::kEBytes + u * kTileA * 16, &tm_e,
-                                    fb, 0,
-                                    (((a0 + at * pair_rows) >> 7) * args.e_chunks +
-                                     kb * C::kEChunks + u) * 16,
-                                    keep);
+                        for (int u = 0; u < C::kEChunks; ++u)
+                            tma_load_2d_pair_hint(st + C::kEOffset + u * kTileA * 16, &tm_e, fb, 0,
+                                                  ((a0 >> 7) * args.e_chunks + kb * C::kEChunks + u) * 16,
+                                                  keep);
                     } else {
                         mbar_arrive_expect_tx(&full[s], tx);
                         tma_load_2d(st, &tm_a, &full[s], kb * C::kARowBytes, a0);
@@ -282,7 +254,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (leader) {
             const uint32_t idesc = make_idesc(kSparse, kInt8, pair_rows, args.bn);
             const uint32_t base = smem_u32(smem);
-            const uint64_t a_desc0 = smem_desc(base, 16, 8 * C::kARowBytes, C::kASwizzle);
+            const uint64_t a_desc0 = smem_desc(base, 16, 8 * C::kARowBytes, kSwizzle128B);
             const uint64_t b_desc0 = smem_desc(base + C::kBOffset, 16, 1024, kSwizzle128B);
             const uint64_t e_desc0 =
                 smem_desc(base + C::kEOffset, 128 * 16, 128, kSwizzleNone);
@@ -291,10 +263,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             bool ok = true;
             int i = 0;
             for (int t = unit; t < n_tiles && ok; t += n_units, ++i) {
-                // kAT = 1: double-buffered accumulator i & 1; kAT = 2: accumulator
-                // at = A tile, single-buffered, one phase per tile.
-                const int buf = kAT == 1 ? (i & 1) : 0;
-                const uint32_t aph = kAT == 1 ? ((i >> 1) & 1) : (i & 1);
+                // double-buffered accumulator: buffer i & 1, one phase per use
+                const int buf = i & 1;
+                const uint32_t aph = (i >> 1) & 1;
                 if (!__all_sync(0xffffffffu, mbar_wait(&acc_empty[buf], aph ^ 1u, abort_flag))) {
                     ok = false;
                     break;
@@ -309,47 +280,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint64_t soff = static_cast<uint64_t>((s * C::kStageBytes) >> 4);
                     const uint32_t e_tmem =
                         tmem_base + C::kECol + C::kESlotCols * s;
+                    const uint32_t d_tmem = tmem_base + buf * C::kAccStride;
+                    if (elect_one()) {
+                        if constexpr (kSparse) {
 #pragma unroll
-                    for (int at = 0; at < kAT; ++at) {
-                        if (kAT == 2 && at == 1 && kb == 0) {  // A tile 1's accumulator drained?
-                            if (!__all_sync(0xffffffffu,
-                                            mbar_wait(&acc_empty[1], aph ^ 1u, abort_flag))) {
-                                ok = false;
-                                break;
+                            for (int u = 0; u < C::kEChunks; ++u)
+                                tc_cp_128x128b_g<kPair>(e_tmem + 4 * u,
+                                                        e_desc0 + soff + ((u * kTileA * 16) >> 4));
+#pragma unroll
+                            for (int j = 0; j < C::kMmaPerStage; ++j) {
+                                const uint64_t a_desc = a_desc0 + soff + ((j * 32) >> 4);
+                                const uint64_t b_desc =
+                                    b_desc0 + soff +
+                                    (((j >> 1) * C::kBAtomBytes + (j & 1) * 64) >> 4);
+                                mma_sparse_g<kPair, kInt8>(d_tmem, a_desc, b_desc, e_tmem + 2 * j,
+                                                           idesc, (kb > 0 || j > 0) ? 1u : 0u);
                             }
-                            tc_fence_after();
-                        }
-                        const uint32_t d_tmem = tmem_base + (buf + at) * C::kAccStride;
-                        if (elect_one()) {
-                            if constexpr (kSparse) {
-                                const uint32_t e_at = e_tmem + at * 4 * C::kEChunks;
+                        } else {
 #pragma unroll
-                                for (int u = 0; u < C::kEChunks; ++u)
-                                    tc_cp_128x128b_g<kPair>(
-                                        e_at + 4 * u,
-                                        e_desc0 + soff + ((at * C::kEBytes + u * kTileA * 16) >> 4));
-#pragma unroll
-                                for (int j = 0; j < C::kMmaPerStage; ++j) {
-                                    const uint64_t a_desc =
-                                        a_desc0 + soff + ((at * C::kABytes + j * 32) >> 4);
-                                    const uint64_t b_desc =
-                                        b_desc0 + soff +
-                                        (((j >> 1) * C::kBAtomBytes + (j & 1) * 64) >> 4);
-                                    mma_sparse_g<kPair, kInt8>(d_tmem, a_desc, b_desc, e_at + 2 * j,
-                                                               idesc, (kb > 0 || j > 0) ? 1u : 0u);
-                                }
-                            } else {
-#pragma unroll
-                                for (int j = 0; j < C::kMmaPerStage; ++j) {
-                                    const uint64_t a_desc = a_desc0 + soff + ((j * 32) >> 4);
-                                    const uint64_t b_desc = b_desc0 + soff + ((j * 32) >> 4);
-                                    mma_dense_g<kPair, kInt8>(d_tmem, a_desc, b_desc, idesc,
-                                                              (kb > 0 || j > 0) ? 1u : 0u);
-                                }
+                            for (int j = 0; j < C::kMmaPerStage; ++j) {
+                                const uint64_t a_desc = a_desc0 + soff + ((j * 32) >> 4);
+                                const uint64_t b_desc = b_desc0 + soff + ((j * 32) >> 4);
+                                mma_dense_g<kPair, kInt8>(d_tmem, a_desc, b_desc, idesc,
+                                                          (kb > 0 || j > 0) ? 1u : 0u);
                             }
                         }
-                        __syncwarp();
                     }
+                    __syncwarp();
                     if (!ok) break;
                     if (elect_one()) tc_commit_g<kPair>(&empty[s]);  // stage free in both CTAs
                     __syncwarp();
@@ -359,10 +316,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
                 if (!ok) break;
-                if (elect_one()) {
-                    tc_commit_g<kPair>(&acc_full[buf]);
-                    if (kAT == 2) tc_commit_g<kPair>(&acc_full[1]);
-                }
+                if (elect_one()) tc_commit_g<kPair>(&acc_full[buf]);
                 __syncwarp();
             }
             if (!ok) {  // wait for every MMA already issued before TMEM is freed
@@ -392,117 +346,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int t = unit; t < n_tiles && ok; t += n_units, ++i) {
             const int a_tile0 = (t % nA) * tile_a_rows + static_cast<int>(rank) * kTileA;
             const int b0 = (t / nA) * args.bn;
-            for (int at = 0; at < kAT; ++at) {
-                const int acc = kAT == 1 ? (i & 1) : at;
-                const uint32_t aph = kAT == 1 ? ((i >> 1) & 1) : (i & 1);
-                // all four epilogue warps take the same decision, so none is left
-                // behind at a named barrier if the wait gives up
-                const bool got = mbar_wait(&acc_full[acc], aph, abort_flag);
-                if (!named_bar_and(1, 128, got)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const int a_cta0 = a_tile0 + at * pair_rows;
-                const int a_row = a_cta0 + lane_row;
-                const bool row_ok = a_row < args.rowsA;
-                const float sa = row_ok ? __ldg(args.s_a + a_row) : 0.0f;
-                const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                                       static_cast<uint32_t>(acc * C::kAccStride);
-                if (args.tma_store && args.a_is_w) {
-                    // Transposed store path.  Each warp reads its 32 channels x 32
-                    // tokens of a chunk as m8n8 fragments (two 16-lane halves),
-                    // scales them, packs bf16 pairs and writes 8x8 blocks with
-                    // stmatrix.trans into [token][channel] staging, 128B-swizzled
-                    // in two 64-channel halves, stored by two TMA stores.
-                    const int t4 = lane >> 2, tm = lane & 3;
-                    float sa2[2][2];
+            const int acc = i & 1;
+            const uint32_t aph = (i >> 1) & 1;
+            // all four epilogue warps take the same decision, so none is left
+            // behind at a named barrier if the wait gives up
+            const bool got = mbar_wait(&acc_full[acc], aph, abort_flag);
+            if (!named_bar_and(1, 128, got)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const int a_cta0 = a_tile0;
+            const int a_row = a_cta0 + lane_row;
+            const bool row_ok = a_row < args.rowsA;
+            const float sa = row_ok ? __ldg(args.s_a + a_row) : 0.0f;
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   static_cast<uint32_t>(acc * C::kAccStride);
+            if (args.tma_store && args.a_is_w) {
+                // Transposed store path.  Each warp reads its 32 channels x 32
+                // tokens of a chunk as m8n8 fragments (two 16-lane halves),
+                // scales them, packs bf16 pairs and writes 8x8 blocks with
+                // stmatrix.trans into [token][channel] staging, 128B-swizzled
+                // in two 64-channel halves, stored by two TMA stores.
+                const int t4 = lane >> 2, tm = lane & 3;
+                float sa2[2][2];
 #pragma unroll
-                    for (int h = 0; h < 2; ++h)
+                for (int h = 0; h < 2; ++h)
 #pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int ch = a_cta0 + q * 32 + 16 * h + t4 + 8 * e;
-                            sa2[h][e] = ch < args.rowsA ? __ldg(args.s_a + ch) : 0.0f;
-                        }
-                    // this thread's stmatrix row: matrix mi, row mj
-                    const int mi = lane >> 3, mj = lane & 7;
-                    for (int c = 0; c < args.bn; c += 32) {
-                        uint32_t v[2][16];
-                        tmem_ld_16x256b_x4(t_row + c, v[0]);
-                        tmem_ld_16x256b_x4(t_row + (16u << 16) + c, v[1]);
-                        tmem_ld_wait();
-                        if (c + 32 >= args.bn) {  // last read of this accumulator: release it
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) {
-                                if constexpr (kPair == 2)
-                                    mbar_arrive_cluster(acc_empty_leader + acc * sizeof(uint64_t));
-                                else
-                                    mbar_arrive(&acc_empty[acc]);
-                            }
-                        }
-                        float sb[4][2];
-#pragma unroll
-                        for (int r = 0; r < 4; ++r)
-#pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const int tok = b0 + c + 8 * r + 2 * tm + e;
-                                sb[r][e] = tok < args.rowsB ? __ldg(args.s_b + tok) : 0.0f;
-                            }
-                        uint32_t pk[2][8];  // [half][column group r * 2 + channel block]
-#pragma unroll
-                        for (int h = 0; h < 2; ++h)
-#pragma unroll
-                            for (int r = 0; r < 4; ++r)
-#pragma unroll
-                                for (int e = 0; e < 2; ++e) {
-                                    float y2[2];
-#pragma unroll
-                                    for (int k = 0; k < 2; ++k) {
-                                        const uint32_t bits = v[h][4 * r + 2 * e + k];
-                                        const float accv =
-                                            kInt8 ? __int2float_rn(static_cast<int32_t>(bits))
-                                                  : __uint_as_float(bits);
-                                        y2[k] = __fmul_rn(__fmul_rn(accv, sb[r][k]), sa2[h][e]);
-                                    }
-                                    const __nv_bfloat162 b2 = __floats2bfloat162_rn(y2[0], y2[1]);
-                                    pk[h][2 * r + e] = *reinterpret_cast<const uint32_t*>(&b2);
-                                }
-                        uint8_t* sy = stage_y + (chunk_iter & 1) * C::kEpiBytes;
-                        if (issuer) bulk_wait_read<1>();  // the stores of two chunks ago have read it
-                        named_bar_sync(1, 128);
-                        const uint32_t sy_u32 = smem_u32(sy);
-#pragma unroll
-                        for (int h = 0; h < 2; ++h)
-#pragma unroll
-                            for (int rp = 0; rp < 2; ++rp) {
-                                // matrices: (r = 2rp, e = 0), (2rp, 1), (2rp+1, 0), (2rp+1, 1)
-                                const int r = 2 * rp + (mi >> 1);
-                                const int e = mi & 1;
-                                const int tok = 8 * r + mj;                 // row of the chunk
-                                const int ch = q * 32 + 16 * h + 8 * e;     // 8-channel block
-                                const int half = ch >> 6;
-                                const int blk = (ch & 63) >> 3;
-                                const uint32_t addr = sy_u32 + half * (32 * 128) + tok * 128 +
-                                                      ((blk ^ (tok & 7)) << 4);
-                                stmatrix_x4_trans(addr, pk[h][4 * rp + 0], pk[h][4 * rp + 1],
-                                                  pk[h][4 * rp + 2], pk[h][4 * rp + 3]);
-                            }
-                        fence_async_shared();
-                        named_bar_sync(1, 128);
-                        if (issuer) {
-                            const uint64_t stream = l2_policy_evict_first();
-                            tma_store_2d_hint(&tm_y, sy, a_cta0, b0 + c, stream);
-                            tma_store_2d_hint(&tm_y, sy + 32 * 128, a_cta0 + 64, b0 + c, stream);
-                            bulk_commit_group();
-                        }
-                        ++chunk_iter;
+                    for (int e = 0; e < 2; ++e) {
+                        const int ch = a_cta0 + q * 32 + 16 * h + t4 + 8 * e;
+                        sa2[h][e] = ch < args.rowsA ? __ldg(args.s_a + ch) : 0.0f;
                     }
-                    continue;
-                }
+                // this thread's stmatrix row: matrix mi, row mj
+                const int mi = lane >> 3, mj = lane & 7;
                 for (int c = 0; c < args.bn; c += 32) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(t_row + c, r);
+                    uint32_t v[2][16];
+                    tmem_ld_16x256b_x4(t_row + c, v[0]);
+                    tmem_ld_16x256b_x4(t_row + (16u << 16) + c, v[1]);
                     tmem_ld_wait();
                     if (c + 32 >= args.bn) {  // last read of this accumulator: release it
                         tc_fence_before();
@@ -514,72 +394,144 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                 mbar_arrive(&acc_empty[acc]);
                         }
                     }
-                    const int bc = b0 + c + lane;  // this lane's B row of the chunk
-                    const float sb_lane = bc < args.rowsB ? __ldg(args.s_b + bc) : 0.0f;
-                    if (args.tma_store) {
-                        uint8_t* sy = stage_y + (chunk_iter & 1) * C::kEpiBytes;
-                        if (issuer) bulk_wait_read<1>();  // the store of two chunks ago has read it
-                        named_bar_sync(1, 128);
-                        if (args.a_is_w) {
-                            // box [32 B rows][128 A rows]: element (u, lane_row)
+                    float sb[4][2];
 #pragma unroll
-                            for (int u = 0; u < 32; ++u) {
-                                const float sb = __shfl_sync(0xffffffffu, sb_lane, u);
-                                const float accv = kInt8
-                                                       ? __int2float_rn(static_cast<int32_t>(r[u]))
-                                                       : __uint_as_float(r[u]);
-                                const float v = __fmul_rn(__fmul_rn(accv, sb), sa);
-                                reinterpret_cast<__nv_bfloat16*>(sy)[u * kTileA + lane_row] =
-                                    __float2bfloat16_rn(v);
-                            }
-                        } else {
-                            // box [128 A rows][32 B rows]: this lane's row is contiguous
-                            uint32_t packed[32 * kEsz / 4];
+                    for (int r = 0; r < 4; ++r)
 #pragma unroll
-                            for (int u = 0; u < 32; ++u) {
-                                const float sb = __shfl_sync(0xffffffffu, sb_lane, u);
-                                const float accv = kInt8
-                                                       ? __int2float_rn(static_cast<int32_t>(r[u]))
-                                                       : __uint_as_float(r[u]);
-                                const float v = __fmul_rn(__fmul_rn(accv, sa), sb);
-                                const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-                                if (u & 1)
-                                    packed[u >> 1] |= h << 16;
-                                else
-                                    packed[u >> 1] = h;
-                            }
-                            uint4* dst = reinterpret_cast<uint4*>(sy + lane_row * 32 * kEsz);
-#pragma unroll
-                            for (int w = 0; w < 32 * kEsz / 16; ++w)
-                                dst[w] = make_uint4(packed[4 * w], packed[4 * w + 1],
-                                                    packed[4 * w + 2], packed[4 * w + 3]);
+                        for (int e = 0; e < 2; ++e) {
+                            const int tok = b0 + c + 8 * r + 2 * tm + e;
+                            sb[r][e] = tok < args.rowsB ? __ldg(args.s_b + tok) : 0.0f;
                         }
-                        fence_async_shared();
-                        named_bar_sync(1, 128);
-                        if (issuer) {
-                            const uint64_t stream = l2_policy_evict_first();
-                            if (args.a_is_w)
-                                tma_store_2d_hint(&tm_y, sy, a_cta0, b0 + c, stream);
-                            else
-                                tma_store_2d_hint(&tm_y, sy, b0 + c, a_cta0, stream);
-                            bulk_commit_group();
+                    uint32_t pk[2][8];  // [half][column group r * 2 + channel block]
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int r = 0; r < 4; ++r)
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                float y2[2];
+#pragma unroll
+                                for (int k = 0; k < 2; ++k) {
+                                    const uint32_t bits = v[h][4 * r + 2 * e + k];
+                                    const float accv =
+                                        kInt8 ? __int2float_rn(static_cast<int32_t>(bits))
+                                              : __uint_as_float(bits);
+                                    y2[k] = __fmul_rn(__fmul_rn(accv, sb[r][k]), sa2[h][e]);
+                                }
+                                const __nv_bfloat162 b2 = __floats2bfloat162_rn(y2[0], y2[1]);
+                                pk[h][2 * r + e] = *reinterpret_cast<const uint32_t*>(&b2);
+                            }
+                    uint8_t* sy = stage_y + (chunk_iter & 1) * C::kEpiBytes;
+                    if (issuer) bulk_wait_read<1>();  // the stores of two chunks ago have read it
+                    named_bar_sync(1, 128);
+                    const uint32_t sy_u32 = smem_u32(sy);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int rp = 0; rp < 2; ++rp) {
+                            // matrices: (r = 2rp, e = 0), (2rp, 1), (2rp+1, 0), (2rp+1, 1)
+                            const int r = 2 * rp + (mi >> 1);
+                            const int e = mi & 1;
+                            const int tok = 8 * r + mj;                 // row of the chunk
+                            const int ch = q * 32 + 16 * h + 8 * e;     // 8-channel block
+                            const int half = ch >> 6;
+                            const int blk = (ch & 63) >> 3;
+                            const uint32_t addr = sy_u32 + half * (32 * 128) + tok * 128 +
+                                                  ((blk ^ (tok & 7)) << 4);
+                            stmatrix_x4_trans(addr, pk[h][4 * rp + 0], pk[h][4 * rp + 1],
+                                              pk[h][4 * rp + 2], pk[h][4 * rp + 3]);
                         }
-                        ++chunk_iter;
-                    } else {
+                    fence_async_shared();
+                    named_bar_sync(1, 128);
+                    if (issuer) {
+                        const uint64_t stream = l2_policy_evict_first();
+                        tma_store_2d_hint(&tm_y, sy, a_cta0, b0 + c, stream);
+                        tma_store_2d_hint(&tm_y, sy + 32 * 128, a_cta0 + 64, b0 + c, stream);
+                        bulk_commit_group();
+                    }
+                    ++chunk_iter;
+                }
+                continue;
+            }
+            for (int c = 0; c < args.bn; c += 32) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(t_row + c, r);
+                tmem_ld_wait();
+                if (c + 32 >= args.bn) {  // last read of this accumulator: release it
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if constexpr (kPair == 2)
+                            mbar_arrive_cluster(acc_empty_leader + acc * sizeof(uint64_t));
+                        else
+                            mbar_arrive(&acc_empty[acc]);
+                    }
+                }
+                const int bc = b0 + c + lane;  // this lane's B row of the chunk
+                const float sb_lane = bc < args.rowsB ? __ldg(args.s_b + bc) : 0.0f;
+                if (args.tma_store) {
+                    uint8_t* sy = stage_y + (chunk_iter & 1) * C::kEpiBytes;
+                    if (issuer) bulk_wait_read<1>();  // the store of two chunks ago has read it
+                    named_bar_sync(1, 128);
+                    if (args.a_is_w) {
+                        // box [32 B rows][128 A rows]: element (u, lane_row)
 #pragma unroll
                         for (int u = 0; u < 32; ++u) {
-                            const int b_row = b0 + c + u;
                             const float sb = __shfl_sync(0xffffffffu, sb_lane, u);
-                            if (row_ok && b_row < args.rowsB) {
-                                if (args.a_is_w)
-                                    store_scaled<kInt8, kOutBf16>(
-                                        args.y, static_cast<int64_t>(b_row) * args.ldy + a_row,
-                                        r[u], sb, sa);
-                                else
-                                    store_scaled<kInt8, kOutBf16>(
-                                        args.y, static_cast<int64_t>(a_row) * args.ldy + b_row,
-                                        r[u], sa, sb);
-                            }
+                            const float accv = kInt8
+                                                   ? __int2float_rn(static_cast<int32_t>(r[u]))
+                                                   : __uint_as_float(r[u]);
+                            const float v = __fmul_rn(__fmul_rn(accv, sb), sa);
+                            reinterpret_cast<__nv_bfloat16*>(sy)[u * kTileA + lane_row] =
+                                __float2bfloat16_rn(v);
+                        }
+                    } else {
+                        // box [128 A rows][32 B rows]: this lane's row is contiguous
+                        uint32_t packed[32 * kEsz / 4];
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) {
+                            const float sb = __shfl_sync(0xffffffffu, sb_lane, u);
+                            const float accv = kInt8
+                                                   ? __int2float_rn(static_cast<int32_t>(r[u]))
+                                                   : __uint_as_float(r[u]);
+                            const float v = __fmul_rn(__fmul_rn(accv, sa), sb);
+                            const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+                            if (u & 1)
+                                packed[u >> 1] |= h << 16;
+                            else
+                                packed[u >> 1] = h;
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(sy + lane_row * 32 * kEsz);
+#pragma unroll
+                        for (int w = 0; w < 32 * kEsz / 16; ++w)
+                            dst[w] = make_uint4(packed[4 * w], packed[4 * w + 1],
+                                                packed[4 * w + 2], packed[4 * w + 3]);
+                    }
+                    fence_async_shared();
+                    named_bar_sync(1, 128);
+                    if (issuer) {
+                        const uint64_t stream = l2_policy_evict_first();
+                        if (args.a_is_w)
+                            tma_store_2d_hint(&tm_y, sy, a_cta0, b0 + c, stream);
+                        else
+                            tma_store_2d_hint(&tm_y, sy, b0 + c, a_cta0, stream);
+                        bulk_commit_group();
+                    }
+                    ++chunk_iter;
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        const int b_row = b0 + c + u;
+                        const float sb = __shfl_sync(0xffffffffu, sb_lane, u);
+                        if (row_ok && b_row < args.rowsB) {
+                            if (args.a_is_w)
+                                store_scaled<kInt8, kOutBf16>(
+                                    args.y, static_cast<int64_t>(b_row) * args.ldy + a_row,
+                                    r[u], sb, sa);
+                            else
+                                store_scaled<kInt8, kOutBf16>(
+                                    args.y, static_cast<int64_t>(a_row) * args.ldy + b_row,
+                                    r[u], sa, sb);
                         }
                     }
                 }
