@@ -90,6 +90,28 @@ __device__ __forceinline__ void top2_of4(const float* v, int& i0, int& i1) {
     i1 = k0 ? (k1 ? 1 : (k2 ? 2 : 3)) : (k1 ? (k2 ? 2 : 3) : 3);
 }
 
+// top2_of4 on four bf16 values given as two 32-bit words (element i in bits
+// 16(i%2) of word i/2), in integer arithmetic: key_i = |x_i| bits * 4 +
+// (3 - i) orders by magnitude and, among equal magnitudes, by lower index --
+// the same order as top2_of4 for every non-NaN input (|bf16| bit patterns
+// are monotone in the value).  Returns the two kept bf16 values, lower index
+// in the low half, picked with one byte permute.
+__device__ __forceinline__ uint32_t top2_of4_bf16(uint32_t lo, uint32_t hi, int& i0, int& i1) {
+    const uint32_t k0 = (lo & 0x7FFFu) * 4u + 3u;
+    const uint32_t k1 = ((lo >> 16) & 0x7FFFu) * 4u + 2u;
+    const uint32_t k2 = (hi & 0x7FFFu) * 4u + 1u;
+    const uint32_t k3 = ((hi >> 16) & 0x7FFFu) * 4u;
+    const uint32_t a = max(k0, k1), b = min(k0, k1), c = max(k2, k3), d = min(k2, k3);
+    const uint32_t first = max(a, c);                   // the largest key
+    const uint32_t second = max(min(a, c), max(b, d));  // the second largest
+    const int ia = static_cast<int>((first & 3u) ^ 3u), ib = static_cast<int>((second & 3u) ^ 3u);
+    i0 = min(ia, ib);
+    i1 = max(ia, ib);
+    // bytes 2 i0, 2 i0 + 1 -> low half; 2 i1, 2 i1 + 1 -> high half
+    const uint32_t sel = static_cast<uint32_t>(i0) * 0x22u + static_cast<uint32_t>(i1) * 0x2200u + 0x1010u;
+    return __byte_perm(lo, hi, sel);
+}
+
 // Value at local index i (0..3) of a group, without indexing registers
 // dynamically.
 __device__ __forceinline__ float pick4(const float* v, int i) {
@@ -279,6 +301,31 @@ __global__ void __launch_bounds__(kWarpRowThreads) prune_act_warp_kernel(
     uint4* vout = reinterpret_cast<uint4*>(Xv + m * (K_lp64 / 2));
     const int n_steps = K_lp / 32;
     for (int st = lane; st < n_steps; st += 32) {
+        if constexpr (sizeof(T) == 2) {
+            if (vec && st * 32 + 32 <= K) {  // bf16: select on the raw words
+                const uint4* p = reinterpret_cast<const uint4*>(x) + 4 * st;
+                const uint4 c0 = __ldg(p), c1 = __ldg(p + 1), c2 = __ldg(p + 2), c3 = __ldg(p + 3);
+                const uint32_t w[16] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w,
+                                        c2.x, c2.y, c2.z, c2.w, c3.x, c3.y, c3.z, c3.w};
+                uint32_t vals[4];
+                uint32_t nibs = 0;
+#pragma unroll
+                for (int gi = 0; gi < 8; ++gi) {
+                    int i0, i1;
+                    const uint32_t kept = top2_of4_bf16(w[2 * gi], w[2 * gi + 1], i0, i1);
+                    const uint32_t q = quantize_pair<kInt8>(__uint_as_float(kept << 16),
+                                                            __uint_as_float(kept & 0xFFFF0000u), inv);
+                    if (gi & 1)
+                        vals[gi >> 1] |= q << 16;
+                    else
+                        vals[gi >> 1] = q;
+                    nibs |= static_cast<uint32_t>(i0 | (i1 << 2)) << (4 * gi);
+                }
+                __stcs(vout + st, make_uint4(vals[0], vals[1], vals[2], vals[3]));
+                __stcs(reinterpret_cast<uint32_t*>(Xm + meta_offset(m, 4 * st, K_lp64)), nibs);
+                continue;
+            }
+        }
         float f[32];
         gload16<T>(x, st * 32, K, vec, *reinterpret_cast<float(*)[16]>(f));
         gload16<T>(x, st * 32 + 16, K, vec, *reinterpret_cast<float(*)[16]>(f + 16));

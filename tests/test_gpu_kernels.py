@@ -105,6 +105,22 @@ def test_compress_weight_with_ties_and_zeros():
                                           oracle.meta_to_tiles(Wm_ref, Wv_ref.shape[1] * 2))
 
 
+@pytest.mark.parametrize("q", ["int8", "fp8"])
+def test_prune_act_ties_and_zeros(q):
+    """Small integers as bf16: exact ties inside most groups of 4 (the lower
+    index wins), all-zero groups, a zero row and -0.0 against +0.0."""
+    rng = np.random.default_rng(11)
+    X = torch.tensor(rng.integers(-3, 4, (300, 512)), dtype=torch.float32)
+    X[7] = 0.0
+    X[9, ::3] = -0.0
+    X = X.to(torch.bfloat16)
+    Xv_ref, Xm_ref, s_ref = oracle.prune_act_2to4(X, Q[q])
+    Xv, Xm, s_x = ss.prune_act_2to4(dev(X), q)
+    np.testing.assert_array_equal(host(s_x), s_ref)
+    np.testing.assert_array_equal(host(Xm), oracle.meta_to_tiles(Xm_ref, Xv_ref.shape[1] * 2))
+    np.testing.assert_array_equal(host(Xv), Xv_ref)
+
+
 def test_nan_weight_reports_data_error():
     W = torch.randn(8, 64)
     W[3, 10] = float("nan")
