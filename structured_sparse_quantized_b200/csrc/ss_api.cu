@@ -384,7 +384,8 @@ ss_status ss_quant_lift_act(const void* X, ss_in_dtype in_dtype, int64_t M, int6
     if (!aligned16(X) || !aligned16(Xq_lift) || !aligned16(s_x)) return SS_ERR_ALIGNMENT;
     // one warp per token row; sliding patterns keep a quantised byte row per
     // warp in shared memory
-    const int q_stride = p.group <= 4 ? 0 : static_cast<int>(round_up(K_pad, 16));
+    // one code row per row slot, with one zero chunk past the last group
+    const int q_stride = p.group <= 4 ? 0 : static_cast<int>(round_up(K_pad, 16) + 16);
     int warps = ss::kWarpRowThreads / 32;
     if (q_stride > 0)
         while (warps > 1 && static_cast<size_t>(warps) * q_stride > kMaxRowSmem) warps /= 2;

@@ -454,8 +454,10 @@ __global__ void __launch_bounds__(kWarpRowThreads) quant_lift_reg_kernel(
             __stcs(z + c8, make_uint2(0, 0));
         return;
     }
-    // 4:6, 8:10: the row's codes go to a shared-memory row, then each 16-byte
-    // output word gathers four windows from it
+    // 4:6, 8:10: the row's codes go to a shared-memory row; each 16-byte output
+    // word (four windows) is then built from the 12 code bytes its windows
+    // span -- two 6-byte groups (4:6) or one 10-byte group (8:10) -- read as
+    // three aligned 32-bit words and recombined with byte permutes.
     uint4* qrow = reinterpret_cast<uint4*>(smem_raw + slot * q_stride);
     const int q_chunks = ((K_lift / (4 * (Nh - 1))) * 2 * Nh + 15) / 16;
 #pragma unroll
@@ -467,36 +469,35 @@ __global__ void __launch_bounds__(kWarpRowThreads) quant_lift_reg_kernel(
             qrow[c] = quant16<kInt8>(f, inv);
         }
     }
-    for (int c = n16 + rt; c < q_chunks; c += kRowThreads) qrow[c] = make_uint4(0, 0, 0, 0);
+    // zero codes from K to one chunk past the last group: the word reads below
+    // may run up to 6 bytes past K_pad
+    for (int c = n16 + rt; c <= q_chunks; c += kRowThreads) qrow[c] = make_uint4(0, 0, 0, 0);
     if constexpr (kWpr > 1)
         named_bar_sync(1 + slot, kRowThreads);
     else
         __syncwarp();
-    const uint16_t* q16 = reinterpret_cast<const uint16_t*>(qrow);
-    const uint32_t n_win = static_cast<uint32_t>(K_lift / 4);
-    const uint32_t per_group = static_cast<uint32_t>(Nh - 1);
+    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qrow);
+    const int n_words = (K_lift + 15) / 16;  // output words holding windows (the rest are zero)
     for (int c = rt; c < n_chunks; c += kRowThreads) {
-        uint32_t win = static_cast<uint32_t>(c) * 4u;
-        uint32_t g = win / per_group;
-        uint32_t j = win - g * per_group;
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint32_t word = 0;
-            if (win < n_win) {
-                const uint32_t half = Nh * g + j;  // base / 2, base = 2Nh g + 2j
-                word = static_cast<uint32_t>(q16[half]) |
-                       (static_cast<uint32_t>(q16[half + 1]) << 16);
-            }
-            w[i] = word;
-            ++win;
-            if (++j == per_group) {
-                j = 0;
-                ++g;
+        uint4 o = make_uint4(0, 0, 0, 0);
+        if (c < n_words) {
+            if (Nh == 3) {
+                // groups 2c, 2c+1: code bytes 12c .. 12c+11; windows at 0, 2, 6, 8
+                const uint32_t u0 = q32[3 * c], u1 = q32[3 * c + 1], u2 = q32[3 * c + 2];
+                o = make_uint4(u0, __byte_perm(u0, u1, 0x5432), __byte_perm(u1, u2, 0x5432), u2);
+            } else {
+                // 8:10, group c: code bytes 10c .. 10c+9; windows at 0, 2, 4, 6
+                const int w0 = (10 * c) >> 2;  // first aligned word
+                const uint32_t u0 = q32[w0], u1 = q32[w0 + 1], u2 = q32[w0 + 2];
+                if ((c & 1) == 0)
+                    o = make_uint4(u0, __byte_perm(u0, u1, 0x5432), u1, __byte_perm(u1, u2, 0x5432));
+                else  // the group starts 2 bytes into u0
+                    o = make_uint4(__byte_perm(u0, u1, 0x5432), u1, __byte_perm(u1, u2, 0x5432), u2);
             }
         }
-        __stcs(out + c, make_uint4(w[0], w[1], w[2], w[3]));
+        __stcs(out + c, o);
     }
 }
+
 
 }  // namespace ss
