@@ -212,6 +212,26 @@ class Path:
         if ev:
             ev[2].record()
 
+    def sparse_rows(self, X_rows, r0: int, r1: int):
+        """The sparse path on token rows r0..r1 (a multiple of 128 apart) of
+        this workload, on the current stream: X_rows in, Y rows r0..r1 out."""
+        ss = self.ss
+        m = r1 - r0
+        if self.online:
+            Xv, Xm, s_x = self.act
+            part = (Xv[r0:r1], Xm[r0 // 128:r1 // 128], s_x[r0:r1])
+            ss.prune_act_2to4(X_rows, self.q, out=part)
+            Wq, _, s_w = self.dense_w
+            ss.sparse_gemm(1, part[0], part[1], part[2], Wq, s_w, m, self.N, self.q,
+                           out=self.Y[r0:r1])
+        else:
+            Xq, s_x = self.act
+            part = (Xq[r0:r1], s_x[r0:r1])
+            ss.quant_lift_act(X_rows, self.pat, self.q, out=part)
+            Wv, Wm, s_w = self.sparse_w
+            ss.sparse_gemm(0, Wv, Wm, s_w, part[0], part[1], m, self.N, self.q,
+                           out=self.Y[r0:r1])
+
     def dense_step(self, ev=None):
         ss = self.ss
         if ev:
@@ -307,23 +327,45 @@ def measure(path: Path, steps: int, warmup: int, dist: Dist, peaks: dict):
     return r
 
 
-def e2e(path: Path, steps: int, warmup: int, dist: Dist):
+def e2e(path: Path, steps: int, warmup: int, dist: Dist, chunks: int = 8):
     """Same metric through the public API with host buffers: pinned X copied
-    in, path run, Y copied out, all inside the timed events."""
+    in, path run, Y copied out, all inside the timed events.  The step's
+    tokens go in `chunks` row blocks on three streams, so the copy of block
+    c+1 in, the path on block c and the copy of block c-1 out overlap."""
     X_pin = path.X_host.pin_memory()
     Y_pin = torch.empty(path.Y.shape, dtype=path.Y.dtype).pin_memory()
     X_dev = torch.empty_like(path.X)
+    M = path.M
+    if M % (128 * chunks) != 0:
+        chunks = 1
+    mc = M // chunks
+    streams = [torch.cuda.Stream() for _ in range(3)]  # copy in, compute, copy out
+    e_in = [torch.cuda.Event() for _ in range(chunks)]
+    e_done = [torch.cuda.Event() for _ in range(chunks)]
 
     def step(ev):
+        cur = torch.cuda.current_stream()
         if ev:
-            ev[0].record()
-        X_dev.copy_(X_pin, non_blocking=True)
-        path.sparse_step(None, X=X_dev)
+            ev[0].record(cur)
+        for st in streams:
+            st.wait_stream(cur)
+        for c in range(chunks):
+            r0, r1 = c * mc, (c + 1) * mc
+            with torch.cuda.stream(streams[0]):
+                X_dev[r0:r1].copy_(X_pin[r0:r1], non_blocking=True)
+                e_in[c].record()
+            with torch.cuda.stream(streams[1]):
+                streams[1].wait_event(e_in[c])
+                path.sparse_rows(X_dev[r0:r1], r0, r1)
+                e_done[c].record()
+            with torch.cuda.stream(streams[2]):
+                streams[2].wait_event(e_done[c])
+                Y_pin[r0:r1].copy_(path.Y[r0:r1], non_blocking=True)
+        for st in streams:
+            cur.wait_stream(st)
         if ev:
-            ev[1].record()
-        Y_pin.copy_(path.Y, non_blocking=True)
-        if ev:
-            ev[2].record()
+            ev[1].record(cur)
+            ev[2].record(cur)
 
     flush = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
     total, _, _ = time_loop(step, steps, warmup, flush)
