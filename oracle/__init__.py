@@ -22,6 +22,7 @@ from . import build as _build
 
 INT8 = 0
 FP8_E4M3 = 1
+BF16 = 2
 OUT_F32 = 0
 OUT_BF16 = 1
 
@@ -48,6 +49,11 @@ def lib() -> ctypes.CDLL:
             "ssref_sparse_gemm": [i32, p, p, p, p, p, i64, i64, i64, i32, p, i64, i32, p],
             "ssref_quantize_value": [ctypes.c_float, ctypes.c_float, i32, p],
             "ssref_scale_from_absmax": [ctypes.c_float, i32, p, p],
+            "ssref_compress_weight_bf16": [p, i64, i64, i32, i32, p, p],
+            "ssref_lift_act_bf16": [p, i64, i64, i32, i32, p],
+            "ssref_decompress_2to4_bf16": [p, p, i64, i64, p],
+            "ssref_matmul_bf16": [p, p, i64, i64, i64, p, i64, i32, p],
+            "ssref_sparse_gemm_bf16": [i32, p, p, p, i64, i64, i64, p, i64, i32, p],
         }
         for name, args in sig.items():
             fn = getattr(_lib, name)
@@ -328,3 +334,81 @@ def meta_from_tiles(At: np.ndarray, rows: int, K_lp: int) -> np.ndarray:
     rt = (rows + 127) // 128
     At = At.reshape(rt, K_lp // 128, 128, 16)
     return np.ascontiguousarray(At.transpose(0, 2, 1, 3).reshape(rt * 128, K_lp // 8)[:rows])
+
+
+# ---------------------------------------------------------------- bf16 tier
+
+def compress_weight_bf16(W, p: str):
+    """-> (Wv uint16 bf16 bits, Wm); Wv is [N, K_lp] for 'dense', else [N, K_lp/2]."""
+    W = _f32(W)
+    N, K = W.shape
+    keep, group = pattern(p)
+    _, _, K_lp = slide_shape(p, K)
+    if group == 0:
+        Wv = np.zeros((N, K_lp), dtype=np.uint16)
+        Wm = None
+    else:
+        Wv = np.zeros((N, K_lp // 2), dtype=np.uint16)
+        Wm = np.zeros((N, K_lp // 8), dtype=np.uint8)
+    _check(lib().ssref_compress_weight_bf16(_ptr(W), N, K, keep, group, _ptr(Wv), _ptr(Wm)),
+           "compress_weight_bf16")
+    return Wv, Wm
+
+
+def lift_act_bf16(X, p: str):
+    """-> Xl [M, K_lp] uint16 bf16 bits."""
+    X = _f32(X)
+    M, K = X.shape
+    keep, group = pattern(p)
+    _, _, K_lp = slide_shape(p, K)
+    Xl = np.zeros((M, K_lp), dtype=np.uint16)
+    _check(lib().ssref_lift_act_bf16(_ptr(X), M, K, keep, group, _ptr(Xl)), "lift_act_bf16")
+    return Xl
+
+
+def decompress_2to4_bf16(Av: np.ndarray, Am: np.ndarray, K_lp: int) -> np.ndarray:
+    Av = np.ascontiguousarray(Av, dtype=np.uint16)
+    Am = np.ascontiguousarray(Am, dtype=np.uint8)
+    rows = Av.shape[0]
+    A = np.zeros((rows, K_lp), dtype=np.uint16)
+    _check(lib().ssref_decompress_2to4_bf16(_ptr(Av), _ptr(Am), rows, K_lp, _ptr(A)),
+           "decompress_bf16")
+    return A
+
+
+def matmul_bf16(X, W, out_dtype: int, m_idx=None):
+    """Y = round_f32(X . W^T) over bf16 bits, double accumulation."""
+    X = np.ascontiguousarray(X, dtype=np.uint16)
+    W = np.ascontiguousarray(W, dtype=np.uint16)
+    M, K = X.shape
+    N = W.shape[0]
+    m_idx, R = _rows(m_idx, M)
+    Y = _out(R, N, out_dtype)
+    _check(lib().ssref_matmul_bf16(_ptr(X), _ptr(W), M, N, K, _ptr(m_idx), R, out_dtype,
+                                   _ptr(Y)), "matmul_bf16")
+    return Y
+
+
+def sparse_gemm_bf16(sparse_operand: int, Av, Am, B, M: int, N: int, K_lp: int,
+                     out_dtype: int, m_idx=None):
+    Av = np.ascontiguousarray(Av, dtype=np.uint16)
+    Am = np.ascontiguousarray(Am, dtype=np.uint8)
+    B = np.ascontiguousarray(B, dtype=np.uint16)
+    m_idx, R = _rows(m_idx, M)
+    Y = _out(R, N, out_dtype)
+    _check(lib().ssref_sparse_gemm_bf16(sparse_operand, _ptr(Av), _ptr(Am), _ptr(B), M, N, K_lp,
+                                        _ptr(m_idx), R, out_dtype, _ptr(Y)), "sparse_gemm_bf16")
+    return Y
+
+
+def plain_linear_bf16(W, X, p: str, out_dtype: int, m_idx=None):
+    """Prune W, round both operands to bf16, naive matmul over the original K."""
+    W = _f32(W)
+    X = _f32(X)
+    keep, group = pattern(p)
+    if group:
+        mask = prune_mask(W, keep, group)[:, :W.shape[1]]
+        W = np.where(mask.astype(bool), W, np.float32(0))
+    Wb, _ = compress_weight_bf16(W, "dense")
+    Xb = lift_act_bf16(X, "dense")
+    return matmul_bf16(Xb, Wb, out_dtype, m_idx)

@@ -45,6 +45,10 @@
  *      then bf16 round-to-nearest-even (or fp32 out).
  *   R8 online 2:4 pruning of activations ranks on the input magnitudes and
  *      quantises afterwards with the row absmax.
+ *   R9 the bf16 tier ([PD] 2.1 "2:4 + FP16", the 16-bit rows of the
+ *      precision-tier tables): values are stored as bf16 (round to nearest
+ *      even from the input), no scale; products of bf16 values are exact in
+ *      double, summed in k order, rounded once to binary32.
  */
 #include <math.h>
 #include <stdint.h>
@@ -57,6 +61,7 @@
 
 #define SSREF_INT8 0
 #define SSREF_FP8_E4M3 1
+#define SSREF_BF16 2
 
 #define SSREF_OUT_F32 0
 #define SSREF_OUT_BF16 1
@@ -298,8 +303,8 @@ int ssref_assign_windows(const uint8_t *mask, int64_t rows, int64_t K_pad, int g
 /* 2:4 packing of one window, reading R4.  `assigned[t]` marks the local */
 /* positions t = 0..3 the window owns; q[t] their quantised bytes.      */
 /* ------------------------------------------------------------------ */
-static uint8_t pack_window(const uint8_t assigned[4], const uint8_t q[4], uint8_t val[2]) {
-    int idx[2], n = 0;
+static uint8_t window_slots(const uint8_t assigned[4], int idx[2]) {
+    int n = 0;
     for (int t = 0; t < 4 && n < 2; t++)
         if (assigned[t]) idx[n++] = t;
     for (int t = 0; t < 4 && n < 2; t++) {       /* pad with lowest unused */
@@ -308,8 +313,22 @@ static uint8_t pack_window(const uint8_t assigned[4], const uint8_t q[4], uint8_
         if (!assigned[t] && !used) idx[n++] = t;
     }
     if (idx[0] > idx[1]) { int tmp = idx[0]; idx[0] = idx[1]; idx[1] = tmp; }
-    for (int s = 0; s < 2; s++) val[s] = assigned[idx[s]] ? q[idx[s]] : 0;
     return (uint8_t)(idx[0] | (idx[1] << 2));
+}
+
+static uint8_t pack_window(const uint8_t assigned[4], const uint8_t q[4], uint8_t val[2]) {
+    int idx[2];
+    uint8_t nib = window_slots(assigned, idx);
+    for (int s = 0; s < 2; s++) val[s] = assigned[idx[s]] ? q[idx[s]] : 0;
+    return nib;
+}
+
+/* The same packing for 16-bit values (the bf16 tier). */
+static uint8_t pack_window16(const uint8_t assigned[4], const uint16_t q[4], uint16_t val[2]) {
+    int idx[2];
+    uint8_t nib = window_slots(assigned, idx);
+    for (int s = 0; s < 2; s++) val[s] = assigned[idx[s]] ? q[idx[s]] : 0;
+    return nib;
 }
 
 static void put_nibble(uint8_t *row_meta, int64_t w, uint8_t nib) {
@@ -483,6 +502,146 @@ int ssref_decompress_2to4(const uint8_t *Av, const uint8_t *Am, int64_t rows, in
         }
     }
     return SSREF_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* The bf16 tier (reading R9): the same pruning, windows and packing,    */
+/* with 16-bit stored values and no quantisation.                        */
+/* ------------------------------------------------------------------ */
+static double bf16_to_double(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* Wv [N, K_lp/2] bf16 (dense: [N, K_lp]), Wm [N, K_lp/8] nibbles. */
+int ssref_compress_weight_bf16(const float *W, int64_t N, int64_t K, int keep, int group,
+                               uint16_t *Wv, uint8_t *Wm) {
+    int64_t K_pad, K_lift, K_lp;
+    int st = ssref_slide_shape(keep, group, K, &K_pad, &K_lift, &K_lp);
+    if (st) return st;
+    for (int64_t i = 0; i < N * K; i++)
+        if (!isfinite(W[i])) return SSREF_EINVAL;
+    if (group == 0) {
+        for (int64_t n = 0; n < N; n++)
+            for (int64_t k = 0; k < K_lp; k++)
+                Wv[n * K_lp + k] = k < K ? ssref_bf16_from_float(W[n * K + k]) : 0;
+        return SSREF_OK;
+    }
+    int Nh = group / 2;
+    uint8_t *mask = (uint8_t *)malloc((size_t)(N * K_pad));
+    int8_t *win = (int8_t *)malloc((size_t)(N * K_pad));
+    st = ssref_prune_mask(W, N, K, keep, group, mask);
+    if (!st) st = ssref_assign_windows(mask, N, K_pad, group, win);
+    if (st) { free(mask); free(win); return st; }
+    for (int64_t n = 0; n < N; n++) {
+        uint16_t *vrow = &Wv[n * (K_lp / 2)];
+        uint8_t *mrow = &Wm[n * (K_lp / 8)];
+        for (int64_t w = 0; w < K_lp / 4; w++) {
+            uint8_t assigned[4] = {0, 0, 0, 0};
+            uint16_t q[4] = {0, 0, 0, 0}, val[2];
+            if (w < K_lift / 4) {
+                int64_t g = w / (Nh - 1);
+                int j = (int)(w % (Nh - 1));
+                for (int t = 0; t < 4; t++) {
+                    int64_t k = g * group + 2 * j + t;
+                    if (win[n * K_pad + k] == j) {
+                        assigned[t] = 1;
+                        q[t] = ssref_bf16_from_float(k < K ? W[n * K + k] : 0.0f);
+                    }
+                }
+            }
+            uint8_t nib = pack_window16(assigned, q, val);
+            vrow[2 * w] = val[0];
+            vrow[2 * w + 1] = val[1];
+            put_nibble(mrow, w, nib);
+        }
+    }
+    free(mask);
+    free(win);
+    return SSREF_OK;
+}
+
+/* Xl [M, K_lp] bf16: the lifted activation ([OM] 3.2 window map), no scale. */
+int ssref_lift_act_bf16(const float *X, int64_t M, int64_t K, int keep, int group, uint16_t *Xl) {
+    int64_t K_pad, K_lift, K_lp;
+    int st = ssref_slide_shape(keep, group, K, &K_pad, &K_lift, &K_lp);
+    if (st) return st;
+    int Nh = group / 2;
+    for (int64_t m = 0; m < M; m++) {
+        const float *x = &X[m * K];
+        uint16_t *out = &Xl[m * K_lp];
+        if (group == 0) {
+            for (int64_t k = 0; k < K_lp; k++) out[k] = k < K ? ssref_bf16_from_float(x[k]) : 0;
+            continue;
+        }
+        for (int64_t w = 0; w < K_lp / 4; w++)
+            for (int t = 0; t < 4; t++) {
+                uint16_t q = 0;
+                if (w < K_lift / 4) {
+                    int64_t g = w / (Nh - 1), j = w % (Nh - 1);
+                    int64_t k = 2 * Nh * g + 2 * j + t;
+                    q = k < K ? ssref_bf16_from_float(x[k]) : 0;
+                }
+                out[4 * w + t] = q;
+            }
+    }
+    return SSREF_OK;
+}
+
+int ssref_decompress_2to4_bf16(const uint16_t *Av, const uint8_t *Am, int64_t rows, int64_t K_lp,
+                               uint16_t *A) {
+    if (K_lp % 8 != 0) return SSREF_EINVAL;
+    for (int64_t r = 0; r < rows; r++) {
+        for (int64_t w = 0; w < K_lp / 4; w++) {
+            uint8_t nib = get_nibble(&Am[r * (K_lp / 8)], w);
+            int i0 = nib & 3, i1 = (nib >> 2) & 3;
+            if (i0 >= i1) return SSREF_EINVAL;
+            for (int t = 0; t < 4; t++) A[r * K_lp + 4 * w + t] = 0;
+            A[r * K_lp + 4 * w + i0] = Av[r * (K_lp / 2) + 2 * w];
+            A[r * K_lp + 4 * w + i1] = Av[r * (K_lp / 2) + 2 * w + 1];
+        }
+    }
+    return SSREF_OK;
+}
+
+/* Y[r, n] = round_binary32(sum_k X[m_r, k] * W[n, k]) (double sum in k
+ * order), then bf16 RNE or fp32 out. */
+int ssref_matmul_bf16(const uint16_t *X, const uint16_t *W, int64_t M, int64_t N, int64_t K,
+                      const int64_t *m_idx, int64_t n_rows, int out_dtype, void *Y) {
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_rows; r++) {
+        int64_t m = m_idx ? m_idx[r] : r;
+        if (m < 0 || m >= M) continue;
+        for (int64_t n = 0; n < N; n++) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                acc += bf16_to_double(X[m * K + k]) * bf16_to_double(W[n * K + k]);
+            volatile float y = (float)acc;
+            if (out_dtype == SSREF_OUT_F32) ((float *)Y)[r * N + n] = y;
+            else ((uint16_t *)Y)[r * N + n] = ssref_bf16_from_float(y);
+        }
+    }
+    return SSREF_OK;
+}
+
+/* Sparse GEMM of the bf16 tier through decompression (sparse_operand as in
+ * ssref_sparse_gemm). */
+int ssref_sparse_gemm_bf16(int sparse_operand, const uint16_t *Av, const uint8_t *Am,
+                           const uint16_t *B, int64_t M, int64_t N, int64_t K_lp,
+                           const int64_t *m_idx, int64_t n_rows, int out_dtype, void *Y) {
+    int64_t rowsA = sparse_operand == 0 ? N : M;
+    uint16_t *A = (uint16_t *)malloc((size_t)(rowsA * K_lp) * sizeof(uint16_t));
+    int st = ssref_decompress_2to4_bf16(Av, Am, rowsA, K_lp, A);
+    if (!st) {
+        if (sparse_operand == 0)
+            st = ssref_matmul_bf16(B, A, M, N, K_lp, m_idx, n_rows, out_dtype, Y);
+        else
+            st = ssref_matmul_bf16(A, B, M, N, K_lp, m_idx, n_rows, out_dtype, Y);
+    }
+    free(A);
+    return st;
 }
 
 /* ------------------------------------------------------------------ */

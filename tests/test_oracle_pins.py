@@ -374,3 +374,110 @@ def test_result_within_quantisation_error_bound(pat, q):
     assert rel < (0.02 if q == oracle.INT8 else 0.06)
     if q == oracle.INT8:
         assert np.median(bound) < 0.2 * np.median(np.abs(ref)) + 1.0
+
+
+# ---------------------------------------------------------------- bf16 tier
+
+def _bf16_vals(bits: np.ndarray) -> np.ndarray:
+    return oracle.bf16_bits_to_float(bits).astype(np.float64)
+
+
+def test_bf16_matmul_matches_numpy_float64():
+    """Products of bf16 values are exact in double: the oracle's sum equals a
+    float64 library matmul of the decoded values up to summation order."""
+    rng = np.random.default_rng(21)
+    X = torch.from_numpy(rng.standard_normal((19, 260)).astype(np.float32)).to(torch.bfloat16)
+    W = torch.from_numpy(rng.standard_normal((11, 260)).astype(np.float32)).to(torch.bfloat16)
+    Xb = X.view(torch.uint16).numpy()
+    Wb = W.view(torch.uint16).numpy()
+    Y = oracle.matmul_bf16(Xb, Wb, oracle.OUT_F32)
+    ref = (_bf16_vals(Xb) @ _bf16_vals(Wb).T).astype(np.float32)
+    np.testing.assert_allclose(Y, ref, rtol=1e-6, atol=1e-6)
+    # bf16 output is the RNE rounding of the fp32 result
+    Yb = oracle.matmul_bf16(Xb, Wb, oracle.OUT_BF16)
+    np.testing.assert_array_equal(
+        Yb, torch.from_numpy(Y).to(torch.bfloat16).view(torch.uint16).numpy())
+
+
+def test_bf16_small_integers_exact():
+    """With small-integer operands every partial sum is an integer well inside
+    binary32: the result is the exact integer product."""
+    rng = np.random.default_rng(22)
+    X = rng.integers(-8, 9, (13, 96)).astype(np.float32)
+    W = rng.integers(-8, 9, (7, 96)).astype(np.float32)
+    Xb = oracle.lift_act_bf16(X, "dense")
+    Wb, _ = oracle.compress_weight_bf16(W, "dense")
+    Y = oracle.matmul_bf16(Xb, Wb, oracle.OUT_F32)
+    np.testing.assert_array_equal(Y, (X.astype(np.int64) @ W.astype(np.int64).T).astype(np.float32))
+
+
+@pytest.mark.parametrize("pat", PATTERNS)
+def test_bf16_decompress_is_lifted_pruned_weight(pat):
+    """Unpacking the compressed bf16 weight gives, window by window, the pruned
+    weight's values at the positions the window map assigns (zero elsewhere);
+    summed back over the windows that cover each k it gives prune(W) exactly."""
+    rng = np.random.default_rng(23)
+    K = 150
+    keep, group = oracle.pattern(pat)
+    W = rng.standard_normal((9, K)).astype(np.float32)
+    Wv, Wm = oracle.compress_weight_bf16(W, pat)
+    _, K_lift, K_lp = oracle.slide_shape(pat, K)
+    Wl = oracle.decompress_2to4_bf16(Wv, Wm, K_lp)
+    Wl_vals = _bf16_vals(Wl)
+    # every window holds at most 2 nonzeros (2:4 on the lifted axis)
+    assert np.all((Wl_vals.reshape(9, -1, 4) != 0).sum(-1) <= 2)
+    # fold the lifted axis back onto k with the window map of the pages
+    Nh = group // 2
+    back = np.zeros((9, K + group), dtype=np.float64)
+    for w in range(K_lift // 4):
+        g, j = divmod(w, Nh - 1)
+        for t in range(4):
+            back[:, g * group + 2 * j + t] += Wl_vals[:, 4 * w + t]
+    mask = oracle.prune_mask(W, keep, group)[:, :K].astype(bool)
+    Wp = np.where(mask, W, 0)
+    Wp_b = _bf16_vals(torch.from_numpy(Wp).to(torch.bfloat16).view(torch.uint16).numpy())
+    np.testing.assert_array_equal(back[:, :K], Wp_b)
+    assert np.all(back[:, K:] == 0)
+    assert np.all(Wl_vals[:, K_lift:] == 0)
+
+
+@pytest.mark.parametrize("pat", PATTERNS + ["dense"])
+def test_bf16_method_equals_plain_path(pat):
+    """Decompose + lift + pack + sparse matmul over K_lp equals prune + naive
+    matmul over K: exactly on small integers, to summation order otherwise."""
+    rng = np.random.default_rng(24)
+    K = 150
+    keep, group = oracle.pattern(pat)
+    _, _, K_lp = oracle.slide_shape(pat, K)
+
+    def method(W, X):
+        Wv, Wm = oracle.compress_weight_bf16(W, pat)
+        Xl = oracle.lift_act_bf16(X, pat)
+        if pat == "dense":
+            return oracle.matmul_bf16(Xl, Wv, oracle.OUT_F32)
+        return oracle.sparse_gemm_bf16(0, Wv, Wm, Xl, X.shape[0], W.shape[0], K_lp,
+                                       oracle.OUT_F32)
+
+    Wi = rng.integers(-6, 7, (40, K)).astype(np.float32)
+    Xi = rng.integers(-6, 7, (23, K)).astype(np.float32)
+    # distinct magnitudes inside each group keep the top-k choice unique
+    Wi = Wi + np.sign(Wi) * (np.arange(K) % 7)[None, :].astype(np.float32) / 8
+    np.testing.assert_array_equal(method(Wi, Xi), oracle.plain_linear_bf16(Wi, Xi, pat, oracle.OUT_F32))
+    W = rng.standard_normal((40, K)).astype(np.float32)
+    X = rng.standard_normal((23, K)).astype(np.float32)
+    np.testing.assert_allclose(method(W, X), oracle.plain_linear_bf16(W, X, pat, oracle.OUT_F32),
+                               rtol=1e-6, atol=1e-6)
+    # and the sparse-activation operand role (A = lifted X, compressed) agrees
+    if pat != "dense":
+        Xv, Xm = oracle.compress_weight_bf16(X, "2:4")
+        Wl = oracle.lift_act_bf16(W, "2:4")
+        K4 = oracle.slide_shape("2:4", K)[2]
+        Y1 = oracle.sparse_gemm_bf16(1, Xv, Xm, Wl, 23, 40, K4, oracle.OUT_F32)
+        Y0 = oracle.sparse_gemm_bf16(0, *oracle.compress_weight_bf16(W, "2:4"),
+                                     oracle.lift_act_bf16(X, "2:4"), 23, 40, K4, oracle.OUT_F32)
+        Xp = np.where(oracle.prune_mask(X, 2, 4)[:, :K].astype(bool), X, 0)
+        Wp = np.where(oracle.prune_mask(W, 2, 4)[:, :K].astype(bool), W, 0)
+        np.testing.assert_allclose(Y1, oracle.plain_linear_bf16(W, Xp, "dense", oracle.OUT_F32),
+                                   rtol=1e-6, atol=1e-6)
+        np.testing.assert_allclose(Y0, oracle.plain_linear_bf16(Wp, X, "dense", oracle.OUT_F32),
+                                   rtol=1e-6, atol=1e-6)
