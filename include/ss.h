@@ -47,7 +47,13 @@ typedef enum {
 } ss_status;
 
 typedef enum { SS_IN_F32 = 0, SS_IN_BF16 = 1 } ss_in_dtype;
-typedef enum { SS_INT8 = 0, SS_FP8_E4M3 = 1 } ss_qdtype;
+/* Stored operand type.  SS_BF16 is the 16-bit tier (the "2:4 + FP16" tier
+ * of the "add 2:4 or drop a precision tier?" study, paper-daily 2610.28947,
+ * section 1; the 16-bit rows of the SlideSparse precision list, 66bd.net):
+ * values are kept as bf16 (round to nearest even from the input), two bytes
+ * each, with no scale -- every s_w / s_x / s_a / s_b argument is then unused
+ * and may be NULL, and the GEMM epilogue is y = fp32 acc (then bf16 RNE). */
+typedef enum { SS_INT8 = 0, SS_FP8_E4M3 = 1, SS_BF16 = 2 } ss_qdtype;
 typedef enum { SS_OUT_F32 = 0, SS_OUT_BF16 = 1 } ss_out_dtype;
 
 /* Sparsity pattern keep:group; {2,4},{4,6},{6,8},{8,10}; {0,0} = dense. */
@@ -79,6 +85,12 @@ ss_status ss_act_2to4_shape(int64_t K, int64_t *K_lp);
  *   byte b of row r (its nibbles as in the row layout [rows, K_lp/8]) is at
  *   ((r / 128) * (K_lp / 128) + b / 16) * 2048 + (r % 128) * 16 + b % 16.
  * Rows are padded to a multiple of 128; padding rows are zero.
+ * SS_BF16 metadata adds one exchange inside each block: the 16-bit sparse
+ * MMA reads the selectors of rows r and r + 8 (r % 16 < 8) for one MMA as
+ * the two 2-byte halves of one 4-byte word, so bytes b of row r with
+ * b % 4 in {2, 3} and r % 16 < 8 swap places with bytes b - 2 of row r + 8:
+ * byte b of row r is at the offset above for row (r & ~8) | (b & 2) << 2 and
+ * byte (b & ~2) | (r & 8) >> 2.
  * Returns 0 for rows < 1 or K_lp not a positive multiple of 128. */
 int64_t ss_meta_bytes(int64_t rows, int64_t K_lp);
 
@@ -100,7 +112,9 @@ int64_t ss_meta_bytes(int64_t rows, int64_t K_lp);
  *       nibbles, window w in its byte w/2, low nibble = even w
  *   s_w [N] fp32
  * Dense: Wv is [N, K_lp] (per-channel quantised W, zero padded), Wm unused
- * (may be NULL).  A NaN/Inf weight sets SS_ERR_DATA in the device status. */
+ * (may be NULL).  A NaN/Inf weight sets SS_ERR_DATA in the device status.
+ * SS_BF16: step 2 is bf16 rounding with no scale; Wv holds 2-byte values
+ * ([N, K_lp/2] bf16, dense [N, K_lp] bf16); s_w is not written. */
 ss_status ss_compress_weight(const void *W, ss_in_dtype in_dtype, int64_t N, int64_t K,
                              ss_pattern p, ss_qdtype q, void *Wv, void *Wm, float *s_w,
                              ss_stream_t stream);
@@ -111,7 +125,9 @@ ss_status ss_compress_weight(const void *W, ss_in_dtype in_dtype, int64_t N, int
  * base = 2Nh * (i / (Nh-1)) + 2 * (i % (Nh-1)), four bytes packed per word).
  * Per token m of X[M, K]: a = max_k |x|, s_x[m] = a / Q, q = RNE(x * (Q / a));
  * Xq_lift[m, 4i + t] = q(X[m, base_i + t]) (0 past K and past K_lift).
- * Outputs: Xq_lift [M, K_lp] bytes, s_x [M] fp32.  Dense: identity map. */
+ * Outputs: Xq_lift [M, K_lp] bytes, s_x [M] fp32.  Dense: identity map.
+ * SS_BF16: no quantisation; Xq_lift [M, K_lp] holds the bf16 of X under the
+ * same map (0 past K and K_lift); s_x is not written. */
 ss_status ss_quant_lift_act(const void *X, ss_in_dtype in_dtype, int64_t M, int64_t K,
                             ss_pattern p, ss_qdtype q, void *Xq_lift, float *s_x,
                             ss_stream_t stream);
@@ -122,7 +138,9 @@ ss_status ss_quant_lift_act(const void *X, ss_in_dtype in_dtype, int64_t M, int6
  * in each group of 4 along K keep the two largest |x| (ties keep the lower
  * index), s_x[m] = row absmax / Q, quantise the kept values, pack as in
  * ss_compress_weight.  Outputs Xv [M, K_lp/2], Xm (ss_meta_bytes(M, K_lp)
- * bytes, tile-major), s_x [M] with K_lp from ss_act_2to4_shape(). */
+ * bytes, tile-major), s_x [M] with K_lp from ss_act_2to4_shape().
+ * SS_BF16: the kept values are stored as bf16 (Xv [M, K_lp/2] bf16), no
+ * scale; s_x is not written. */
 ss_status ss_prune_act_2to4(const void *X, ss_in_dtype in_dtype, int64_t M, int64_t K,
                             ss_qdtype q, void *Xv, void *Xm, float *s_x, ss_stream_t stream);
 
@@ -134,11 +152,12 @@ ss_status ss_prune_act_2to4(const void *X, ss_in_dtype in_dtype, int64_t M, int6
  * sparse_operand = 1: A = activation.  Av = Xv [M, K_lp/2], Am = Xm
  *                     (tile-major), s_a = s_x [M]; B = Wq [N, K_lp] (dense),
  *                     s_b = s_w [N].
- * acc is exact int32 for INT8 and fp32 (tensor-core accumulation) for E4M3.
+ * acc is exact int32 for INT8 and fp32 (tensor-core accumulation) for E4M3
+ * and SS_BF16 (kind::f16; Av, B hold 2-byte values, s_a / s_b unused).
  * K_lp must be a positive multiple of 128; M, N in [1, 2^31).
  * Kernel shape: with more than 128 weight rows and bf16 Y, large problems
  * run output tiles of 256 channels x 2 token tiles (one A slice feeds two
- * MMAs), the rest 256 x 1.  The choice follows the wave count; the
+ * MMAs), the rest (and every SS_BF16 problem) 256 x 1.  The choice follows the wave count; the
  * environment variable SS_SPARSE_KERNEL=narrow|wide pins it (same results). */
 ss_status ss_sparse_gemm(int sparse_operand, const void *Av, const void *Am, const float *s_a,
                          const void *B, const float *s_b, int64_t M, int64_t N, int64_t K_lp,
@@ -147,7 +166,8 @@ ss_status ss_sparse_gemm(int sparse_operand, const void *Av, const void *Am, con
 /* Dense GEMM of the same construction (tcgen05.mma), the like-for-like
  * comparison: Y = dequant(Xq [M, K_p] . Wq [N, K_p]^T) with the same
  * epilogue; Xq from ss_quant_lift_act(dense), Wq from
- * ss_compress_weight(dense).  K_p must be a positive multiple of 128. */
+ * ss_compress_weight(dense).  K_p must be a positive multiple of 128.
+ * SS_BF16: Xq, Wq hold bf16 ([M, K_p], [N, K_p]); s_x, s_w unused. */
 ss_status ss_dense_gemm(const void *Xq, const float *s_x, const void *Wq, const float *s_w,
                         int64_t M, int64_t N, int64_t K_p, ss_qdtype q, void *Y,
                         ss_out_dtype out_dtype, ss_stream_t stream);

@@ -312,12 +312,24 @@ def bf16_bits_to_float(y: np.ndarray) -> np.ndarray:
 
 # ------------------------------------------------------------------ storage layout
 
-def meta_to_tiles(Am: np.ndarray, K_lp: int) -> np.ndarray:
+def _swap_r8_halves(At: np.ndarray) -> np.ndarray:
+    """Inside each 2 KB block [128 rows][16 bytes], exchange row bit 3 with
+    byte bit 1: the 2-byte half h of 4-byte word c of row 16a + 8x + r goes to
+    row 16a + 8h + r, half x of word c (its own inverse)."""
+    rt, kt = At.shape[:2]
+    # [rt, kt, a, x, r, c, h, byte]
+    v = At.reshape(rt, kt, 8, 2, 8, 4, 2, 2)
+    return np.ascontiguousarray(v.transpose(0, 1, 2, 6, 4, 5, 3, 7).reshape(rt, kt, 128, 16))
+
+
+def meta_to_tiles(Am: np.ndarray, K_lp: int, i16: bool = False) -> np.ndarray:
     """Row-layout selectors [rows, K_lp/8] -> the library's tile-major storage
     [ceil(rows/128), K_lp/128, 128, 16]: block (row tile, K tile) holds the 16
     selector bytes of 128 lifted K for each of the tile's 128 rows; padding
-    rows are zero.  A pure relabelling of bytes (no arithmetic), used to hand
-    oracle metadata to the GPU and to compare the GPU's metadata with it."""
+    rows are zero.  With i16 (the bf16 tier) the 2-byte halves of rows r and
+    r + 8 of each 16-row group are exchanged as well (_swap_r8_halves).  A
+    pure relabelling of bytes (no arithmetic), used to hand oracle metadata to
+    the GPU and to compare the GPU's metadata with it."""
     Am = np.ascontiguousarray(Am, dtype=np.uint8)
     rows, nb = Am.shape
     assert nb == K_lp // 8 and K_lp % 128 == 0
@@ -325,14 +337,17 @@ def meta_to_tiles(Am: np.ndarray, K_lp: int) -> np.ndarray:
     padded = np.zeros((rt * 128, nb), dtype=np.uint8)
     padded[:rows] = Am
     # [row tile, row in tile, K tile, byte in K tile] -> [row tile, K tile, row, byte]
-    return np.ascontiguousarray(padded.reshape(rt, 128, K_lp // 128, 16).transpose(0, 2, 1, 3))
+    At = np.ascontiguousarray(padded.reshape(rt, 128, K_lp // 128, 16).transpose(0, 2, 1, 3))
+    return _swap_r8_halves(At) if i16 else At
 
 
-def meta_from_tiles(At: np.ndarray, rows: int, K_lp: int) -> np.ndarray:
+def meta_from_tiles(At: np.ndarray, rows: int, K_lp: int, i16: bool = False) -> np.ndarray:
     """Inverse of meta_to_tiles: tile-major storage -> [rows, K_lp/8]."""
     At = np.ascontiguousarray(At, dtype=np.uint8)
     rt = (rows + 127) // 128
     At = At.reshape(rt, K_lp // 128, 128, 16)
+    if i16:
+        At = _swap_r8_halves(At)
     return np.ascontiguousarray(At.transpose(0, 2, 1, 3).reshape(rt * 128, K_lp // 8)[:rows])
 
 
@@ -412,3 +427,10 @@ def plain_linear_bf16(W, X, p: str, out_dtype: int, m_idx=None):
     Wb, _ = compress_weight_bf16(W, "dense")
     Xb = lift_act_bf16(X, "dense")
     return matmul_bf16(Xb, Wb, out_dtype, m_idx)
+
+
+def prune_act_2to4_bf16(X):
+    """Online 2:4 prune of an activation in the bf16 tier -> (Xv bf16 bits,
+    Xm).  With no scale, this is the 2:4 weight compression applied to the
+    token rows: the same magnitude ranking, tie rule and packing."""
+    return compress_weight_bf16(X, "2:4")

@@ -1,6 +1,7 @@
 """structured_sparse_quantized_b200 -- Python binding of libss.
 
-Quantized (INT8 / FP8-E4M3) matmul on the Blackwell sparse tensor cores for
+Quantized (INT8 / FP8-E4M3, and the unscaled BF16 tier) matmul on the
+Blackwell sparse tensor cores for
 structured-sparse weights: hardware 2:4 and the milder (2Nh-2):2Nh patterns
 (4:6, 6:8, 8:10) brought to 2:4 by SlideSparse's sliding-window
 decomposition.  Every step runs in the CUDA kernels of ``libss.so`` (see
@@ -38,10 +39,10 @@ SS_ERR_TIMEOUT = 6
 SS_ERR_DATA = 7
 
 SS_IN_F32, SS_IN_BF16 = 0, 1
-SS_INT8, SS_FP8_E4M3 = 0, 1
+SS_INT8, SS_FP8_E4M3, SS_BF16 = 0, 1, 2
 SS_OUT_F32, SS_OUT_BF16 = 0, 1
 
-QDTYPES = {"int8": SS_INT8, "fp8": SS_FP8_E4M3, "e4m3": SS_FP8_E4M3}
+QDTYPES = {"int8": SS_INT8, "fp8": SS_FP8_E4M3, "e4m3": SS_FP8_E4M3, "bf16": SS_BF16}
 
 
 class SSError(RuntimeError):
@@ -226,6 +227,16 @@ def ss_get_device_status(stream=None) -> int:
 
 
 # ------------------------------------------------------------------ allocating wrappers
+# Stored values are uint8 codes for the 8-bit tiers and bfloat16 for the bf16
+# tier, which has no scales (its s_* entries are None).
+
+def _vals_dtype(q) -> torch.dtype:
+    return torch.bfloat16 if _qdtype(q) == SS_BF16 else torch.uint8
+
+
+def _scales(n: int, q, dev):
+    return None if _qdtype(q) == SS_BF16 else torch.empty(n, dtype=torch.float32, device=dev)
+
 
 def compress_weight(W: torch.Tensor, pattern, q, stream=None):
     """-> (Wv, Wm, s_w); Wm is None for 'dense'."""
@@ -233,13 +244,14 @@ def compress_weight(W: torch.Tensor, pattern, q, stream=None):
     p = _pattern(pattern)
     _, _, K_lp = ss_slide_shape(p, K)
     dev = W.device
+    vd = _vals_dtype(q)
     if p.group == 0:
-        Wv = torch.empty((N, K_lp), dtype=torch.uint8, device=dev)
+        Wv = torch.empty((N, K_lp), dtype=vd, device=dev)
         Wm = None
     else:
-        Wv = torch.empty((N, K_lp // 2), dtype=torch.uint8, device=dev)
+        Wv = torch.empty((N, K_lp // 2), dtype=vd, device=dev)
         Wm = torch.empty(meta_shape(N, K_lp), dtype=torch.uint8, device=dev)
-    s_w = torch.empty(N, dtype=torch.float32, device=dev)
+    s_w = _scales(N, q, dev)
     ss_compress_weight(W, p, q, Wv, Wm, s_w, stream)
     return Wv, Wm, s_w
 
@@ -249,8 +261,8 @@ def quant_lift_act(X: torch.Tensor, pattern, q, stream=None, out=None):
     p = _pattern(pattern)
     _, _, K_lp = ss_slide_shape(p, K)
     if out is None:
-        out = (torch.empty((M, K_lp), dtype=torch.uint8, device=X.device),
-               torch.empty(M, dtype=torch.float32, device=X.device))
+        out = (torch.empty((M, K_lp), dtype=_vals_dtype(q), device=X.device),
+               _scales(M, q, X.device))
     ss_quant_lift_act(X, p, q, out[0], out[1], stream)
     return out
 
@@ -259,9 +271,9 @@ def prune_act_2to4(X: torch.Tensor, q, stream=None, out=None):
     M, K = X.shape
     K_lp = ss_act_2to4_shape(K)
     if out is None:
-        out = (torch.empty((M, K_lp // 2), dtype=torch.uint8, device=X.device),
+        out = (torch.empty((M, K_lp // 2), dtype=_vals_dtype(q), device=X.device),
                torch.empty(meta_shape(M, K_lp), dtype=torch.uint8, device=X.device),
-               torch.empty(M, dtype=torch.float32, device=X.device))
+               _scales(M, q, X.device))
     ss_prune_act_2to4(X, q, out[0], out[1], out[2], stream)
     return out
 

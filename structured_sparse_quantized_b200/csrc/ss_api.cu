@@ -113,11 +113,11 @@ bool make_y_map(CUtensorMap* map, void* Y, int64_t M, int64_t N, bool out_bf16, 
                   : make_map_2d(map, Y, M, N, ss::kTileA, 32, CU_TENSOR_MAP_SWIZZLE_NONE, dt, esz);
 }
 
-template <bool kSparse, bool kInt8, bool kOutBf16, int kPair>
+template <bool kSparse, int kQ, bool kOutBf16, int kPair>
 ss_status launch_gemm(int dev, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& e,
                       const CUtensorMap& y, const ss::GemmArgs& args, cudaStream_t stream) {
-    using C = ss::GemmCfg<kSparse, kPair>;
-    auto kern = ss::gemm_kernel<kSparse, kInt8, kOutBf16, kPair>;
+    using C = ss::GemmCfg<kSparse, kPair, kQ == ss::kQBf16 ? 2 : 1>;
+    auto kern = ss::gemm_kernel<kSparse, kQ, kOutBf16, kPair>;
     static std::once_flag once[kMaxDevices];
     static cudaError_t attr_err[kMaxDevices];
     std::call_once(once[dev], [&] {
@@ -149,15 +149,30 @@ ss_status launch_gemm(int dev, const CUtensorMap& a, const CUtensorMap& b, const
     return launched();
 }
 
+// q: ss::kQE4M3, kQInt8 or kQBf16; bf16: Y element type.
 template <bool kSparse, int kPair>
-ss_status dispatch_gemm(int dev, bool int8, bool bf16, const CUtensorMap& a, const CUtensorMap& b,
+ss_status dispatch_gemm(int dev, int q, bool bf16, const CUtensorMap& a, const CUtensorMap& b,
                         const CUtensorMap& e, const CUtensorMap& y, const ss::GemmArgs& args,
                         cudaStream_t st) {
-    if (int8)
-        return bf16 ? launch_gemm<kSparse, true, true, kPair>(dev, a, b, e, y, args, st)
-                    : launch_gemm<kSparse, true, false, kPair>(dev, a, b, e, y, args, st);
-    return bf16 ? launch_gemm<kSparse, false, true, kPair>(dev, a, b, e, y, args, st)
-                : launch_gemm<kSparse, false, false, kPair>(dev, a, b, e, y, args, st);
+    using namespace ss;
+    if (q == kQInt8)
+        return bf16 ? launch_gemm<kSparse, kQInt8, true, kPair>(dev, a, b, e, y, args, st)
+                    : launch_gemm<kSparse, kQInt8, false, kPair>(dev, a, b, e, y, args, st);
+    if (q == kQBf16)
+        return bf16 ? launch_gemm<kSparse, kQBf16, true, kPair>(dev, a, b, e, y, args, st)
+                    : launch_gemm<kSparse, kQBf16, false, kPair>(dev, a, b, e, y, args, st);
+    return bf16 ? launch_gemm<kSparse, kQE4M3, true, kPair>(dev, a, b, e, y, args, st)
+                : launch_gemm<kSparse, kQE4M3, false, kPair>(dev, a, b, e, y, args, st);
+}
+
+// Operand type of the kernels for a public ss_qdtype (-1: not one).
+int kernel_q(ss_qdtype q) {
+    switch (q) {
+        case SS_INT8: return ss::kQInt8;
+        case SS_FP8_E4M3: return ss::kQE4M3;
+        case SS_BF16: return ss::kQBf16;
+    }
+    return -1;
 }
 
 template <bool kInt8, bool kAIsW>
@@ -339,10 +354,14 @@ ss_status ss_compress_weight(const void* W, ss_in_dtype in_dtype, int64_t N, int
     ss_status st = ss_slide_shape(p, K, &K_pad, &K_lift, &K_lp);
     if (st != SS_OK) return st;
     const bool dense = p.group == 0;
-    if (!W || !Wv || !s_w || (!dense && !Wm) || N <= 0 || N > INT32_MAX) return SS_ERR_INVALID_ARG;
+    const int kq = kernel_q(q);
+    if (kq < 0) return SS_ERR_INVALID_ARG;
+    const bool scaled = kq != ss::kQBf16;  // the bf16 tier has no scale (s_w unused)
+    if (!W || !Wv || (scaled && !s_w) || (!dense && !Wm) || N <= 0 || N > INT32_MAX)
+        return SS_ERR_INVALID_ARG;
     if (in_dtype != SS_IN_F32 && in_dtype != SS_IN_BF16) return SS_ERR_INVALID_ARG;
-    if (q != SS_INT8 && q != SS_FP8_E4M3) return SS_ERR_INVALID_ARG;
-    if (!aligned16(W) || !aligned16(Wv) || !aligned16(s_w) || (!dense && !aligned16(Wm)))
+    if (!aligned16(W) || !aligned16(Wv) || (scaled && !aligned16(s_w)) ||
+        (!dense && !aligned16(Wm)))
         return SS_ERR_ALIGNMENT;
     const size_t smem = static_cast<size_t>((K_pad * 4 + 15) / 16 * 16) +
                         (dense ? 0 : 2 * static_cast<size_t>(K_pad / p.group)) + 16;
@@ -354,19 +373,21 @@ ss_status ss_compress_weight(const void* W, ss_in_dtype in_dtype, int64_t N, int
     uint8_t* wm = static_cast<uint8_t*>(Wm);
     // sparse: one more CTA per padding row of the last 128-row metadata tile
     const int64_t rows_grid = dense ? N : (N + 127) / 128 * 128;
-#define SS_COMPRESS(T, I8)                                                                     \
+#define SS_COMPRESS(T, Q)                                                                      \
     do {                                                                                      \
-        auto kern = ss::compress_weight_kernel<T, I8>;                                        \
+        auto kern = ss::compress_weight_kernel<T, Q>;                                         \
         if ((st = set_smem(kern, dev, smem)) != SS_OK) return st;                             \
         kern<<<static_cast<unsigned>(rows_grid), ss::kCompressThreads, smem, s>>>(            \
             static_cast<const T*>(W), N, K, p.keep, p.group, K_lift, K_lp, wv, wm, s_w);      \
     } while (0)
     if (in_dtype == SS_IN_BF16) {
-        if (q == SS_INT8) SS_COMPRESS(__nv_bfloat16, true);
-        else SS_COMPRESS(__nv_bfloat16, false);
+        if (kq == ss::kQInt8) SS_COMPRESS(__nv_bfloat16, ss::kQInt8);
+        else if (kq == ss::kQBf16) SS_COMPRESS(__nv_bfloat16, ss::kQBf16);
+        else SS_COMPRESS(__nv_bfloat16, ss::kQE4M3);
     } else {
-        if (q == SS_INT8) SS_COMPRESS(float, true);
-        else SS_COMPRESS(float, false);
+        if (kq == ss::kQInt8) SS_COMPRESS(float, ss::kQInt8);
+        else if (kq == ss::kQBf16) SS_COMPRESS(float, ss::kQBf16);
+        else SS_COMPRESS(float, ss::kQE4M3);
     }
 #undef SS_COMPRESS
     return launched();
@@ -378,10 +399,31 @@ ss_status ss_quant_lift_act(const void* X, ss_in_dtype in_dtype, int64_t M, int6
     int64_t K_pad, K_lift, K_lp;
     ss_status st = ss_slide_shape(p, K, &K_pad, &K_lift, &K_lp);
     if (st != SS_OK) return st;
-    if (!X || !Xq_lift || !s_x || M <= 0 || M > INT32_MAX) return SS_ERR_INVALID_ARG;
+    const int kq = kernel_q(q);
+    if (kq < 0) return SS_ERR_INVALID_ARG;
+    const bool scaled = kq != ss::kQBf16;  // the bf16 tier only lifts (s_x unused)
+    if (!X || !Xq_lift || (scaled && !s_x) || M <= 0 || M > INT32_MAX) return SS_ERR_INVALID_ARG;
     if (in_dtype != SS_IN_F32 && in_dtype != SS_IN_BF16) return SS_ERR_INVALID_ARG;
-    if (q != SS_INT8 && q != SS_FP8_E4M3) return SS_ERR_INVALID_ARG;
-    if (!aligned16(X) || !aligned16(Xq_lift) || !aligned16(s_x)) return SS_ERR_ALIGNMENT;
+    if (!aligned16(X) || !aligned16(Xq_lift) || (scaled && !aligned16(s_x)))
+        return SS_ERR_ALIGNMENT;
+    if (!scaled) {
+        int dev;
+        if ((st = check_device(&dev)) != SS_OK) return st;
+        cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+        const int Nh = p.group / 2;
+        const int64_t units =
+            Nh <= 2 ? K_lp / 8 : K_lift / (4 * (Nh - 1)) + (K_lp - K_lift) / 4;
+        const dim3 grid(static_cast<unsigned>((units + ss::kLiftThreads - 1) / ss::kLiftThreads),
+                        static_cast<unsigned>(M < 65535 ? M : 65535));
+        uint16_t* xl = static_cast<uint16_t*>(Xq_lift);
+        if (in_dtype == SS_IN_BF16)
+            ss::lift_bf16_kernel<__nv_bfloat16><<<grid, ss::kLiftThreads, 0, s>>>(
+                static_cast<const __nv_bfloat16*>(X), M, K, Nh, K_lift, K_lp, xl);
+        else
+            ss::lift_bf16_kernel<float><<<grid, ss::kLiftThreads, 0, s>>>(
+                static_cast<const float*>(X), M, K, Nh, K_lift, K_lp, xl);
+        return launched();
+    }
     // one warp per token row; sliding patterns keep a quantised byte row per
     // warp in shared memory
     // one code row per row slot, with one zero chunk past the last group
@@ -461,10 +503,13 @@ ss_status ss_prune_act_2to4(const void* X, ss_in_dtype in_dtype, int64_t M, int6
     int64_t K_lp;
     ss_status st = ss_act_2to4_shape(K, &K_lp);
     if (st != SS_OK) return st;
-    if (!X || !Xv || !Xm || !s_x || M <= 0 || M > INT32_MAX) return SS_ERR_INVALID_ARG;
+    const int kq = kernel_q(q);
+    if (kq < 0) return SS_ERR_INVALID_ARG;
+    const bool scaled = kq != ss::kQBf16;  // the bf16 tier has no scale (s_x unused)
+    if (!X || !Xv || !Xm || (scaled && !s_x) || M <= 0 || M > INT32_MAX)
+        return SS_ERR_INVALID_ARG;
     if (in_dtype != SS_IN_F32 && in_dtype != SS_IN_BF16) return SS_ERR_INVALID_ARG;
-    if (q != SS_INT8 && q != SS_FP8_E4M3) return SS_ERR_INVALID_ARG;
-    if (!aligned16(X) || !aligned16(Xv) || !aligned16(Xm) || !aligned16(s_x))
+    if (!aligned16(X) || !aligned16(Xv) || !aligned16(Xm) || (scaled && !aligned16(s_x)))
         return SS_ERR_ALIGNMENT;
     int dev;
     if ((st = check_device(&dev)) != SS_OK) return st;
@@ -474,17 +519,19 @@ ss_status ss_prune_act_2to4(const void* X, ss_in_dtype in_dtype, int64_t M, int6
     const int warps = ss::kWarpRowThreads / 32;
     // warps past M zero the padding rows of the last 128-row metadata tile
     const unsigned grid = static_cast<unsigned>(((M + 127) / 128 * 128 + warps - 1) / warps);
-#define SS_PRUNE(T, I8)                                                                        \
+#define SS_PRUNE(T, Q)                                                                         \
     do {                                                                                      \
-        ss::prune_act_warp_kernel<T, I8><<<grid, ss::kWarpRowThreads, 0, s>>>(               \
+        ss::prune_act_warp_kernel<T, Q><<<grid, ss::kWarpRowThreads, 0, s>>>(                \
             static_cast<const T*>(X), M, K, K_lp, xv, xm, s_x);                               \
     } while (0)
     if (in_dtype == SS_IN_BF16) {
-        if (q == SS_INT8) SS_PRUNE(__nv_bfloat16, true);
-        else SS_PRUNE(__nv_bfloat16, false);
+        if (kq == ss::kQInt8) SS_PRUNE(__nv_bfloat16, ss::kQInt8);
+        else if (kq == ss::kQBf16) SS_PRUNE(__nv_bfloat16, ss::kQBf16);
+        else SS_PRUNE(__nv_bfloat16, ss::kQE4M3);
     } else {
-        if (q == SS_INT8) SS_PRUNE(float, true);
-        else SS_PRUNE(float, false);
+        if (kq == ss::kQInt8) SS_PRUNE(float, ss::kQInt8);
+        else if (kq == ss::kQBf16) SS_PRUNE(float, ss::kQBf16);
+        else SS_PRUNE(float, ss::kQE4M3);
     }
 #undef SS_PRUNE
     return launched();
@@ -494,11 +541,13 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
                          const void* B, const float* s_b, int64_t M, int64_t N, int64_t K_lp,
                          ss_qdtype q, void* Y, ss_out_dtype out_dtype, ss_stream_t stream) {
     if (sparse_operand != 0 && sparse_operand != 1) return SS_ERR_INVALID_ARG;
-    if (!Av || !Am || !s_a || !B || !s_b || !Y) return SS_ERR_INVALID_ARG;
+    const int kq = kernel_q(q);
+    if (kq < 0) return SS_ERR_INVALID_ARG;
+    const bool scaled = kq != ss::kQBf16;  // bf16 tier: s_a, s_b unused
+    if (!Av || !Am || (scaled && (!s_a || !s_b)) || !B || !Y) return SS_ERR_INVALID_ARG;
     if (M <= 0 || N <= 0 || M > INT32_MAX || N > INT32_MAX || K_lp <= 0 || K_lp % 128 != 0 ||
         K_lp > (int64_t{1} << 30))
         return SS_ERR_INVALID_ARG;
-    if (q != SS_INT8 && q != SS_FP8_E4M3) return SS_ERR_INVALID_ARG;
     if (out_dtype != SS_OUT_F32 && out_dtype != SS_OUT_BF16) return SS_ERR_INVALID_ARG;
     if (!aligned16(Av) || !aligned16(Am) || !aligned16(B) || !aligned16(Y)) return SS_ERR_ALIGNMENT;
     int dev;
@@ -508,19 +557,23 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
     const int64_t rowsB = sparse_operand == 0 ? M : N;
     const int pair = rowsA > ss::kTileA ? 2 : 1;
     const int bn = choose_bn(rowsB, ss::GemmCfg<true, 1>::kBnMax);
+    // operand element bytes: the maps address bytes, so a bf16 row is twice as wide
+    const int64_t eb = scaled ? 1 : 2;
     CUtensorMap ta, tb, te;
     using CS = ss::GemmCfg<true, 1>;
-    if (!make_map_2d(&ta, Av, rowsA, K_lp / 2, ss::kTileA, CS::kARowBytes,
+    if (!make_map_2d(&ta, Av, rowsA, K_lp / 2 * eb, ss::kTileA, CS::kARowBytes,
                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_2d(&tb, B, rowsB, K_lp, bn / pair, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tb, B, rowsB, K_lp * eb, bn / pair, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&te, Am, (rowsA + 127) / 128 * (K_lp / 128) * 16, 128, 16, 128,
                      CU_TENSOR_MAP_SWIZZLE_NONE))
         return SS_ERR_CUDA;
     ss::GemmArgs args;
     args.rowsA = static_cast<int>(rowsA);
     args.rowsB = static_cast<int>(rowsB);
-    // a last half stage (K_lp an odd multiple of 128) reads zeros past the rows
-    args.k_stages = static_cast<int>((K_lp + CS::kStageK - 1) / CS::kStageK);
+    // 8-bit: a last half stage (K_lp an odd multiple of 128) reads zeros past
+    // the rows; bf16 stages are 128 K
+    const int64_t stage_k = scaled ? CS::kStageK : ss::GemmCfg<true, 1, 2>::kStageK;
+    args.k_stages = static_cast<int>((K_lp + stage_k - 1) / stage_k);
     args.bn = bn;
     args.a_is_w = sparse_operand == 0 ? 1 : 0;
     args.ldy = static_cast<int>(N);
@@ -534,10 +587,11 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
     cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
     const bool i8 = q == SS_INT8, bf = out_dtype == SS_OUT_BF16;
 #if SS_SPARSE_WIDE
+    // (8-bit operands only: the bf16 tier runs the one-B-tile kernel)
     // Large problems with bf16 Y may take two B tiles per output tile: fewer
     // bytes per MMA, but single-buffered accumulators.
     const int forced = forced_sparse_kernel();
-    if (pair == 2 && args.tma_store && forced != 1 &&
+    if (scaled && pair == 2 && args.tma_store && forced != 1 &&
         (forced == 2 || (rowsB > 2 * ss::WideCfg::kBnMax &&
                          prefer_wide(rowsA, rowsB, bn, g_num_sms[dev] / 2)))) {
         using CW = ss::WideCfg;
@@ -557,18 +611,20 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
                   : launch_gemm_wide<false, false>(dev, wa, wb, te, ty, wargs, st_);
     }
 #endif
-    if (pair == 1) return dispatch_gemm<true, 1>(dev, i8, bf, ta, tb, te, ty, args, st_);
-    return dispatch_gemm<true, 2>(dev, i8, bf, ta, tb, te, ty, args, st_);
+    if (pair == 1) return dispatch_gemm<true, 1>(dev, kq, bf, ta, tb, te, ty, args, st_);
+    return dispatch_gemm<true, 2>(dev, kq, bf, ta, tb, te, ty, args, st_);
 }
 
 ss_status ss_dense_gemm(const void* Xq, const float* s_x, const void* Wq, const float* s_w,
                         int64_t M, int64_t N, int64_t K_p, ss_qdtype q, void* Y,
                         ss_out_dtype out_dtype, ss_stream_t stream) {
-    if (!Xq || !s_x || !Wq || !s_w || !Y) return SS_ERR_INVALID_ARG;
+    const int kq = kernel_q(q);
+    if (kq < 0) return SS_ERR_INVALID_ARG;
+    const bool scaled = kq != ss::kQBf16;  // bf16 tier: s_x, s_w unused
+    if (!Xq || (scaled && (!s_x || !s_w)) || !Wq || !Y) return SS_ERR_INVALID_ARG;
     if (M <= 0 || N <= 0 || M > INT32_MAX || N > INT32_MAX || K_p <= 0 || K_p % 128 != 0 ||
         K_p > (int64_t{1} << 30))
         return SS_ERR_INVALID_ARG;
-    if (q != SS_INT8 && q != SS_FP8_E4M3) return SS_ERR_INVALID_ARG;
     if (out_dtype != SS_OUT_F32 && out_dtype != SS_OUT_BF16) return SS_ERR_INVALID_ARG;
     if (!aligned16(Xq) || !aligned16(Wq) || !aligned16(Y)) return SS_ERR_ALIGNMENT;
     int dev;
@@ -576,14 +632,15 @@ ss_status ss_dense_gemm(const void* Xq, const float* s_x, const void* Wq, const 
     if (st != SS_OK) return st;
     const int pair = N > ss::kTileA ? 2 : 1;
     const int bn = choose_bn(M, ss::GemmCfg<false, 1>::kBnMax);
+    const int64_t eb = scaled ? 1 : 2;  // operand element bytes
     CUtensorMap ta, tb;
-    if (!make_map_2d(&ta, Wq, N, K_p, ss::kTileA, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_2d(&tb, Xq, M, K_p, bn / pair, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!make_map_2d(&ta, Wq, N, K_p * eb, ss::kTileA, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tb, Xq, M, K_p * eb, bn / pair, 128, CU_TENSOR_MAP_SWIZZLE_128B))
         return SS_ERR_CUDA;
     ss::GemmArgs args;
     args.rowsA = static_cast<int>(N);
     args.rowsB = static_cast<int>(M);
-    args.k_stages = static_cast<int>(K_p / 128);
+    args.k_stages = static_cast<int>(K_p * eb / 128);  // 128 bytes of K per stage
     args.bn = bn;
     args.a_is_w = 1;
     args.ldy = static_cast<int>(N);
@@ -594,9 +651,9 @@ ss_status ss_dense_gemm(const void* Xq, const float* s_x, const void* Wq, const 
     args.tma_store = make_y_map(&ty, Y, M, N, out_dtype == SS_OUT_BF16, true) ? 1 : 0;
     if (!args.tma_store) ty = ta;  // unused
     cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
-    const bool i8 = q == SS_INT8, bf = out_dtype == SS_OUT_BF16;
-    return pair == 2 ? dispatch_gemm<false, 2>(dev, i8, bf, ta, tb, ta, ty, args, st_)
-                     : dispatch_gemm<false, 1>(dev, i8, bf, ta, tb, ta, ty, args, st_);
+    const bool bf = out_dtype == SS_OUT_BF16;
+    return pair == 2 ? dispatch_gemm<false, 2>(dev, kq, bf, ta, tb, ta, ty, args, st_)
+                     : dispatch_gemm<false, 1>(dev, kq, bf, ta, tb, ta, ty, args, st_);
 }
 
 ss_status ss_get_device_status(ss_stream_t stream) {

@@ -107,6 +107,18 @@ __host__ __device__ __forceinline__ int64_t meta_offset(int64_t r, int64_t b, in
     return ((r >> 7) * (K_lp >> 7) + (b >> 4)) * 2048 + (r & 127) * 16 + (b & 15);
 }
 
+// The 16-bit sparse MMA (kind::f16) reads the 32 selector bits of one MMA for
+// rows r and r + 8 of each 16-row group from one tensor-memory column as two
+// 16-bit halves (the pairing of the warp-level 16-bit sparse MMA's metadata
+// register).  The bf16 tier therefore stores the selectors with row bit 3 and
+// byte bit 1 exchanged inside that layout: the 2-byte half h of 4-byte word c
+// of row r lands in row (r & ~8) | 8h, half ((r >> 3) & 1) of the same word.
+__host__ __device__ __forceinline__ int64_t meta_offset_i16(int64_t r, int64_t b, int64_t K_lp) {
+    const int64_t r2 = (r & ~int64_t{8}) | (((b >> 1) & 1) << 3);
+    const int64_t b2 = (b & ~int64_t{2}) | (((r >> 3) & 1) << 1);
+    return meta_offset(r2, b2, K_lp);
+}
+
 // ---------------------------------------------------------------------------
 // TMA (no multicast anywhere in this library).
 // ---------------------------------------------------------------------------
@@ -250,6 +262,8 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
 }
 
 // Instruction descriptor for kind::i8 / kind::f8f6f4, both operands K-major.
+//   bits 0-1   sparsity selector (which part of an aligned metadata column
+//              pair a sparse MMA reads; 0 for the 8-bit kinds)
 //   bit 2      sparse flag
 //   bits 4-5   accumulator format (1 = f32, 2 = s32)
 //   bits 7-9   A format, 10-12 B format (i8: 1 = signed; f8f6f4: 0 = E4M3)
@@ -258,6 +272,23 @@ __host__ __device__ constexpr uint32_t make_idesc(bool sparse, bool is_int8, uin
                                                   uint32_t N) {
     return (sparse ? (1u << 2) : 0u) | ((is_int8 ? 2u : 1u) << 4) | ((is_int8 ? 1u : 0u) << 7) |
            ((is_int8 ? 1u : 0u) << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// Operand types of the GEMM kernels: the two 8-bit kinds and the 16-bit tier
+// (bf16 operands, kind::f16, fp32 accumulator, no scales).
+constexpr int kQE4M3 = 0;
+constexpr int kQInt8 = 1;
+constexpr int kQBf16 = 2;
+
+// Instruction descriptor for kind::f16 with bf16 A and B (format 1 in bits
+// 7-9 and 10-12), fp32 accumulator, both operands K-major.
+__host__ __device__ constexpr uint32_t make_idesc_bf16(bool sparse, uint32_t M, uint32_t N) {
+    return (sparse ? (1u << 2) : 0u) | (1u << 4) | (1u << 7) | (1u << 10) | ((N >> 3) << 17) |
+           ((M >> 4) << 24);
+}
+
+__host__ __device__ constexpr uint32_t make_idesc_q(bool sparse, int q, uint32_t M, uint32_t N) {
+    return q == kQBf16 ? make_idesc_bf16(sparse, M, N) : make_idesc(sparse, q == kQInt8, M, N);
 }
 
 template <bool kInt8>
@@ -490,6 +521,45 @@ __device__ __forceinline__ void mma_sparse_g(uint32_t d_tmem, uint64_t a_desc, u
     }
 }
 
+// kind::f16 MMAs of the bf16 tier (dense K = 16, sparse K = 32 per MMA).
+template <int kPair>
+__device__ __forceinline__ void mma_dense_bf16_g(uint32_t d_tmem, uint64_t a_desc,
+                                                 uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+    if constexpr (kPair == 2)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+            : "memory");
+}
+
+template <int kPair>
+__device__ __forceinline__ void mma_sparse_bf16_g(uint32_t d_tmem, uint64_t a_desc,
+                                                  uint64_t b_desc, uint32_t e_tmem,
+                                                  uint32_t idesc, uint32_t accumulate) {
+    if constexpr (kPair == 2)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %5, 0;\n\t"
+            "tcgen05.mma.sp.cta_group::2.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(
+                d_tmem),
+            "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %5, 0;\n\t"
+            "tcgen05.mma.sp.cta_group::1.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(
+                d_tmem),
+            "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+            : "memory");
+}
+
 // Two fp32 products in one instruction (mul.rn.f32x2): (a0 * b0, a1 * b1),
 // each rounded to nearest even as __fmul_rn would.
 __device__ __forceinline__ void mul_rn_f32x2(float a0, float a1, float b0, float b1, float& r0,
@@ -565,6 +635,11 @@ __device__ __forceinline__ uint32_t quantize(float x, float inv) {
     } else {
         return static_cast<uint32_t>(__nv_cvt_float_to_fp8(p, __NV_SATFINITE, __NV_E4M3));
     }
+}
+
+// bf16 bits of x, rounded to nearest even (the stored values of the bf16 tier).
+__device__ __forceinline__ uint32_t bf16_bits(float x) {
+    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(x)));
 }
 
 template <typename T>

@@ -5,6 +5,9 @@
 // Fig. 2: windows 0-3, 2-5, 4-7 of each group of 8 for 6:8; LLM-Compressor
 // W8A8: channel-wise weight scales).
 //
+// The bf16 tier (kQ = kQBf16) stores the kept weights as bf16 (round to
+// nearest even), two bytes per value, and has no scale.
+//
 // One CTA per output channel.  Pass 1 stages the row in shared memory, marks
 // the kept positions of every group (keep the 2Nh-2 largest |w|, ties keep the
 // lower index) and reduces the absmax of the kept weights.  Pass 2 walks the
@@ -72,16 +75,22 @@ __device__ __forceinline__ void window_indices(uint32_t own, int& i0, int& i1) {
     i1 = max(idx[0], idx[1]);
 }
 
-template <typename T, bool kInt8>
+template <typename T, int kQ>
 __global__ void __launch_bounds__(kCompressThreads) compress_weight_kernel(
     const T* __restrict__ W, int64_t N, int64_t K, int keep, int group, int64_t K_lift,
     int64_t K_lp, uint8_t* __restrict__ Wv, uint8_t* __restrict__ Wm, float* __restrict__ s_w) {
+    constexpr bool kInt8 = kQ == kQInt8;
+    constexpr bool kBf16 = kQ == kQBf16;
     extern __shared__ __align__(16) uint8_t smem_raw[];
     __shared__ float red[32];
     __shared__ int bad;
     const int64_t n = blockIdx.x;
+    // selector byte b of row n in the storage layout of this tier
+    auto meta_at = [&](int64_t b) -> uint8_t& {
+        return Wm[kQ == kQBf16 ? meta_offset_i16(n, b, K_lp) : meta_offset(n, b, K_lp)];
+    };
     if (n >= N) {  // padding row of the last 128-row metadata tile
-        for (int64_t b = threadIdx.x; b < K_lp / 8; b += blockDim.x) Wm[meta_offset(n, b, K_lp)] = 0;
+        for (int64_t b = threadIdx.x; b < K_lp / 8; b += blockDim.x) meta_at(b) = 0;
         return;
     }
     const T* w = W + n * K;
@@ -124,22 +133,35 @@ __global__ void __launch_bounds__(kCompressThreads) compress_weight_kernel(
         if (threadIdx.x == 0) record_status(kErrData);
         return;
     }
-    float inv, s;
-    scale_from_absmax<kInt8>(a, inv, s);
-    if (threadIdx.x == 0) s_w[n] = s;
+    float inv = 0.0f, s;
+    if constexpr (!kBf16) {
+        scale_from_absmax<kInt8>(a, inv, s);
+        if (threadIdx.x == 0) s_w[n] = s;
+    }
+    // stored code of one kept value
+    auto code = [&](float v) -> uint32_t {
+        if constexpr (kBf16) return bf16_bits(v);
+        else return quantize<kInt8>(v, inv);
+    };
 
     if (dense) {
-        uint8_t* out = Wv + n * K_lp;
-        for (int64_t k = threadIdx.x; k < K_lp; k += blockDim.x)
-            out[k] = k < K ? static_cast<uint8_t>(quantize<kInt8>(srow[k], inv)) : 0;
+        if constexpr (kBf16) {
+            uint16_t* out = reinterpret_cast<uint16_t*>(Wv) + n * K_lp;
+            for (int64_t k = threadIdx.x; k < K_lp; k += blockDim.x)
+                out[k] = k < K ? static_cast<uint16_t>(code(srow[k])) : 0;
+        } else {
+            uint8_t* out = Wv + n * K_lp;
+            for (int64_t k = threadIdx.x; k < K_lp; k += blockDim.x)
+                out[k] = k < K ? static_cast<uint8_t>(code(srow[k])) : 0;
+        }
         return;
     }
     const int Nh = group / 2;
     const int64_t n_win = K_lift / 4;
-    uint8_t* vrow = Wv + n * (K_lp / 2);
+    uint8_t* vrow = Wv + n * (K_lp / 2) * (kBf16 ? 2 : 1);
     const uint8_t* kept_hi = kept + K_pad / group;
     for (int64_t pr = threadIdx.x; pr < K_lp / 8; pr += blockDim.x) {
-        uint32_t vals = 0;
+        uint32_t vals[2] = {0u, 0u};  // 8-bit: vals[0] holds both windows
         uint32_t meta = 0;
         for (int h = 0; h < 2; ++h) {
             const int64_t win = pr * 2 + h;
@@ -154,13 +176,19 @@ __global__ void __launch_bounds__(kCompressThreads) compress_weight_kernel(
             }
             int i0, i1;
             window_indices(own, i0, i1);
-            const uint32_t q0 = ((own >> i0) & 1u) ? quantize<kInt8>(srow[base + i0], inv) : 0u;
-            const uint32_t q1 = ((own >> i1) & 1u) ? quantize<kInt8>(srow[base + i1], inv) : 0u;
-            vals |= (q0 | (q1 << 8)) << (16 * h);
+            const uint32_t q0 = ((own >> i0) & 1u) ? code(srow[base + i0]) : 0u;
+            const uint32_t q1 = ((own >> i1) & 1u) ? code(srow[base + i1]) : 0u;
+            if constexpr (kBf16)
+                vals[h] = q0 | (q1 << 16);
+            else
+                vals[0] |= (q0 | (q1 << 8)) << (16 * h);
             meta |= static_cast<uint32_t>(i0 | (i1 << 2)) << (4 * h);
         }
-        reinterpret_cast<uint32_t*>(vrow)[pr] = vals;  // 4 value bytes
-        Wm[meta_offset(n, pr, K_lp)] = static_cast<uint8_t>(meta);
+        if constexpr (kBf16)
+            reinterpret_cast<uint2*>(vrow)[pr] = make_uint2(vals[0], vals[1]);  // 4 values
+        else
+            reinterpret_cast<uint32_t*>(vrow)[pr] = vals[0];  // 4 value bytes
+        meta_at(pr) = static_cast<uint8_t>(meta);
     }
 }
 

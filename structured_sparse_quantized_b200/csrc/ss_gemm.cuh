@@ -48,17 +48,23 @@ constexpr int kGemmThreads = 192;
 constexpr int kTileA = 128;  // A rows per CTA per A tile
 constexpr int kTmemCols = 512;
 
-template <bool kSparse, int kPair>
+template <bool kSparse, int kPair, int kEb = 1>
 struct GemmCfg {
-    // One pipeline stage covers kStageK logical K: dense 128 (4 MMAs of K=32),
-    // sparse 256 (4 MMAs of K=64).  Either way an A row holds 128 bytes of the
-    // stage (128B swizzle).
-    static constexpr int kStageK = kSparse ? 256 : 128;
-    static constexpr int kMmaK = kSparse ? 64 : 32;
+    // One pipeline stage covers kStageK logical K: for 8-bit operands dense
+    // 128 (4 MMAs of K=32) and sparse 256 (4 MMAs of K=64); for bf16 (kEb = 2
+    // bytes) half of that, 4 MMAs of K=16 / K=32.  Either way an A row holds
+    // 128 bytes of the stage (128B swizzle) and each MMA reads 32 bytes of an
+    // A row and 32 (dense) or 64 (sparse) bytes of a B row.
+    static constexpr int kStageK = (kSparse ? 256 : 128) / kEb;
+    static constexpr int kMmaK = (kSparse ? 64 : 32) / kEb;
     static constexpr int kMmaPerStage = kStageK / kMmaK;
-    static constexpr int kARowBytes = kSparse ? kStageK / 2 : kStageK;  // 128
+    static constexpr int kARowBytes = kSparse ? kStageK * kEb / 2 : kStageK * kEb;  // 128
     static constexpr int kABytes = kTileA * kARowBytes;    // one A tile, 16 KB
-    static constexpr int kBAtoms = kStageK / 128;          // 128-byte K atoms of B per stage
+    static constexpr int kBAtoms = kStageK * kEb / 128;    // 128-byte K atoms of B per stage
+    // Metadata of a sparse MMA is addressed in tensor memory as aligned pairs
+    // of 32-bit columns: an 8-bit MMA (K=64, 64 selector bits per row) uses a
+    // whole pair, a bf16 MMA (K=32, 32 bits) one column of it, picked by the
+    // sparsity selector of the instruction descriptor (bits 0-1).
     static constexpr int kBnMax = kSparse ? 224 : 256;     // MMA N; accumulators + metadata
     static constexpr int kBRowsMax = kBnMax / kPair;       // B rows held per CTA
     static constexpr int kBAtomBytes = kBRowsMax * 128;
@@ -84,7 +90,9 @@ struct GemmCfg {
     static constexpr int kSmemBytes =
         kEpiOffset + 2 * kEpiBytes + 1024 /*align*/ + 256 /*barriers*/;
     static_assert(kABytes % 1024 == 0 && kBAtomBytes % 1024 == 0, "tile alignment");
+    static_assert(kARowBytes == 128 && kMmaPerStage == 4, "stage geometry");
     static_assert(!kSparse || kECol + kESlots * kESlotCols <= kTmemCols, "TMEM budget");
+    static_assert(kECol % 2 == 0 && kESlotCols % 2 == 0, "metadata column pairs stay aligned");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
     static_assert(kStages >= (kPair == 2 ? 3 : 2), "pipeline depth");
     static_assert((2 * kStages + 5) * 8 + 4 <= 256, "barrier area");
@@ -93,7 +101,7 @@ struct GemmCfg {
 struct GemmArgs {
     int rowsA;        // rows of A
     int rowsB;        // rows of B
-    int k_stages;     // ceil(K / kStageK)
+    int k_stages;     // ceil(K_lp / kStageK)
     int bn;           // B rows per tile (MMA N; multiple of 32, <= kBnMax)
     int a_is_w;       // 1: A rows are output channels (Y[b, a]); 0: Y[a, b]
     int ldy;          // leading dimension of Y (= N)
@@ -117,12 +125,23 @@ __device__ __forceinline__ void store_scaled(void* y, int64_t off, uint32_t acc_
         reinterpret_cast<float*>(y)[off] = v;
 }
 
-template <bool kSparse, bool kInt8, bool kOutBf16, int kPair>
+// Scale of row i, or 1 for the unscaled bf16 tier (the product with 1.0f
+// is exact, so both tiers share the epilogue arithmetic).
+template <bool kUnit>
+__device__ __forceinline__ float load_scale(const float* s, int i, bool in_range) {
+    if constexpr (kUnit) return 1.0f;
+    else return in_range ? __ldg(s + i) : 0.0f;
+}
+
+// kQ: kQE4M3, kQInt8 (kind::f8f6f4 / kind::i8) or kQBf16 (kind::f16).
+template <bool kSparse, int kQ, bool kOutBf16, int kPair>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_e, const __grid_constant__ CUtensorMap tm_y,
                 const GemmArgs args) {
-    using C = GemmCfg<kSparse, kPair>;
+    constexpr bool kInt8 = kQ == kQInt8;
+    constexpr bool kBf16 = kQ == kQBf16;
+    using C = GemmCfg<kSparse, kPair, kBf16 ? 2 : 1>;
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -209,7 +228,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                         for (int u = 0; u < C::kBAtoms; ++u)
                             tma_load_2d_pair_hint(st + C::kBOffset + u * C::kBAtomBytes, &tm_b,
-                                                  fb, kb * C::kStageK + u * 128, b0, keep);
+                                                  fb, (kb * C::kBAtoms + u) * 128, b0, keep);
 #pragma unroll
                         for (int u = 0; u < C::kEChunks; ++u)
                             tma_load_2d_pair_hint(st + C::kEOffset + u * kTileA * 16, &tm_e, fb, 0,
@@ -221,7 +240,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                         for (int u = 0; u < C::kBAtoms; ++u)
                             tma_load_2d(st + C::kBOffset + u * C::kBAtomBytes, &tm_b, &full[s],
-                                        kb * C::kStageK + u * 128, b0);
+                                        (kb * C::kBAtoms + u) * 128, b0);
 #pragma unroll
                         for (int u = 0; u < C::kEChunks; ++u)
                             tma_load_2d(st + C::kEOffset + u * kTileA * 16, &tm_e, &full[s], 0,
@@ -252,7 +271,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // Descriptors are built once; a stage, A tile or K step only adds its
         // byte offset (>> 4) to the start-address field.
         if (leader) {
-            const uint32_t idesc = make_idesc(kSparse, kInt8, pair_rows, args.bn);
+            const uint32_t idesc = make_idesc_q(kSparse, kQ, pair_rows, args.bn);
             const uint32_t base = smem_u32(smem);
             const uint64_t a_desc0 = smem_desc(base, 16, 8 * C::kARowBytes, kSwizzle128B);
             const uint64_t b_desc0 = smem_desc(base + C::kBOffset, 16, 1024, kSwizzle128B);
@@ -293,16 +312,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                 const uint64_t b_desc =
                                     b_desc0 + soff +
                                     (((j >> 1) * C::kBAtomBytes + (j & 1) * 64) >> 4);
-                                mma_sparse_g<kPair, kInt8>(d_tmem, a_desc, b_desc, e_tmem + 2 * j,
-                                                           idesc, (kb > 0 || j > 0) ? 1u : 0u);
+                                const uint32_t accum = (kb > 0 || j > 0) ? 1u : 0u;
+                                if constexpr (kBf16)  // 32 selector bits: half j & 1 of a pair
+                                    mma_sparse_bf16_g<kPair>(d_tmem, a_desc, b_desc,
+                                                             e_tmem + 2 * (j >> 1),
+                                                             idesc | static_cast<uint32_t>(j & 1),
+                                                             accum);
+                                else
+                                    mma_sparse_g<kPair, kInt8>(d_tmem, a_desc, b_desc,
+                                                               e_tmem + 2 * j, idesc, accum);
                             }
                         } else {
 #pragma unroll
                             for (int j = 0; j < C::kMmaPerStage; ++j) {
                                 const uint64_t a_desc = a_desc0 + soff + ((j * 32) >> 4);
                                 const uint64_t b_desc = b_desc0 + soff + ((j * 32) >> 4);
-                                mma_dense_g<kPair, kInt8>(d_tmem, a_desc, b_desc, idesc,
-                                                          (kb > 0 || j > 0) ? 1u : 0u);
+                                const uint32_t accum = (kb > 0 || j > 0) ? 1u : 0u;
+                                if constexpr (kBf16)
+                                    mma_dense_bf16_g<kPair>(d_tmem, a_desc, b_desc, idesc, accum);
+                                else
+                                    mma_dense_g<kPair, kInt8>(d_tmem, a_desc, b_desc, idesc,
+                                                              accum);
                             }
                         }
                     }
@@ -359,7 +389,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int a_cta0 = a_tile0;
             const int a_row = a_cta0 + lane_row;
             const bool row_ok = a_row < args.rowsA;
-            const float sa = row_ok ? __ldg(args.s_a + a_row) : 0.0f;
+            const float sa = load_scale<kBf16>(args.s_a, a_row, row_ok);
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    static_cast<uint32_t>(acc * C::kAccStride);
             if (args.tma_store && args.a_is_w) {
@@ -375,7 +405,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int ch = a_cta0 + q * 32 + 16 * h + t4 + 8 * e;
-                        sa2[h][e] = ch < args.rowsA ? __ldg(args.s_a + ch) : 0.0f;
+                        sa2[h][e] = load_scale<kBf16>(args.s_a, ch, ch < args.rowsA);
                     }
                 // this thread's stmatrix row: matrix mi, row mj
                 const int mi = lane >> 3, mj = lane & 7;
@@ -400,7 +430,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                         for (int e = 0; e < 2; ++e) {
                             const int tok = b0 + c + 8 * r + 2 * tm + e;
-                            sb[r][e] = tok < args.rowsB ? __ldg(args.s_b + tok) : 0.0f;
+                            sb[r][e] = load_scale<kBf16>(args.s_b, tok, tok < args.rowsB);
                         }
                     uint32_t pk[2][8];  // [half][column group r * 2 + channel block]
 #pragma unroll
@@ -468,7 +498,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
                 const int bc = b0 + c + lane;  // this lane's B row of the chunk
-                const float sb_lane = bc < args.rowsB ? __ldg(args.s_b + bc) : 0.0f;
+                const float sb_lane = load_scale<kBf16>(args.s_b, bc, bc < args.rowsB);
                 if (args.tma_store) {
                     uint8_t* sy = stage_y + (chunk_iter & 1) * C::kEpiBytes;
                     if (issuer) bulk_wait_read<1>();  // the store of two chunks ago has read it

@@ -275,17 +275,33 @@ __global__ void __launch_bounds__(kWarpRowThreads) quant_lift_warp_kernel(
     }
 }
 
-template <typename T, bool kInt8>
+// Online 2:4 prune + compress of one token row per warp.  The 8-bit tiers
+// take the row absmax first and quantise the kept values; the bf16 tier
+// (kQ = kQBf16) keeps them as bf16 (two bytes each, no scale, one pass).
+template <typename T, int kQ>
 __global__ void __launch_bounds__(kWarpRowThreads) prune_act_warp_kernel(
     const T* __restrict__ X, int64_t M, int64_t K64, int64_t K_lp64, uint8_t* __restrict__ Xv,
     uint8_t* __restrict__ Xm, float* __restrict__ s_x) {
+    constexpr bool kInt8 = kQ == kQInt8;
+    constexpr bool kBf16 = kQ == kQBf16;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t m = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
     const int64_t M_pad = (M + 127) / 128 * 128;
     if (m >= M_pad) return;
+    // the 4 selector bytes of step st (one word; the bf16 tier stores its two
+    // halves in rows m and m ^ 8, see meta_offset_i16)
+    auto put_meta = [&](int64_t st, uint32_t nibs) {
+        if constexpr (kBf16) {
+            __stcs(reinterpret_cast<uint16_t*>(Xm + meta_offset_i16(m, 4 * st, K_lp64)),
+                   static_cast<uint16_t>(nibs & 0xFFFFu));
+            __stcs(reinterpret_cast<uint16_t*>(Xm + meta_offset_i16(m, 4 * st + 2, K_lp64)),
+                   static_cast<uint16_t>(nibs >> 16));
+        } else {
+            __stcs(reinterpret_cast<uint32_t*>(Xm + meta_offset(m, 4 * st, K_lp64)), nibs);
+        }
+    };
     if (m >= M) {  // padding row of the last 128-row metadata tile
-        for (int64_t st = lane; st < K_lp64 / 32; st += 32)
-            *reinterpret_cast<uint32_t*>(Xm + meta_offset(m, 4 * st, K_lp64)) = 0u;
+        for (int64_t st = lane; st < K_lp64 / 32; st += 32) put_meta(st, 0u);
         return;
     }
     const int K = static_cast<int>(K64);
@@ -293,12 +309,17 @@ __global__ void __launch_bounds__(kWarpRowThreads) prune_act_warp_kernel(
     const T* x = X + m * K64;
     const bool vec = (K * static_cast<int>(sizeof(T))) % 16 == 0 &&
                      (reinterpret_cast<uintptr_t>(X) & 15) == 0;
-    const float a = warp_row_absmax<T>(x, K, vec, lane);
-    float inv, s;
-    scale_from_absmax<kInt8>(a, inv, s);
-    if (lane == 0) s_x[m] = s;
-    // One step = 8 groups of 4 = 32 inputs -> 16 value bytes + 4 nibble bytes.
-    uint4* vout = reinterpret_cast<uint4*>(Xv + m * (K_lp64 / 2));
+    float inv = 0.0f;
+    if constexpr (!kBf16) {
+        const float a = warp_row_absmax<T>(x, K, vec, lane);
+        float s;
+        scale_from_absmax<kInt8>(a, inv, s);
+        if (lane == 0) s_x[m] = s;
+    }
+    // One step = 8 groups of 4 = 32 inputs -> 16 values (16 bytes, 32 for
+    // bf16) + 4 nibble bytes.
+    constexpr int kVq = kBf16 ? 2 : 1;  // uint4 of values per step
+    uint4* vout = reinterpret_cast<uint4*>(Xv + m * (K_lp64 / 2) * (kBf16 ? 2 : 1));
     const int n_steps = K_lp / 32;
     for (int st = lane; st < n_steps; st += 32) {
         if constexpr (sizeof(T) == 2) {
@@ -307,44 +328,59 @@ __global__ void __launch_bounds__(kWarpRowThreads) prune_act_warp_kernel(
                 const uint4 c0 = __ldg(p), c1 = __ldg(p + 1), c2 = __ldg(p + 2), c3 = __ldg(p + 3);
                 const uint32_t w[16] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w,
                                         c2.x, c2.y, c2.z, c2.w, c3.x, c3.y, c3.z, c3.w};
-                uint32_t vals[4];
+                uint32_t vals[8];
                 uint32_t nibs = 0;
 #pragma unroll
                 for (int gi = 0; gi < 8; ++gi) {
                     int i0, i1;
                     const uint32_t kept = top2_of4_bf16(w[2 * gi], w[2 * gi + 1], i0, i1);
-                    const uint32_t q = quantize_pair<kInt8>(__uint_as_float(kept << 16),
-                                                            __uint_as_float(kept & 0xFFFF0000u), inv);
-                    if (gi & 1)
-                        vals[gi >> 1] |= q << 16;
-                    else
-                        vals[gi >> 1] = q;
+                    if constexpr (kBf16) {
+                        vals[gi] = kept;
+                    } else {
+                        const uint32_t q = quantize_pair<kInt8>(
+                            __uint_as_float(kept << 16), __uint_as_float(kept & 0xFFFF0000u), inv);
+                        if (gi & 1)
+                            vals[gi >> 1] |= q << 16;
+                        else
+                            vals[gi >> 1] = q;
+                    }
                     nibs |= static_cast<uint32_t>(i0 | (i1 << 2)) << (4 * gi);
                 }
-                __stcs(vout + st, make_uint4(vals[0], vals[1], vals[2], vals[3]));
-                __stcs(reinterpret_cast<uint32_t*>(Xm + meta_offset(m, 4 * st, K_lp64)), nibs);
+#pragma unroll
+                for (int v = 0; v < kVq; ++v)
+                    __stcs(vout + kVq * st + v,
+                           make_uint4(vals[4 * v], vals[4 * v + 1], vals[4 * v + 2], vals[4 * v + 3]));
+                put_meta(st, nibs);
                 continue;
             }
         }
         float f[32];
         gload16<T>(x, st * 32, K, vec, *reinterpret_cast<float(*)[16]>(f));
         gload16<T>(x, st * 32 + 16, K, vec, *reinterpret_cast<float(*)[16]>(f + 16));
-        uint32_t vals[4];
+        uint32_t vals[8];
         uint32_t nibs = 0;
 #pragma unroll
         for (int gi = 0; gi < 8; ++gi) {
             int i0, i1;
             top2_of4(f + 4 * gi, i0, i1);
-            const uint32_t q =
-                quantize_pair<kInt8>(pick4(f + 4 * gi, i0), pick4(f + 4 * gi, i1), inv);
-            if (gi & 1)
-                vals[gi >> 1] |= q << 16;
-            else
-                vals[gi >> 1] = q;
+            if constexpr (kBf16) {
+                vals[gi] = bf16_bits(pick4(f + 4 * gi, i0)) |
+                           (bf16_bits(pick4(f + 4 * gi, i1)) << 16);
+            } else {
+                const uint32_t q =
+                    quantize_pair<kInt8>(pick4(f + 4 * gi, i0), pick4(f + 4 * gi, i1), inv);
+                if (gi & 1)
+                    vals[gi >> 1] |= q << 16;
+                else
+                    vals[gi >> 1] = q;
+            }
             nibs |= static_cast<uint32_t>(i0 | (i1 << 2)) << (4 * gi);
         }
-        __stcs(vout + st, make_uint4(vals[0], vals[1], vals[2], vals[3]));
-        __stcs(reinterpret_cast<uint32_t*>(Xm + meta_offset(m, 4 * st, K_lp64)), nibs);
+#pragma unroll
+        for (int v = 0; v < kVq; ++v)
+            __stcs(vout + kVq * st + v,
+                   make_uint4(vals[4 * v], vals[4 * v + 1], vals[4 * v + 2], vals[4 * v + 3]));
+        put_meta(st, nibs);
     }
 }
 
@@ -499,5 +535,83 @@ __global__ void __launch_bounds__(kWarpRowThreads) quant_lift_reg_kernel(
     }
 }
 
+
+}  // namespace ss
+
+namespace ss {
+
+// ---------------------------------------------------------------------------
+// Activation lift of the bf16 tier: the same window map as the 8-bit tiers
+// (SlideSparse write-up, omica.com.cn, 3.2: window i of group g reads the
+// four activations at 2Nh g + 2(i % (Nh-1))), no quantisation, bf16 out.
+// Window j of a group is the word pair (u_j, u_{j+1}) of the group's Nh
+// 32-bit words of bf16 pairs, so a group of 2Nh inputs becomes 2(Nh-1)
+// output words.  Dense and 2:4 are the identity (zero padded to K_lp).
+//
+// One thread per unit, grid-strided over rows: a unit is a group (sliding
+// patterns) or 8 outputs (identity); the zero tail [K_lift, K_lp) goes in
+// units of 4 outputs.
+// ---------------------------------------------------------------------------
+constexpr int kLiftThreads = 256;
+
+template <typename T>
+__device__ __forceinline__ uint32_t bf16_pair_at(const T* __restrict__ x, int64_t k, int64_t K) {
+    const uint32_t lo = k < K ? bf16_bits(to_f32<T>(x[k])) : 0u;
+    const uint32_t hi = k + 1 < K ? bf16_bits(to_f32<T>(x[k + 1])) : 0u;
+    return lo | (hi << 16);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kLiftThreads) lift_bf16_kernel(
+    const T* __restrict__ X, int64_t M, int64_t K, int Nh, int64_t K_lift, int64_t K_lp,
+    uint16_t* __restrict__ Xl) {
+    const int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    // bf16 words can be read straight from X when every pair is whole
+    constexpr bool kRaw = sizeof(T) == 2;
+    const bool raw_ok = kRaw && (K % 2 == 0);
+    if (Nh <= 2) {
+        if (u >= K_lp / 8) return;
+        const int64_t k0 = u * 8;
+        for (int64_t m = blockIdx.y; m < M; m += gridDim.y) {
+            const T* x = X + m * K;
+            uint4 v;
+            if (kRaw && K % 8 == 0 && k0 + 8 <= K) {
+                v = __ldg(reinterpret_cast<const uint4*>(x + k0));
+            } else {
+                v = make_uint4(bf16_pair_at<T>(x, k0, K), bf16_pair_at<T>(x, k0 + 2, K),
+                               bf16_pair_at<T>(x, k0 + 4, K), bf16_pair_at<T>(x, k0 + 6, K));
+            }
+            __stcs(reinterpret_cast<uint4*>(Xl + m * K_lp + k0), v);
+        }
+        return;
+    }
+    const int64_t G = K_lift / (4 * (Nh - 1));
+    const int64_t tail_units = (K_lp - K_lift) / 4;
+    if (u >= G + tail_units) return;
+    for (int64_t m = blockIdx.y; m < M; m += gridDim.y) {
+        uint16_t* out_row = Xl + m * K_lp;
+        if (u >= G) {  // zero tail, 4 outputs (8 bytes) per unit
+            __stcs(reinterpret_cast<uint2*>(out_row + K_lift + 4 * (u - G)), make_uint2(0u, 0u));
+            continue;
+        }
+        const T* x = X + m * K;
+        const int64_t k0 = u * 2 * Nh;
+        uint32_t w[5];
+        if (raw_ok && k0 + 2 * Nh <= K) {
+            const uint32_t* xw = reinterpret_cast<const uint32_t*>(x + k0);
+#pragma unroll
+            for (int i = 0; i < 5; ++i)
+                if (i < Nh) w[i] = __ldg(xw + i);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 5; ++i)
+                if (i < Nh) w[i] = bf16_pair_at<T>(x, k0 + 2 * i, K);
+        }
+        uint2* o = reinterpret_cast<uint2*>(out_row + u * 4 * (Nh - 1));
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (j < Nh - 1) __stcs(o + j, make_uint2(w[j], w[j + 1]));
+    }
+}
 
 }  // namespace ss

@@ -4,8 +4,14 @@ import torch
 
 import oracle
 
-Q = {"int8": oracle.INT8, "fp8": oracle.FP8_E4M3}
+Q = {"int8": oracle.INT8, "fp8": oracle.FP8_E4M3, "bf16": oracle.BF16}
 FP8_TOL = 1e-2
+# bf16 tier: exact products, fp32 accumulation in the tensor core's order
+# against the oracle's double sum rounded once.  Reordering the sum of K
+# products changes it by at most about K * 2^-24 * sum|x w| (2^-10 of the
+# largest |y| at K = 16384 for Gaussian data), and bf16 output can then move
+# by one unit in the last place (2^-8 relative): 1e-2 covers both.
+BF16_TOL = 1e-2
 
 
 def dev(a) -> torch.Tensor:
@@ -39,5 +45,6 @@ def assert_y_matches(y_gpu: np.ndarray, y_ref: np.ndarray, q: str, out_bf16: boo
     if q == "int8":
         np.testing.assert_array_equal(y_gpu, y_ref)   # bit-exact
     else:
+        tol = BF16_TOL if q == "bf16" else FP8_TOL
         err = fp8_rel_error(y_to_float(y_gpu, out_bf16), y_to_float(y_ref, out_bf16))
-        assert err <= FP8_TOL, f"fp8 relative error {err:.3e} > {FP8_TOL}"
+        assert err <= tol, f"{q} relative error {err:.3e} > {tol}"

@@ -88,6 +88,27 @@ def test_argument_errors_return_before_any_launch(L):
         == ss.SS_ERR_INVALID_ARG
     assert L.ss_sparse_gemm(0, odd, good, good, good, good, 16, 64, 128, 0, good, 1, None) \
         == ss.SS_ERR_ALIGNMENT
+    assert L.ss_sparse_gemm(0, good, good, good, good, good, 16, 64, 128, 3, good, 1, None) \
+        == ss.SS_ERR_INVALID_ARG
+    # scales are required by the 8-bit tiers and unused (NULL allowed) by bf16
+    assert L.ss_sparse_gemm(0, good, good, None, good, good, 16, 64, 128, 1, good, 1, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_sparse_gemm(0, good, good, None, good, None, 16, 64, 128, ss.SS_BF16, odd, 1,
+                            None) == ss.SS_ERR_ALIGNMENT
+    assert L.ss_dense_gemm(good, None, good, None, 16, 64, 128, 0, good, 1, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_dense_gemm(good, None, odd, None, 16, 64, 128, ss.SS_BF16, good, 1, None) \
+        == ss.SS_ERR_ALIGNMENT
+    assert L.ss_quant_lift_act(good, 1, 16, 64, pat, 0, good, None, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_quant_lift_act(odd, 1, 16, 64, pat, ss.SS_BF16, good, None, None) \
+        == ss.SS_ERR_ALIGNMENT
+    assert L.ss_prune_act_2to4(good, 1, 16, 64, ss.SS_BF16, good, odd, None, None) \
+        == ss.SS_ERR_ALIGNMENT
+    assert L.ss_compress_weight(good, 1, 64, 64, pat, 0, good, good, None, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_compress_weight(odd, 1, 64, 64, pat, ss.SS_BF16, good, good, None, None) \
+        == ss.SS_ERR_ALIGNMENT
     assert L.ss_dense_gemm(good, good, good, good, 16, 64, 96, 0, good, 1, None) \
         == ss.SS_ERR_INVALID_ARG
     assert L.ss_dense_gemm(good, good, odd, good, 16, 64, 128, 0, good, 1, None) \
@@ -125,6 +146,32 @@ def test_metadata_storage_layout(L, rows, K_lp):
     mask[off.reshape(-1)] = False
     assert not flat[mask].any()                          # padding rows
     np.testing.assert_array_equal(oracle.meta_from_tiles(At, rows, K_lp), Am)
+
+
+@pytest.mark.parametrize("rows,K_lp", [(16, 128), (130, 256), (300, 384)])
+def test_metadata_storage_layout_bf16(rows, K_lp):
+    """The bf16 tier's storage: the tile-major offset of ss.h taken at row
+    (r & ~8) | (b & 2) << 2 and byte (b & ~2) | (r & 8) >> 2 -- rows r and
+    r + 8 exchange the 2-byte halves of each 4-byte word."""
+    rng = np.random.default_rng(rows * K_lp)
+    Am = rng.integers(0, 256, (rows, K_lp // 8), dtype=np.uint8)
+    At = oracle.meta_to_tiles(Am, K_lp, i16=True)
+    assert At.shape == ss.meta_shape(rows, K_lp)
+    flat = At.reshape(-1)
+    r, b = np.meshgrid(np.arange(rows), np.arange(K_lp // 8), indexing="ij")
+    r2 = (r & ~8) | ((b & 2) << 2)
+    b2 = (b & ~2) | ((r & 8) >> 2)
+    off = ((r2 // 128) * (K_lp // 128) + b2 // 16) * 2048 + (r2 % 128) * 16 + b2 % 16
+    np.testing.assert_array_equal(flat[off], Am)
+    mask = np.ones(flat.size, dtype=bool)
+    mask[off.reshape(-1)] = False
+    assert not flat[mask].any()
+    np.testing.assert_array_equal(oracle.meta_from_tiles(At, rows, K_lp, i16=True), Am)
+    # rows 0..7 keep the first half of each word and hold row r + 8's first half second
+    if rows >= 16:
+        np.testing.assert_array_equal(At[0, 0, 3, 0:2], Am[3, 0:2])
+        np.testing.assert_array_equal(At[0, 0, 3, 2:4], Am[11, 0:2])
+        np.testing.assert_array_equal(At[0, 0, 11, 0:2], Am[3, 2:4])
 
 
 def test_meta_bytes_rejects_bad_shapes(L):
