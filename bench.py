@@ -7,7 +7,10 @@ resident in HBM:
                             -> ss_sparse_gemm (sparse tensor cores + dequant)
   online-activation workload: ss_prune_act_2to4 -> ss_sparse_gemm (sparse X)
 The dense comparator (ss_quant_lift_act dense -> ss_dense_gemm, same
-construction) is timed in the same run on the same inputs.
+construction) is timed in the same run on the same inputs.  For the bf16
+tier (--qdtype bf16 or a *_bf16 workload) the step is the lift and the
+kind::f16 sparse GEMM, and the dense FP8 path is timed as well: the pages'
+"2x tier" compares 2:4 + 16-bit against dense 8-bit.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--m M]
     python bench.py --impl reference ...   # the CPU oracle, timed on the host
@@ -217,16 +220,17 @@ class Path:
         this workload, on the current stream: X_rows in, Y rows r0..r1 out."""
         ss = self.ss
         m = r1 - r0
+        rows = lambda t: None if t is None else t[r0:r1]  # bf16 tier: no scales
         if self.online:
             Xv, Xm, s_x = self.act
-            part = (Xv[r0:r1], Xm[r0 // 128:r1 // 128], s_x[r0:r1])
+            part = (Xv[r0:r1], Xm[r0 // 128:r1 // 128], rows(s_x))
             ss.prune_act_2to4(X_rows, self.q, out=part)
             Wq, _, s_w = self.dense_w
             ss.sparse_gemm(1, part[0], part[1], part[2], Wq, s_w, m, self.N, self.q,
                            out=self.Y[r0:r1])
         else:
             Xq, s_x = self.act
-            part = (Xq[r0:r1], s_x[r0:r1])
+            part = (Xq[r0:r1], rows(s_x))
             ss.quant_lift_act(X_rows, self.pat, self.q, out=part)
             Wv, Wm, s_w = self.sparse_w
             ss.sparse_gemm(0, Wv, Wm, s_w, part[0], part[1], m, self.N, self.q,
@@ -257,12 +261,47 @@ class Path:
 
     def act_kernel_bytes(self):
         esz = self.X.element_size()
+        vb, sb = (2, 0) if self.q == "bf16" else (1, 4)   # value bytes, scale bytes
         if self.online:
-            return self.M * (esz * self.K + self.K_lp // 2 + self.K_lp // 8 + 4)
-        return self.M * (esz * self.K + self.K_lp + 4)
+            return self.M * (esz * self.K + vb * self.K_lp // 2 + self.K_lp // 8 + sb)
+        return self.M * (esz * self.K + vb * self.K_lp + sb)
 
     def dense_act_bytes(self):
-        return self.M * (self.X.element_size() * self.K + self.dense_act[0].shape[1] + 4)
+        vb, sb = (2, 0) if self.q == "bf16" else (1, 4)
+        return self.M * (self.X.element_size() * self.K + vb * self.dense_act[0].shape[1] + sb)
+
+    # peaks: dense bf16 measured; 8-bit dense = 2x, 2:4 sparse = 2x dense
+    def dense_peak(self, bf16_peak: float) -> float:
+        return bf16_peak * (1.0 if self.q == "bf16" else 2.0)
+
+    def sparse_peak(self, bf16_peak: float) -> float:
+        return 2.0 * self.dense_peak(bf16_peak)
+
+
+class DenseFp8:
+    """Dense FP8 comparator of a bf16-tier workload (per-token quant + dense
+    E4M3 GEMM, the like-for-like 8-bit path) on the same W and X."""
+
+    def __init__(self, path: "Path"):
+        ss = path.ss
+        self.ss, self.path = ss, path
+        W = synth.make_weight(path.N, path.K, path.w["w_std"], path.w["in_dtype"]).to(path.X.device)
+        self.w = ss.compress_weight(W, "dense", "fp8")
+        self.act = ss.quant_lift_act(path.X, "dense", "fp8")
+        del W
+
+    def step(self, ev=None):
+        ss, p = self.ss, self.path
+        if ev:
+            ev[0].record()
+        ss.quant_lift_act(p.X, "dense", "fp8", out=self.act)
+        if ev:
+            ev[1].record()
+        Xq, s_x = self.act
+        Wq, _, s_w = self.w
+        ss.dense_gemm(Xq, s_x, Wq, s_w, "fp8", out=p.Y)
+        if ev:
+            ev[2].record()
 
 
 def flush_l2(buf):
@@ -315,15 +354,20 @@ def measure(path: Path, steps: int, warmup: int, dist: Dist, peaks: dict):
         "t_dense_act_ms": mean(dn_act), "t_dense_gemm_ms": mean(dn_gemm),
         "launches": launches, "clocks": clk.summary(),
     }
-    bf16 = peaks["bf16_tflops"]
-    sparse_peak = bf16 * 4.0   # 8-bit dense = 2x bf16, 2:4 sparse = 2x dense (nominal ratios)
-    dense_peak = bf16 * 2.0
+    sparse_peak = path.sparse_peak(peaks["bf16_tflops"])
+    dense_peak = path.dense_peak(peaks["bf16_tflops"])
     r["sparse_gemm_tflops"] = path.sparse_gemm_ops() / (r["t_gemm_ms"] * 1e-3) / 1e12
     r["dense_gemm_tflops"] = path.dense_gemm_ops() / (r["t_dense_gemm_ms"] * 1e-3) / 1e12
     r["sparse_peak"] = sparse_peak
     r["dense_peak"] = dense_peak
     r["act_gbs"] = path.act_kernel_bytes() / (r["t_act_ms"] * 1e-3) / 1e9
     r["dense_act_gbs"] = path.dense_act_bytes() / (r["t_dense_act_ms"] * 1e-3) / 1e9
+    if path.q == "bf16":
+        f8 = DenseFp8(path)
+        f8_total, _, f8_gemm = time_loop(f8.step, steps, warmup, flush)
+        r["t_fp8_step_ms"] = dist.max(mean(f8_total))
+        r["t_fp8_gemm_ms"] = mean(f8_gemm)
+        del f8
     return r
 
 
@@ -385,20 +429,27 @@ def oracle_sample(name: str, M: int, budget_s: float):
     import oracle
     w = synth.WORKLOADS[name]
     N, K = w["N"], w["K"]
-    q = oracle.INT8 if w["qdtype"] == "int8" else oracle.FP8_E4M3
+    bf16 = w["qdtype"] == "bf16"
+    q = {"int8": oracle.INT8, "fp8": oracle.FP8_E4M3, "bf16": oracle.BF16}[w["qdtype"]]
     out = oracle.OUT_F32 if w["out"] == "f32" else oracle.OUT_BF16
     W = synth.make_weight(N, K, w["w_std"], w["in_dtype"])
     online = name.startswith("online")
-    if online:
-        packed = oracle.compress_weight(W, "dense", q)
-    else:
-        packed = oracle.compress_weight(W, w["pattern"], q)
+    pat = "dense" if online else w["pattern"]
+    packed = oracle.compress_weight_bf16(W, pat) if bf16 else oracle.compress_weight(W, pat, q)
     X = synth.make_activation(M, K, w["x_kind"], w["in_dtype"])
 
     def run(rows):
         Xs = X[rows]
         t0 = time.perf_counter()
-        if online:
+        if bf16 and online:
+            Xv, Xm = oracle.prune_act_2to4_bf16(Xs)
+            Wb, _ = packed
+            oracle.sparse_gemm_bf16(1, Xv, Xm, Wb, len(rows), N, Wb.shape[1], out)
+        elif bf16:
+            Wv, Wm = packed
+            Xl = oracle.lift_act_bf16(Xs, pat)
+            oracle.sparse_gemm_bf16(0, Wv, Wm, Xl, len(rows), N, Xl.shape[1], out)
+        elif online:
             Xv, Xm, s_x = oracle.prune_act_2to4(Xs, q)
             Wq, _, s_w = packed
             oracle.sparse_gemm(1, Xv, Xm, s_x, Wq, s_w, len(rows), N, Wq.shape[1], q, out)
@@ -470,7 +521,7 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=6.0)
     ap.add_argument("--pattern", default=None, choices=["2:4", "4:6", "6:8", "8:10"],
                     help="override the workload's pattern (the Llama-layer sweep)")
-    ap.add_argument("--qdtype", default=None, choices=["int8", "fp8"],
+    ap.add_argument("--qdtype", default=None, choices=["int8", "fp8", "bf16"],
                     help="override the workload's quantised type")
     args = ap.parse_args()
     if args.pattern or args.qdtype:
@@ -514,13 +565,20 @@ def main():
         "roofline": {"bound": "tensor", "kernel": "sparse_gemm",
                      "achieved": r["sparse_gemm_tflops"], "peak": r["sparse_peak"],
                      "unit": "TFLOP/s", "frac": r["sparse_gemm_tflops"] / r["sparse_peak"],
-                     "peak_source": f"{peaks['source']} bf16 burst x4 (8-bit x2, 2:4 x2)",
+                     "peak_source": f"{peaks['source']} bf16 burst x"
+                                    f"{r['sparse_peak'] / peaks['bf16_tflops']:.0f}"
+                                    + (" (2:4 x2)" if path.q == "bf16" else " (8-bit x2, 2:4 x2)"),
                      "traffic": tr},
         "e2e": {"value": n * path.dense_equiv_ops() / (t_e2e * 1e-3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
     })
+    if path.q == "bf16":  # the 2x tier: 2:4 + bf16 against dense FP8
+        line["vs_dense_fp8"] = {"speedup": r["t_fp8_step_ms"] / r["t_step_ms"],
+                                "gemm_speedup": r["t_fp8_gemm_ms"] / r["t_gemm_ms"],
+                                "fp8_step_us": r["t_fp8_step_ms"] * 1e3,
+                                "fp8_gemm_us": r["t_fp8_gemm_ms"] * 1e3}
     if not args.no_also and dist.world == 1 and args.workload != ALSO_WORKLOAD[0]:
         del path
         torch.cuda.empty_cache()

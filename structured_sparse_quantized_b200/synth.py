@@ -70,6 +70,10 @@ WORKLOADS = {
                                  in_dtype="bf16", w_std=0.02, out="bf16", x_kind="gauss"),
     "online_x_2of4_fp8": dict(M=8192, K=4096, N=14336, pattern="2:4", qdtype="fp8",
                               in_dtype="bf16", w_std=0.02, out="bf16", x_kind="heavy"),
+    # the 16-bit tier of the precision-tier study: 2:4 + bf16 on the
+    # Llama-3.1-8B q_proj shape (compared with dense bf16 and dense FP8)
+    "llama_q_2of4_bf16": dict(M=8192, K=4096, N=4096, pattern="2:4", qdtype="bf16",
+                              in_dtype="bf16", w_std=0.02, out="bf16", x_kind="outlier"),
 }
 
 # Llama-3.1-8B layer projections (N, K) for the pattern sweep.
