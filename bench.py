@@ -200,14 +200,14 @@ class Path:
             ev[0].record()
         if self.online:
             ss.prune_act_2to4(X, self.q, out=self.act)
-            if ev:
+            if ev and ev[1] is not None:
                 ev[1].record()
             Xv, Xm, s_x = self.act
             Wq, _, s_w = self.dense_w
             ss.sparse_gemm(1, Xv, Xm, s_x, Wq, s_w, self.M, self.N, self.q, out=self.Y)
         else:
             ss.quant_lift_act(X, self.pat, self.q, out=self.act)
-            if ev:
+            if ev and ev[1] is not None:
                 ev[1].record()
             Wv, Wm, s_w = self.sparse_w
             Xq, s_x = self.act
@@ -241,7 +241,7 @@ class Path:
         if ev:
             ev[0].record()
         ss.quant_lift_act(self.X, "dense", self.q, out=self.dense_act)
-        if ev:
+        if ev and ev[1] is not None:
             ev[1].record()
         Xq, s_x = self.dense_act
         Wq, _, s_w = self.dense_w
@@ -295,7 +295,7 @@ class DenseFp8:
         if ev:
             ev[0].record()
         ss.quant_lift_act(p.X, "dense", "fp8", out=self.act)
-        if ev:
+        if ev and ev[1] is not None:
             ev[1].record()
         Xq, s_x = self.act
         Wq, _, s_w = self.w
@@ -312,19 +312,27 @@ def flush_l2(buf):
     return buf.sum(dtype=torch.int64)
 
 
-def time_loop(fn, steps, warmup, flush):
+def time_loop(fn, steps, warmup, flush, split=True):
     """Per-step CUDA-event times (ms) of fn(ev) with an L2 flush before each
-    step, outside the events."""
+    step, outside the events.  With split, an event between the activation
+    kernel and the GEMM also times each part; without it the step has only
+    its start and end events, so nothing on the stream separates the two
+    kernels and the GEMM may start early (programmatic dependent launch)."""
     for _ in range(warmup):
         flush_l2(flush)
         fn(None)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    if not split:
+        for e in evs:
+            e[1] = None
     torch.cuda.synchronize()
     for i in range(steps):
         flush_l2(flush)
         fn(evs[i])
     torch.cuda.synchronize()
     total = [e[0].elapsed_time(e[2]) for e in evs]
+    if not split:
+        return total, None, None
     first = [e[0].elapsed_time(e[1]) for e in evs]
     second = [e[1].elapsed_time(e[2]) for e in evs]
     return total, first, second
@@ -337,9 +345,12 @@ def measure(path: Path, steps: int, warmup: int, dist: Dist, peaks: dict):
     torch.cuda.synchronize()
     launches0 = ss.ss_kernel_launches()
     with ClockSampler(torch.cuda.current_device()) as clk:
-        sp_total, sp_act, sp_gemm = time_loop(path.sparse_step, steps, warmup, flush)
+        sp_total, _, _ = time_loop(path.sparse_step, steps, warmup, flush, split=False)
     launches = ss.ss_kernel_launches() - launches0 - 2 * warmup
-    dn_total, dn_act, dn_gemm = time_loop(path.dense_step, steps, warmup, flush)
+    dn_total, _, _ = time_loop(path.dense_step, steps, warmup, flush, split=False)
+    # the per-kernel split (an event between the two kernels) in separate runs
+    _, sp_act, sp_gemm = time_loop(path.sparse_step, steps, warmup, flush)
+    _, dn_act, dn_gemm = time_loop(path.dense_step, steps, warmup, flush)
     torch.cuda.synchronize()
     dist.barrier()
     status = ss.ss_get_device_status()
@@ -364,7 +375,8 @@ def measure(path: Path, steps: int, warmup: int, dist: Dist, peaks: dict):
     r["dense_act_gbs"] = path.dense_act_bytes() / (r["t_dense_act_ms"] * 1e-3) / 1e9
     if path.q == "bf16":
         f8 = DenseFp8(path)
-        f8_total, _, f8_gemm = time_loop(f8.step, steps, warmup, flush)
+        f8_total, _, _ = time_loop(f8.step, steps, warmup, flush, split=False)
+        _, _, f8_gemm = time_loop(f8.step, steps, warmup, flush)
         r["t_fp8_step_ms"] = dist.max(mean(f8_total))
         r["t_fp8_gemm_ms"] = mean(f8_gemm)
         del f8

@@ -56,6 +56,50 @@ ss_status launched() {
     return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 
+// Programmatic dependent launch for every kernel (SS_PDL=0 turns it off).
+// Each kernel takes griddepcontrol.wait before touching memory that earlier
+// work on the stream may write, so results do not depend on this switch.
+bool pdl_enabled() {
+    static const bool on = [] {
+        const char* v = std::getenv("SS_PDL");
+        return !(v && std::strcmp(v, "0") == 0);
+    }();
+    return on;
+}
+
+// Launch `kern` on `stream` with programmatic stream serialisation allowed
+// and, for cluster > 1, that cluster size.
+template <typename... KArgs, typename... Args>
+ss_status launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                    cudaStream_t stream, int cluster, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    if (cluster > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = static_cast<unsigned>(cluster);
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    if (pdl_enabled()) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) {
+        cudaGetLastError();
+        return SS_ERR_CUDA;
+    }
+    return launched();
+}
+
 bool valid_pattern(ss_pattern p) {
     if (p.keep == 0 && p.group == 0) return true;
     return (p.group == 4 || p.group == 6 || p.group == 8 || p.group == 10) &&
@@ -130,23 +174,8 @@ ss_status launch_gemm(int dev, const CUtensorMap& a, const CUtensorMap& b, const
         ((args.rowsA + tile_rows - 1) / tile_rows) * ((args.rowsB + args.bn - 1) / args.bn);
     const int64_t units = g_num_sms[dev] / kPair;
     const int grid = static_cast<int>((tiles < units ? tiles : units) * kPair);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid, 1, 1);
-    cfg.blockDim = dim3(ss::kGemmThreads, 1, 1);
-    cfg.dynamicSmemBytes = C::kSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kPair;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, a, b, e, y, args) != cudaSuccess) {
-        cudaGetLastError();
-        return SS_ERR_CUDA;
-    }
-    return launched();
+    return launch_ex(kern, dim3(grid), dim3(ss::kGemmThreads), C::kSmemBytes, stream, kPair, a, b,
+                     e, y, args);
 }
 
 // q: ss::kQE4M3, kQInt8 or kQBf16; bf16: Y element type.
@@ -193,23 +222,8 @@ ss_status launch_gemm_wide(int dev, const CUtensorMap& a, const CUtensorMap& b,
                           ((args.rowsB + tile_b - 1) / tile_b);
     const int64_t units = g_num_sms[dev] / 2;
     const int grid = static_cast<int>((tiles < units ? tiles : units) * 2);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid, 1, 1);
-    cfg.blockDim = dim3(ss::kWideThreads, 1, 1);
-    cfg.dynamicSmemBytes = C::kSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, a, b, e, y, args) != cudaSuccess) {
-        cudaGetLastError();
-        return SS_ERR_CUDA;
-    }
-    return launched();
+    return launch_ex(kern, dim3(grid), dim3(ss::kWideThreads), C::kSmemBytes, stream, 2, a, b, e,
+                     y, args);
 }
 
 // B-tile width of the wide sparse GEMM: the multiple of 32 (<= 224) whose
@@ -377,8 +391,9 @@ ss_status ss_compress_weight(const void* W, ss_in_dtype in_dtype, int64_t N, int
     do {                                                                                      \
         auto kern = ss::compress_weight_kernel<T, Q>;                                         \
         if ((st = set_smem(kern, dev, smem)) != SS_OK) return st;                             \
-        kern<<<static_cast<unsigned>(rows_grid), ss::kCompressThreads, smem, s>>>(            \
-            static_cast<const T*>(W), N, K, p.keep, p.group, K_lift, K_lp, wv, wm, s_w);      \
+        st = launch_ex(kern, dim3(static_cast<unsigned>(rows_grid)), dim3(ss::kCompressThreads), \
+                       smem, s, 1, static_cast<const T*>(W), N, K, p.keep, p.group, K_lift,   \
+                       K_lp, wv, wm, s_w);                                                    \
     } while (0)
     if (in_dtype == SS_IN_BF16) {
         if (kq == ss::kQInt8) SS_COMPRESS(__nv_bfloat16, ss::kQInt8);
@@ -390,7 +405,7 @@ ss_status ss_compress_weight(const void* W, ss_in_dtype in_dtype, int64_t N, int
         else SS_COMPRESS(float, ss::kQE4M3);
     }
 #undef SS_COMPRESS
-    return launched();
+    return st;
 }
 
 ss_status ss_quant_lift_act(const void* X, ss_in_dtype in_dtype, int64_t M, int64_t K,
@@ -417,12 +432,11 @@ ss_status ss_quant_lift_act(const void* X, ss_in_dtype in_dtype, int64_t M, int6
                         static_cast<unsigned>(M < 65535 ? M : 65535));
         uint16_t* xl = static_cast<uint16_t*>(Xq_lift);
         if (in_dtype == SS_IN_BF16)
-            ss::lift_bf16_kernel<__nv_bfloat16><<<grid, ss::kLiftThreads, 0, s>>>(
-                static_cast<const __nv_bfloat16*>(X), M, K, Nh, K_lift, K_lp, xl);
-        else
-            ss::lift_bf16_kernel<float><<<grid, ss::kLiftThreads, 0, s>>>(
-                static_cast<const float*>(X), M, K, Nh, K_lift, K_lp, xl);
-        return launched();
+            return launch_ex(ss::lift_bf16_kernel<__nv_bfloat16>, grid, dim3(ss::kLiftThreads), 0,
+                             s, 1, static_cast<const __nv_bfloat16*>(X), M, K, Nh, K_lift, K_lp,
+                             xl);
+        return launch_ex(ss::lift_bf16_kernel<float>, grid, dim3(ss::kLiftThreads), 0, s, 1,
+                         static_cast<const float*>(X), M, K, Nh, K_lift, K_lp, xl);
     }
     // one warp per token row; sliding patterns keep a quantised byte row per
     // warp in shared memory
@@ -443,8 +457,8 @@ ss_status ss_quant_lift_act(const void* X, ss_in_dtype in_dtype, int64_t M, int6
     do {                                                                                      \
         auto kern = ss::quant_lift_warp_kernel<T, I8>;                                        \
         if ((st = set_smem(kern, dev, smem)) != SS_OK) return st;                             \
-        kern<<<grid, warps * 32, smem, s>>>(static_cast<const T*>(X), M, K, Nh, K_lift, K_lp,  \
-                                            q_stride, xq, s_x);                               \
+        st = launch_ex(kern, dim3(grid), dim3(warps * 32), smem, s, 1,                        \
+                       static_cast<const T*>(X), M, K, Nh, K_lift, K_lp, q_stride, xq, s_x);  \
     } while (0)
     // bf16 rows of up to 4096 elements (K % 16 == 0) are read once, into registers
     const bool reg_path = in_dtype == SS_IN_BF16 && K % 16 == 0 && K <= ss::kRegK;
@@ -462,8 +476,8 @@ ss_status ss_quant_lift_act(const void* X, ss_in_dtype in_dtype, int64_t M, int6
     do {                                                                                      \
         auto kern = ss::quant_lift_reg_kernel<I8, C, W>;                                      \
         if ((st = set_smem(kern, dev, rsmem)) != SS_OK) return st;                            \
-        kern<<<rgrid, ss::kWarpRowThreads, rsmem, s>>>(xb, M, K, Nh, K_lift, K_lp, q_stride,  \
-                                                       xq, s_x);                              \
+        st = launch_ex(kern, dim3(rgrid), dim3(ss::kWarpRowThreads), rsmem, s, 1, xb, M, K,   \
+                       Nh, K_lift, K_lp, q_stride, xq, s_x);                                 \
     } while (0)
 #define SS_QREG_C(I8)                                                                          \
     do {                                                                                      \
@@ -495,7 +509,7 @@ ss_status ss_quant_lift_act(const void* X, ss_in_dtype in_dtype, int64_t M, int6
         else SS_QLIFT(float, false);
     }
 #undef SS_QLIFT
-    return launched();
+    return st;
 }
 
 ss_status ss_prune_act_2to4(const void* X, ss_in_dtype in_dtype, int64_t M, int64_t K,
@@ -521,8 +535,8 @@ ss_status ss_prune_act_2to4(const void* X, ss_in_dtype in_dtype, int64_t M, int6
     const unsigned grid = static_cast<unsigned>(((M + 127) / 128 * 128 + warps - 1) / warps);
 #define SS_PRUNE(T, Q)                                                                         \
     do {                                                                                      \
-        ss::prune_act_warp_kernel<T, Q><<<grid, ss::kWarpRowThreads, 0, s>>>(                \
-            static_cast<const T*>(X), M, K, K_lp, xv, xm, s_x);                               \
+        st = launch_ex(ss::prune_act_warp_kernel<T, Q>, dim3(grid), dim3(ss::kWarpRowThreads), \
+                       0, s, 1, static_cast<const T*>(X), M, K, K_lp, xv, xm, s_x);           \
     } while (0)
     if (in_dtype == SS_IN_BF16) {
         if (kq == ss::kQInt8) SS_PRUNE(__nv_bfloat16, ss::kQInt8);
@@ -534,7 +548,7 @@ ss_status ss_prune_act_2to4(const void* X, ss_in_dtype in_dtype, int64_t M, int6
         else SS_PRUNE(float, ss::kQE4M3);
     }
 #undef SS_PRUNE
-    return launched();
+    return st;
 }
 
 ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, const float* s_a,

@@ -120,10 +120,37 @@ __host__ __device__ __forceinline__ int64_t meta_offset_i16(int64_t r, int64_t b
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  Every kernel of this library is launched
+// with programmatic stream serialisation allowed: it may start while the
+// previous kernel on the stream is still running, and pdl_wait() -- taken by
+// every thread before its first access to memory that other work may write --
+// returns once that kernel has completed and its writes are visible.
+// pdl_trigger() lets the next kernel start early; it takes effect once every
+// CTA of this grid has issued it (or exited), i.e. when all of them are
+// already resident, so an early dependent cannot keep this grid from running.
+// Without the launch attribute both are no-ops.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // TMA (no multicast anywhere in this library).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Prefetch one box of a 2-D tensor map into L2 (no shared-memory write, no
+// barrier).  L2 is the point of coherence, so this is safe even before
+// pdl_wait(): a later load still sees any write made in between.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int32_t x, int32_t y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y)
+                 : "memory");
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,

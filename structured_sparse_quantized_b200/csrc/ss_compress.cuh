@@ -82,6 +82,8 @@ __global__ void __launch_bounds__(kCompressThreads) compress_weight_kernel(
     constexpr bool kInt8 = kQ == kQInt8;
     constexpr bool kBf16 = kQ == kQBf16;
     extern __shared__ __align__(16) uint8_t smem_raw[];
+    pdl_trigger();
+    pdl_wait();
     __shared__ float red[32];
     __shared__ int bad;
     const int64_t n = blockIdx.x;

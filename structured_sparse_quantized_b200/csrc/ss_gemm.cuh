@@ -45,6 +45,7 @@
 namespace ss {
 
 constexpr int kGemmThreads = 192;
+constexpr int kL2PrefetchStages = 16;  // weight stages a CTA prefetches before pdl_wait
 constexpr int kTileA = 128;  // A rows per CTA per A tile
 constexpr int kTmemCols = 512;
 
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(drain + 1);
     __shared__ int abort_flag_storage;
     volatile int* abort_flag = &abort_flag_storage;
+    pdl_trigger();
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -191,6 +193,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_base_slot;
+    // Until the previous kernel on the stream has finished, only the weight
+    // operand may be touched, and only through L2 prefetches (the producer's,
+    // below); every other access waits here.
+    if (warp != 0) pdl_wait();
 
     // The producer and MMA roles run as whole, converged warps: every lane
     // takes the barrier waits (the outcome is made warp-uniform) and one
@@ -203,8 +209,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tma_prefetch_desc(&tm_a);
             tma_prefetch_desc(&tm_b);
             if (kSparse) tma_prefetch_desc(&tm_e);
+            if (args.a_is_w && unit < n_tiles) {
+                // A (and its metadata) is the weight: start streaming the first
+                // tile's K stages into L2 while the previous kernel finishes.
+                const int a0 = (unit % nA) * tile_a_rows + static_cast<int>(rank) * kTileA;
+                const int n_pre = args.k_stages < kL2PrefetchStages ? args.k_stages
+                                                                    : kL2PrefetchStages;
+                for (int kb = 0; kb < n_pre; ++kb) {
+                    tma_prefetch_l2_2d(&tm_a, kb * C::kARowBytes, a0);
+#pragma unroll
+                    for (int u = 0; u < C::kEChunks; ++u)
+                        tma_prefetch_l2_2d(&tm_e, 0,
+                                           ((a0 >> 7) * args.e_chunks + kb * C::kEChunks + u) * 16);
+                }
+            }
         }
         __syncwarp();
+        pdl_wait();
         const uint32_t tx =
             kPair * (C::kABytes + C::kEBytes + C::kBAtoms * b_rows_cta * 128);
         int s = 0;

@@ -104,6 +104,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(drain + 1);
     __shared__ int abort_flag_storage;
     volatile int* abort_flag = &abort_flag_storage;
+    pdl_trigger();
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -137,6 +138,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     cluster_sync_all();  // peer barriers initialised before any remote use
     tc_fence_after();
     const uint32_t tmem_base = *tmem_base_slot;
+    // Every access to global memory waits for the previous kernel on the
+    // stream (programmatic dependent launch); only the producer's L2
+    // prefetches of the weight go first.
+    if (warp != 0) pdl_wait();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -144,8 +149,19 @@ __global__ void __launch_bounds__(kWideThreads, 1)
             tma_prefetch_desc(&tm_a);
             tma_prefetch_desc(&tm_b);
             tma_prefetch_desc(&tm_e);
+            const int t0 = snake_tile(0, unit, n_units);
+            if (kAIsW && t0 < n_tiles) {  // the weight's first tile into L2
+                const int a0 = (t0 % nA) * kPairRows + static_cast<int>(rank) * kTileA;
+                const int n_pre = args.k_stages < 2 * kL2PrefetchStages ? args.k_stages
+                                                                        : 2 * kL2PrefetchStages;
+                for (int kb = 0; kb < n_pre; ++kb) {
+                    tma_prefetch_l2_2d(&tm_a, kb * C::kARowBytes, a0);
+                    tma_prefetch_l2_2d(&tm_e, 0, ((a0 >> 7) * args.e_chunks + kb) * 16);
+                }
+            }
         }
         __syncwarp();
+        pdl_wait();
         const uint32_t tx = 2 * (C::kABytes + C::kEBytes + kWideBT * b_rows_cta * 128);
         int s = 0;
         uint32_t ph = 0, armed = 0, armed_par = 0;

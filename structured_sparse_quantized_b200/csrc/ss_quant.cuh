@@ -199,6 +199,8 @@ __global__ void __launch_bounds__(kWarpRowThreads) quant_lift_warp_kernel(
     int q_stride, uint8_t* __restrict__ Xq, float* __restrict__ s_x) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_trigger();
+    pdl_wait();
     const int64_t m = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
     if (m >= M) return;
     const int K = static_cast<int>(K64);
@@ -284,6 +286,8 @@ __global__ void __launch_bounds__(kWarpRowThreads) prune_act_warp_kernel(
     uint8_t* __restrict__ Xm, float* __restrict__ s_x) {
     constexpr bool kInt8 = kQ == kQInt8;
     constexpr bool kBf16 = kQ == kQBf16;
+    pdl_trigger();
+    pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t m = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
     const int64_t M_pad = (M + 127) / 128 * 128;
@@ -410,6 +414,8 @@ __global__ void __launch_bounds__(kWarpRowThreads) quant_lift_reg_kernel(
     const __nv_bfloat16* __restrict__ X, int64_t M, int64_t K64, int Nh, int64_t K_lift64,
     int64_t K_lp64, int q_stride, uint8_t* __restrict__ Xq, float* __restrict__ s_x) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
+    pdl_trigger();
+    pdl_wait();
     constexpr int kRowsPerCta = kWarpRowThreads / (32 * kWpr);
     __shared__ float part[kRowsPerCta][kWpr];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -565,6 +571,8 @@ template <typename T>
 __global__ void __launch_bounds__(kLiftThreads) lift_bf16_kernel(
     const T* __restrict__ X, int64_t M, int64_t K, int Nh, int64_t K_lift, int64_t K_lp,
     uint16_t* __restrict__ Xl) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     // bf16 words can be read straight from X when every pair is whole
     constexpr bool kRaw = sizeof(T) == 2;
