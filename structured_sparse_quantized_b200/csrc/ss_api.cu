@@ -16,6 +16,7 @@
 #include "ss_common.cuh"
 #include "ss_compress.cuh"
 #include "ss_gemm.cuh"
+#include "ss_gemm_splitk.cuh"
 #include "ss_gemm_wide.cuh"
 #include "ss_quant.cuh"
 
@@ -194,6 +195,100 @@ ss_status dispatch_gemm(int dev, int q, bool bf16, const CUtensorMap& a, const C
                 : launch_gemm<kSparse, kQE4M3, false, kPair>(dev, a, b, e, y, args, st);
 }
 
+// Split-K GEMM (decode sizes, A = weight): S K parts on the S CTAs of a
+// cluster.  Returns the number of clusters of S CTAs that can be resident at
+// once (0 if the kernel cannot run), cached per device.
+template <bool kSparse, int kQ, bool kOutBf16>
+int splitk_max_clusters(int dev, int S) {
+    using C = ss::SplitKCfg<kSparse, kQ == ss::kQBf16 ? 2 : 1>;
+    auto kern = ss::gemm_splitk_kernel<kSparse, kQ, kOutBf16>;
+    static std::once_flag once[kMaxDevices];
+    static int cached[kMaxDevices][4];  // S = 2, 4, 8
+    std::call_once(once[dev], [&] {
+        for (int i = 0; i < 4; ++i) cached[dev][i] = 0;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmemBytes) != cudaSuccess) {
+            cudaGetLastError();
+            return;
+        }
+        for (int i = 1; i < 4; ++i) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(1 << i);
+            cfg.blockDim = dim3(ss::kGemmThreads);
+            cfg.dynamicSmemBytes = C::kSmemBytes;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 1u << i;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+                cudaGetLastError();
+                n = 0;
+            }
+            cached[dev][i] = n;
+        }
+    });
+    return S == 2 ? cached[dev][1] : (S == 4 ? cached[dev][2] : (S == 8 ? cached[dev][3] : 0));
+}
+
+template <bool kSparse, int kQ, bool kOutBf16>
+ss_status launch_splitk(int S, int64_t tiles, const CUtensorMap& a, const CUtensorMap& b,
+                        const CUtensorMap& e, const ss::GemmArgs& args, cudaStream_t stream) {
+    using C = ss::SplitKCfg<kSparse, kQ == ss::kQBf16 ? 2 : 1>;
+    return launch_ex(ss::gemm_splitk_kernel<kSparse, kQ, kOutBf16>,
+                     dim3(static_cast<unsigned>(tiles * S)), dim3(ss::kGemmThreads), C::kSmemBytes,
+                     stream, S, a, b, e, args);
+}
+
+// The K split for a decode-sized problem (A = weight, every B row in one
+// tile of at most ss::kSkBn): the largest S in {8, 4, 2} whose tiles x S CTAs
+// are all resident at once, with at least one K stage per part, and which
+// keeps more SMs busy than the one-pass kernel's CTA pairs.  0: no split.
+template <bool kSparse, int kQ, bool kOutBf16>
+int choose_split(int dev, int64_t rowsA, int64_t rowsB, int k_stages) {
+    if (rowsB > ss::kSkBn) return 0;
+    const int64_t tiles = (rowsA + ss::kTileA - 1) / ss::kTileA;
+    const int64_t pair_ctas = rowsA > ss::kTileA ? (rowsA + 2 * ss::kTileA - 1) / (2 * ss::kTileA) * 2
+                                                 : 1;
+    for (int S = 8; S >= 2; S /= 2) {
+        if (S > k_stages || tiles * S > g_num_sms[dev] || tiles * S <= pair_ctas) continue;
+        if (tiles <= splitk_max_clusters<kSparse, kQ, kOutBf16>(dev, S)) return S;
+    }
+    return 0;
+}
+
+// Split-K dispatch on the operand type and Y type; returns SS_ERR_UNSUPPORTED
+// (nothing launched) when no split applies.
+template <bool kSparse>
+ss_status try_splitk(int dev, int q, bool bf16, int64_t rowsA, int64_t rowsB,
+                     const void* Av, int64_t a_cols, const void* B, int64_t b_cols,
+                     const CUtensorMap& e, const ss::GemmArgs& args, cudaStream_t stream) {
+    using namespace ss;
+    int S = 0;
+#define SS_SK_PICK(Q, BF) S = choose_split<kSparse, Q, BF>(dev, rowsA, rowsB, args.k_stages)
+    if (q == kQInt8) { if (bf16) SS_SK_PICK(kQInt8, true); else SS_SK_PICK(kQInt8, false); }
+    else if (q == kQBf16) { if (bf16) SS_SK_PICK(kQBf16, true); else SS_SK_PICK(kQBf16, false); }
+    else { if (bf16) SS_SK_PICK(kQE4M3, true); else SS_SK_PICK(kQE4M3, false); }
+#undef SS_SK_PICK
+    if (S == 0) return SS_ERR_UNSUPPORTED;
+    ss::GemmArgs a2 = args;
+    a2.bn = static_cast<int>(round_up(rowsB, 32));
+    CUtensorMap ta, tb;
+    if (!make_map_2d(&ta, Av, rowsA, a_cols, ss::kTileA, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tb, B, rowsB, b_cols, a2.bn, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+        return SS_ERR_CUDA;
+    const int64_t tiles = (rowsA + ss::kTileA - 1) / ss::kTileA;
+#define SS_SK_GO(Q, BF) return launch_splitk<kSparse, Q, BF>(S, tiles, ta, tb, e, a2, stream)
+    if (q == kQInt8) { if (bf16) SS_SK_GO(kQInt8, true); SS_SK_GO(kQInt8, false); }
+    if (q == kQBf16) { if (bf16) SS_SK_GO(kQBf16, true); SS_SK_GO(kQBf16, false); }
+    if (bf16) SS_SK_GO(kQE4M3, true);
+    SS_SK_GO(kQE4M3, false);
+#undef SS_SK_GO
+}
+
 // Operand type of the kernels for a public ss_qdtype (-1: not one).
 int kernel_q(ss_qdtype q) {
     switch (q) {
@@ -255,13 +350,15 @@ int choose_bn_wide(int64_t rowsA, int64_t rowsB, int units) {
     return best;
 }
 
-// SS_SPARSE_KERNEL=narrow|wide pins the sparse GEMM shape where both apply
-// (for tests and measurements); unset or anything else: chosen per problem.
+// SS_SPARSE_KERNEL=narrow|wide|splitk pins the GEMM shape where it applies
+// (for tests and measurements; "narrow" also keeps decode-sized problems off
+// the split-K kernel); unset or anything else: chosen per problem.
 int forced_sparse_kernel() {
     const char* v = std::getenv("SS_SPARSE_KERNEL");
     if (!v) return 0;
     if (std::strcmp(v, "narrow") == 0) return 1;
     if (std::strcmp(v, "wide") == 0) return 2;
+    if (std::strcmp(v, "splitk") == 0) return 3;
     return 0;
 }
 
@@ -600,11 +697,16 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
     if (!args.tma_store) ty = ta;  // unused
     cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
     const bool i8 = q == SS_INT8, bf = out_dtype == SS_OUT_BF16;
+    const int forced = forced_sparse_kernel();
+    if (args.a_is_w && forced != 1 && forced != 2) {  // decode sizes: split K over a cluster
+        const ss_status sk = try_splitk<true>(dev, kq, bf, rowsA, rowsB, Av, K_lp / 2 * eb, B,
+                                              K_lp * eb, te, args, st_);
+        if (sk != SS_ERR_UNSUPPORTED) return sk;
+    }
 #if SS_SPARSE_WIDE
     // (8-bit operands only: the bf16 tier runs the one-B-tile kernel)
     // Large problems with bf16 Y may take two B tiles per output tile: fewer
     // bytes per MMA, but single-buffered accumulators.
-    const int forced = forced_sparse_kernel();
     if (scaled && pair == 2 && args.tma_store && forced != 1 &&
         (forced == 2 || (rowsB > 2 * ss::WideCfg::kBnMax &&
                          prefer_wide(rowsA, rowsB, bn, g_num_sms[dev] / 2)))) {
@@ -658,6 +760,7 @@ ss_status ss_dense_gemm(const void* Xq, const float* s_x, const void* Wq, const 
     args.bn = bn;
     args.a_is_w = 1;
     args.ldy = static_cast<int>(N);
+    args.e_chunks = 0;
     args.s_a = s_w;
     args.s_b = s_x;
     args.y = Y;
@@ -666,6 +769,11 @@ ss_status ss_dense_gemm(const void* Xq, const float* s_x, const void* Wq, const 
     if (!args.tma_store) ty = ta;  // unused
     cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
     const bool bf = out_dtype == SS_OUT_BF16;
+    if (forced_sparse_kernel() != 1) {  // decode sizes: split K over a cluster
+        const ss_status sk =
+            try_splitk<false>(dev, kq, bf, N, M, Wq, K_p * eb, Xq, K_p * eb, ta, args, st_);
+        if (sk != SS_ERR_UNSUPPORTED) return sk;
+    }
     return pair == 2 ? dispatch_gemm<false, 2>(dev, kq, bf, ta, tb, ta, ty, args, st_)
                      : dispatch_gemm<false, 1>(dev, kq, bf, ta, tb, ta, ty, args, st_);
 }
