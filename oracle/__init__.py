@@ -23,6 +23,7 @@ from . import build as _build
 INT8 = 0
 FP8_E4M3 = 1
 BF16 = 2
+NVFP4 = 3
 OUT_F32 = 0
 OUT_BF16 = 1
 
@@ -54,6 +55,13 @@ def lib() -> ctypes.CDLL:
             "ssref_decompress_2to4_bf16": [p, p, i64, i64, p],
             "ssref_matmul_bf16": [p, p, i64, i64, i64, p, i64, i32, p],
             "ssref_sparse_gemm_bf16": [i32, p, p, p, i64, i64, i64, p, i64, i32, p],
+            "ssref_fp4_shape": [i32, i32, i64, p, p],
+            "ssref_prune_pairs": [p, i64, i64, i32, i32, p],
+            "ssref_compress_weight_nvfp4": [p, i64, i64, i32, i32, p, p, p, p],
+            "ssref_quant_nvfp4": [p, i64, i64, i32, i32, i32, i32, p, p, p],
+            "ssref_decode_sparse_nvfp4": [p, p, p, i64, i64, p],
+            "ssref_decode_dense_nvfp4": [p, p, i64, i64, i32, p],
+            "ssref_matmul_nvfp4": [p, p, p, p, i64, i64, i64, p, i64, i32, p],
         }
         for name, args in sig.items():
             fn = getattr(_lib, name)
@@ -67,6 +75,12 @@ def lib() -> ctypes.CDLL:
         _lib.ssref_bf16_from_float.restype = ctypes.c_uint16
         _lib.ssref_bits_per_element.argtypes = [i32, i32]
         _lib.ssref_bits_per_element.restype = ctypes.c_double
+        _lib.ssref_e2m1_from_float.argtypes = [ctypes.c_float]
+        _lib.ssref_e2m1_from_float.restype = ctypes.c_uint8
+        _lib.ssref_e2m1_to_double.argtypes = [ctypes.c_uint8]
+        _lib.ssref_e2m1_to_double.restype = ctypes.c_double
+        _lib.ssref_nvfp4_global.argtypes = [ctypes.c_float]
+        _lib.ssref_nvfp4_global.restype = ctypes.c_float
     return _lib
 
 
@@ -434,3 +448,120 @@ def prune_act_2to4_bf16(X):
     Xm).  With no scale, this is the 2:4 weight compression applied to the
     token rows: the same magnitude ranking, tie rule and packing."""
     return compress_weight_bf16(X, "2:4")
+
+
+
+# ---------------------------------------------------------------- NVFP4 (pairs)
+
+def e2m1_from_float(v: float) -> int:
+    return int(lib().ssref_e2m1_from_float(float(v)))
+
+
+def e2m1_to_float(c: int) -> float:
+    return float(lib().ssref_e2m1_to_double(int(c)))
+
+
+def nvfp4_global(amax: float) -> float:
+    return float(lib().ssref_nvfp4_global(float(amax)))
+
+
+def fp4_shape(p: str, K: int) -> tuple[int, int]:
+    """(K_lift, K_lp) in elements for pattern p counted in pairs."""
+    keep, group = pattern(p)
+    a, b = ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().ssref_fp4_shape(keep, group, K, ctypes.byref(a), ctypes.byref(b)), "fp4_shape")
+    return a.value, b.value
+
+
+def prune_pairs(W, keep: int, group: int) -> np.ndarray:
+    """Pair mask [rows, P_pad] (P = ceil(K/2) pairs)."""
+    W = _f32(W)
+    rows, K = W.shape
+    P = (K + 1) // 2
+    P_pad = -(-P // group) * group
+    mask = np.zeros((rows, P_pad), dtype=np.uint8)
+    _check(lib().ssref_prune_pairs(_ptr(W), rows, K, keep, group, _ptr(mask)), "prune_pairs")
+    return mask
+
+
+def compress_weight_nvfp4(W, p: str):
+    """-> (Wv [N, K_lp/4] bytes, Wm [N, K_lp/16], Ws [N, K_lp/32] UE4M3, g_w)."""
+    W = _f32(W)
+    N, K = W.shape
+    keep, group = pattern(p)
+    _, K_lp = fp4_shape(p, K)
+    Wv = np.zeros((N, K_lp // 4), dtype=np.uint8)
+    Wm = np.zeros((N, K_lp // 16), dtype=np.uint8)
+    Ws = np.zeros((N, K_lp // 32), dtype=np.uint8)
+    g = np.zeros(1, dtype=np.float32)
+    _check(lib().ssref_compress_weight_nvfp4(_ptr(W), N, K, keep, group, _ptr(Wv), _ptr(Wm),
+                                             _ptr(Ws), _ptr(g)), "compress_weight_nvfp4")
+    return Wv, Wm, Ws, float(g[0])
+
+
+def quant_nvfp4(X, p: str, block: int, per_row: bool = True):
+    """Dense NVFP4 rows (lifted on pairs for a pattern) -> (Xv [rows, K_lp/2]
+    bytes, Xs [rows, K_lp/block] UE4M3, g [rows])."""
+    X = _f32(X)
+    rows, K = X.shape
+    keep, group = pattern(p)
+    _, K_lp = fp4_shape(p, K)
+    Xv = np.zeros((rows, K_lp // 2), dtype=np.uint8)
+    Xs = np.zeros((rows, K_lp // block), dtype=np.uint8)
+    g = np.zeros(rows, dtype=np.float32)
+    _check(lib().ssref_quant_nvfp4(_ptr(X), rows, K, keep, group, block, 1 if per_row else 0,
+                                   _ptr(Xv), _ptr(Xs), _ptr(g)), "quant_nvfp4")
+    return Xv, Xs, g
+
+
+def decode_sparse_nvfp4(Av, Am, As, K_lp: int) -> np.ndarray:
+    Av = np.ascontiguousarray(Av, dtype=np.uint8)
+    rows = Av.shape[0]
+    A = np.zeros((rows, K_lp), dtype=np.float64)
+    _check(lib().ssref_decode_sparse_nvfp4(_ptr(Av), _ptr(np.ascontiguousarray(Am, np.uint8)),
+                                           _ptr(np.ascontiguousarray(As, np.uint8)), rows, K_lp,
+                                           _ptr(A)), "decode_sparse_nvfp4")
+    return A
+
+
+def decode_dense_nvfp4(Xv, Xs, K_lp: int, block: int) -> np.ndarray:
+    Xv = np.ascontiguousarray(Xv, dtype=np.uint8)
+    rows = Xv.shape[0]
+    X = np.zeros((rows, K_lp), dtype=np.float64)
+    _check(lib().ssref_decode_dense_nvfp4(_ptr(Xv), _ptr(np.ascontiguousarray(Xs, np.uint8)),
+                                          rows, K_lp, block, _ptr(X)), "decode_dense_nvfp4")
+    return X
+
+
+def matmul_nvfp4(Xd, g_x, Wd, g_w, out_dtype: int, m_idx=None):
+    """Y = ((float)(Xd . Wd^T) * g_x[m]) * g_w[n] over decoded operands."""
+    Xd = np.ascontiguousarray(Xd, dtype=np.float64)
+    Wd = np.ascontiguousarray(Wd, dtype=np.float64)
+    g_x = np.ascontiguousarray(g_x, dtype=np.float32)
+    g_w = np.ascontiguousarray(g_w, dtype=np.float32)
+    M, K = Xd.shape
+    N = Wd.shape[0]
+    m_idx, R = _rows(m_idx, M)
+    Y = _out(R, N, out_dtype)
+    _check(lib().ssref_matmul_nvfp4(_ptr(Xd), _ptr(g_x), _ptr(Wd), _ptr(g_w), M, N, K,
+                                    _ptr(m_idx), R, out_dtype, _ptr(Y)), "matmul_nvfp4")
+    return Y
+
+
+def sparse_gemm_nvfp4(Wv, Wm, Ws, g_w: float, Xv, Xs, g_x, M: int, N: int, K_lp: int,
+                      out_dtype: int, m_idx=None):
+    """The sparse NVFP4 product: decoded W (2 kept pairs per window of 4,
+    16-value blocks) against decoded lifted X (32-element blocks)."""
+    Wd = decode_sparse_nvfp4(Wv, Wm, Ws, K_lp)
+    Xd = decode_dense_nvfp4(Xv, Xs, K_lp, 32)
+    return matmul_nvfp4(Xd, g_x, Wd, np.full(N, g_w, dtype=np.float32), out_dtype, m_idx)
+
+
+def dense_gemm_nvfp4(Xv, Xs, g_x, Wv, Ws, g_w, out_dtype: int, m_idx=None):
+    """The dense NVFP4 comparator (16-element blocks on both operands)."""
+    K_lp = Xv.shape[1] * 2
+    Xd = decode_dense_nvfp4(Xv, Xs, K_lp, 16)
+    Wd = decode_dense_nvfp4(Wv, Ws, K_lp, 16)
+    g_w = np.ascontiguousarray(g_w, dtype=np.float32)
+    return matmul_nvfp4(Xd, g_x, Wd, np.broadcast_to(g_w, (Wd.shape[0],)).copy(), out_dtype,
+                        m_idx)

@@ -49,6 +49,27 @@
  *      precision-tier tables): values are stored as bf16 (round to nearest
  *      even from the input), no scale; products of bf16 values are exact in
  *      double, summed in k order, rounded once to binary32.
+ *   R10 NVFP4 ([LC] NVFP4 row: 4-bit floats, a local scale per group of 16
+ *      elements and a global scale per tensor; [PD] 3.3: Blackwell's sparse
+ *      FP4 keeps 2 of every 4 adjacent pairs in 8 elements):
+ *      - elements are E2M1 (sign, 2 exponent bits with bias 1, 1 mantissa
+ *        bit: 0, 0.5, 1, 1.5, 2, 3, 4, 6), round to nearest even, saturating;
+ *        code = sign << 3 | magnitude index; two per byte, low nibble first;
+ *      - local scales are E4M3 with the sign clear (UE4M3); global scale
+ *        g = amax / (6 * 448) in fp32; a block with amax a gets
+ *        s = UE4M3(a / (6 g)), divisor d = s * g, inv = 1 / d (0 if d = 0)
+ *        and codes E2M1(x * inv), every step one fp32 operation;
+ *      - weights: one global scale per tensor; activations: one per token
+ *        (no calibration set exists here, so it is taken from the row);
+ *      - sparsity is on pairs of adjacent elements: a pattern keep:group
+ *        counts pairs (2:4 is the hardware's pairwise 4:8), pairs are ranked
+ *        by x0^2 + x1^2 (ties keep the lower pair) and slid as units, and a
+ *        window of 4 pairs stores its 2 kept pairs with the nibble
+ *        p0 | p1 << 2;
+ *      - block size: 16 stored values of a sparse operand (= 32 lifted
+ *        elements), 32 lifted elements of the dense operand of a sparse
+ *        product, 16 elements in a dense product -- the sparse FP4 tensor-core
+ *        instruction applies one scale per 32 lifted K to both operands.
  */
 #include <math.h>
 #include <stdint.h>
@@ -62,6 +83,7 @@
 #define SSREF_INT8 0
 #define SSREF_FP8_E4M3 1
 #define SSREF_BF16 2
+#define SSREF_NVFP4 3
 
 #define SSREF_OUT_F32 0
 #define SSREF_OUT_BF16 1
@@ -726,4 +748,264 @@ int ssref_sparse_gemm(int sparse_operand, const uint8_t *Av, const uint8_t *Am,
     }
     free(A);
     return st;
+}
+
+
+/* ------------------------------------------------------------------ */
+/* NVFP4 (reading R10).                                                  */
+/* ------------------------------------------------------------------ */
+static const double E2M1_MAG[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+/* Nearest E2M1 value, ties to the even code (the one with mantissa bit 0),
+ * |v| above 6 saturating to 6; the sign is kept, so a negative value that
+ * rounds to zero gives -0 (IEEE rounding keeps the sign of a zero result). */
+uint8_t ssref_e2m1_from_float(float v) {
+    double a = fabs((double)v);
+    int best = 0;
+    for (int i = 1; i < 8; i++) {
+        double di = fabs(a - E2M1_MAG[i]), db = fabs(a - E2M1_MAG[best]);
+        if (di < db || (di == db && (i & 1) == 0)) best = i;
+    }
+    if (a > 6.0) best = 7;
+    uint8_t sign = signbit(v) ? 8 : 0;
+    return (uint8_t)(sign | best);
+}
+
+double ssref_e2m1_to_double(uint8_t c) {
+    double m = E2M1_MAG[c & 7];
+    return (c & 8) ? -m : m;
+}
+
+float ssref_nvfp4_global(float amax) {
+    volatile float g = amax / 2688.0f;   /* 6 * 448 */
+    return g;
+}
+
+/* One block of n values with global scale g: codes[i] and the UE4M3 scale. */
+static void nvfp4_block(const float *x, int n, float g, uint8_t *codes, uint8_t *sc) {
+    float a = 0.0f;
+    for (int i = 0; i < n; i++) a = fmaxf(a, fabsf(x[i]));
+    *sc = 0;
+    for (int i = 0; i < n; i++) codes[i] = 0;
+    if (g == 0.0f) return;
+    volatile float den = 6.0f * g;
+    volatile float t = a / den;
+    *sc = ssref_e4m3_from_float(t);
+    volatile float d = (float)ssref_e4m3_to_double(*sc) * g;
+    if (d == 0.0f) return;
+    volatile float inv = 1.0f / d;
+    for (int i = 0; i < n; i++) {
+        volatile float y = x[i] * inv;
+        codes[i] = ssref_e2m1_from_float(y);
+    }
+}
+
+static void put_fp4(uint8_t *row, int64_t i, uint8_t c) {
+    if (i & 1) row[i / 2] = (uint8_t)((row[i / 2] & 0x0F) | (c << 4));
+    else row[i / 2] = (uint8_t)((row[i / 2] & 0xF0) | (c & 0x0F));
+}
+
+static uint8_t get_fp4(const uint8_t *row, int64_t i) {
+    return (uint8_t)((row[i / 2] >> (4 * (i & 1))) & 0x0F);
+}
+
+/* Shapes on pairs: K_pairs = ceil(K / 2) is slid like K for elements; the
+ * lifted length in elements is 2 * K_lift_pairs, padded to K_lp (a multiple
+ * of 256: one metadata block of the GEMM).  Dense: K_lp = K rounded to 256. */
+int ssref_fp4_shape(int keep, int group, int64_t K, int64_t *K_lift, int64_t *K_lp) {
+    if (K <= 0) return SSREF_EINVAL;
+    if (group == 0) {
+        *K_lift = K;
+        *K_lp = round_up(K, 256);
+        return SSREF_OK;
+    }
+    int64_t Kp_pad, Kp_lift, Kp_lp;
+    int st = ssref_slide_shape(keep, group, (K + 1) / 2, &Kp_pad, &Kp_lift, &Kp_lp);
+    if (st) return st;
+    *K_lift = 2 * Kp_lift;
+    *K_lp = 2 * Kp_lp;
+    return SSREF_OK;
+}
+
+/* Pair mask: per group of `group` pairs keep the `keep` pairs of largest
+ * x0^2 + x1^2 (double), ties keep the lower pair.  mask[r * P_pad + p]. */
+int ssref_prune_pairs(const float *W, int64_t rows, int64_t K, int keep, int group,
+                      uint8_t *mask) {
+    int64_t P = (K + 1) / 2, P_pad = round_up(P, group);
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t g = 0; g < P_pad / group; g++)
+            for (int p = 0; p < group; p++) {
+                double e[32];
+                for (int q = 0; q < group; q++) {
+                    int64_t k0 = 2 * (g * group + q);
+                    double x0 = k0 < K ? W[r * K + k0] : 0.0;
+                    double x1 = k0 + 1 < K ? W[r * K + k0 + 1] : 0.0;
+                    e[q] = x0 * x0 + x1 * x1;
+                }
+                int rank = 0;
+                for (int q = 0; q < group; q++)
+                    if (q != p && (e[q] > e[p] || (e[q] == e[p] && q < p))) rank++;
+                mask[r * P_pad + g * group + p] = rank < keep ? 1 : 0;
+            }
+    return SSREF_OK;
+}
+
+/* Sparse NVFP4 weight: prune pairs, slide them into windows of 4 pairs (the
+ * first-fit of R3 on pairs), store each window's 2 kept pairs (4 values) and
+ * a nibble, then quantise the stored values in blocks of 16 with one
+ * global scale for the tensor.
+ *   Wv [N, K_lp/4] bytes (K_lp/2 stored codes), Wm [N, K_lp/16] bytes
+ *   (nibble per window of 8 lifted elements, low nibble first), Ws [N,
+ *   K_lp/32] UE4M3, *g_w. */
+int ssref_compress_weight_nvfp4(const float *W, int64_t N, int64_t K, int keep, int group,
+                                uint8_t *Wv, uint8_t *Wm, uint8_t *Ws, float *g_w) {
+    int64_t K_lift, K_lp;
+    int st = ssref_fp4_shape(keep, group, K, &K_lift, &K_lp);
+    if (st || group == 0) return SSREF_EINVAL;
+    for (int64_t i = 0; i < N * K; i++)
+        if (!isfinite(W[i])) return SSREF_EINVAL;
+    int Nh = group / 2;
+    int64_t P = (K + 1) / 2, P_pad = round_up(P, group);
+    uint8_t *mask = (uint8_t *)malloc((size_t)(N * P_pad));
+    int8_t *win = (int8_t *)malloc((size_t)(N * P_pad));
+    float *stored = (float *)malloc((size_t)(K_lp / 2) * sizeof(float));
+    ssref_prune_pairs(W, N, K, keep, group, mask);
+    st = ssref_assign_windows(mask, N, P_pad, group, win);
+    if (st) { free(mask); free(win); free(stored); return st; }
+    /* global amax over the kept weights */
+    float amax = 0.0f;
+    for (int64_t r = 0; r < N; r++)
+        for (int64_t p = 0; p < P; p++)
+            if (mask[r * P_pad + p])
+                for (int h = 0; h < 2; h++)
+                    if (2 * p + h < K) amax = fmaxf(amax, fabsf(W[r * K + 2 * p + h]));
+    float g = ssref_nvfp4_global(amax);
+    *g_w = g;
+    memset(Wv, 0, (size_t)(N * K_lp / 4));
+    memset(Wm, 0, (size_t)(N * K_lp / 16));
+    for (int64_t r = 0; r < N; r++) {
+        for (int64_t i = 0; i < K_lp / 2; i++) stored[i] = 0.0f;
+        for (int64_t w = 0; w < K_lp / 8; w++) {       /* windows of 4 pairs */
+            uint8_t assigned[4] = {0, 0, 0, 0};
+            int64_t pbase = 0;
+            if (w < K_lift / 8) {
+                int64_t gi = w / (Nh - 1);
+                int j = (int)(w % (Nh - 1));
+                pbase = gi * group + 2 * j;
+                for (int t = 0; t < 4; t++)
+                    if (win[r * P_pad + pbase + t] == j) assigned[t] = 1;
+            }
+            int idx[2];
+            uint8_t nib = window_slots(assigned, idx);
+            for (int s2 = 0; s2 < 2; s2++)
+                for (int h = 0; h < 2; h++) {
+                    int64_t k = 2 * (pbase + idx[s2]) + h;
+                    stored[4 * w + 2 * s2 + h] = (assigned[idx[s2]] && k < K) ? W[r * K + k] : 0.0f;
+                }
+            put_nibble(&Wm[r * (K_lp / 16)], w, nib);
+        }
+        for (int64_t b = 0; b < K_lp / 32; b++) {        /* blocks of 16 stored */
+            uint8_t codes[16];
+            nvfp4_block(&stored[16 * b], 16, g, codes, &Ws[r * (K_lp / 32) + b]);
+            for (int i = 0; i < 16; i++) put_fp4(&Wv[r * (K_lp / 4)], 16 * b + i, codes[i]);
+        }
+    }
+    free(mask);
+    free(win);
+    free(stored);
+    return SSREF_OK;
+}
+
+/* Dense NVFP4 matrix (the comparator's operands, or the dense operand of a
+ * sparse product): rows of K (lifted on pairs for a pattern), zero-padded to
+ * K_lp, blocks of `block` elements, global scale per row (per_row) or one for
+ * the whole matrix.  Xv [rows, K_lp/2] bytes, Xs [rows, K_lp/block], g[rows]. */
+int ssref_quant_nvfp4(const float *X, int64_t rows, int64_t K, int keep, int group, int block,
+                      int per_row, uint8_t *Xv, uint8_t *Xs, float *g_out) {
+    int64_t K_lift, K_lp;
+    int st = ssref_fp4_shape(keep, group, K, &K_lift, &K_lp);
+    if (st || (block != 16 && block != 32)) return SSREF_EINVAL;
+    int Nh = group / 2;
+    float amax_all = 0.0f;
+    for (int64_t i = 0; i < rows * K; i++) amax_all = fmaxf(amax_all, fabsf(X[i]));
+    float *lifted = (float *)malloc((size_t)K_lp * sizeof(float));
+    memset(Xv, 0, (size_t)(rows * K_lp / 2));
+    for (int64_t r = 0; r < rows; r++) {
+        const float *x = &X[r * K];
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; k++) amax = fmaxf(amax, fabsf(x[k]));
+        float g = ssref_nvfp4_global(per_row ? amax : amax_all);
+        g_out[r] = g;
+        for (int64_t k = 0; k < K_lp; k++) {
+            int64_t src = -1;
+            if (group == 0) {
+                src = k;
+            } else if (k < K_lift) {           /* window i of 4 pairs, element t */
+                int64_t wi = k / 8, t = k % 8;
+                int64_t gi = wi / (Nh - 1), j = wi % (Nh - 1);
+                src = 2 * (gi * group + 2 * j) + t;
+            }
+            lifted[k] = (src >= 0 && src < K) ? x[src] : 0.0f;
+        }
+        for (int64_t b = 0; b < K_lp / block; b++) {
+            uint8_t codes[32];
+            nvfp4_block(&lifted[block * b], block, g, codes, &Xs[r * (K_lp / block) + b]);
+            for (int i = 0; i < block; i++) put_fp4(&Xv[r * (K_lp / 2)], block * b + i, codes[i]);
+        }
+    }
+    free(lifted);
+    return SSREF_OK;
+}
+
+/* Decode a sparse NVFP4 operand to lifted values (block scales applied, the
+ * global scale not): A[r, k] for k < K_lp. */
+int ssref_decode_sparse_nvfp4(const uint8_t *Av, const uint8_t *Am, const uint8_t *As,
+                              int64_t rows, int64_t K_lp, double *A) {
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t w = 0; w < K_lp / 8; w++) {
+            uint8_t nib = get_nibble(&Am[r * (K_lp / 16)], w);
+            int p0 = nib & 3, p1 = (nib >> 2) & 3;
+            if (p0 >= p1) return SSREF_EINVAL;
+            for (int t = 0; t < 8; t++) A[r * K_lp + 8 * w + t] = 0.0;
+            for (int s2 = 0; s2 < 2; s2++)
+                for (int h = 0; h < 2; h++) {
+                    int64_t i = 4 * w + 2 * s2 + h;          /* stored index */
+                    double sc = ssref_e4m3_to_double(As[r * (K_lp / 32) + i / 16]);
+                    double v = ssref_e2m1_to_double(get_fp4(&Av[r * (K_lp / 4)], i)) * sc;
+                    A[r * K_lp + 8 * w + 2 * (s2 ? p1 : p0) + h] = v;
+                }
+        }
+    return SSREF_OK;
+}
+
+int ssref_decode_dense_nvfp4(const uint8_t *Xv, const uint8_t *Xs, int64_t rows, int64_t K_lp,
+                             int block, double *X) {
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t k = 0; k < K_lp; k++)
+            X[r * K_lp + k] = ssref_e2m1_to_double(get_fp4(&Xv[r * (K_lp / 2)], k)) *
+                              ssref_e4m3_to_double(Xs[r * (K_lp / block) + k / block]);
+    return SSREF_OK;
+}
+
+/* Y[i, n] = ((float)sum_k Xd[m_i, k] Wd[n, k] * g_x[m_i]) * g_w[n] over
+ * decoded operands (double sum of exact products, k order), bf16 RNE or
+ * fp32 out. */
+int ssref_matmul_nvfp4(const double *Xd, const float *g_x, const double *Wd, const float *g_w,
+                       int64_t M, int64_t N, int64_t K, const int64_t *m_idx, int64_t n_rows,
+                       int out_dtype, void *Y) {
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < n_rows; i++) {
+        int64_t m = m_idx ? m_idx[i] : i;
+        if (m < 0 || m >= M) continue;
+        for (int64_t n = 0; n < N; n++) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; k++) acc += Xd[m * K + k] * Wd[n * K + k];
+            volatile float a = (float)acc;
+            volatile float t = a * g_x[m];
+            volatile float y = t * g_w[n];
+            if (out_dtype == SSREF_OUT_F32) ((float *)Y)[i * N + n] = y;
+            else ((uint16_t *)Y)[i * N + n] = ssref_bf16_from_float(y);
+        }
+    }
+    return SSREF_OK;
 }
