@@ -172,6 +172,82 @@ ss_status ss_dense_gemm(const void *Xq, const float *s_x, const void *Wq, const 
                         int64_t M, int64_t N, int64_t K_p, ss_qdtype q, void *Y,
                         ss_out_dtype out_dtype, ss_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * NVFP4 with pairwise sparsity (the Blackwell sparse FP4 of the "add 2:4 or
+ * drop a precision tier?" study, paper-daily 2610.28947, 3.3: 2 of every 4
+ * adjacent pairs in 8 elements kept; the NVFP4 row of the LLM-Compressor
+ * compression-schemes page: E2M1 elements, a local scale per group of 16,
+ * a global scale per tensor).
+ *
+ * Elements are E2M1 codes (sign << 3 | magnitude index of 0, .5, 1, 1.5, 2,
+ * 3, 4, 6), two per byte, low nibble = lower K.  Local scales are UE4M3
+ * (E4M3 with the sign clear).  With global scale g = amax / 2688 (fp32), a
+ * block of absolute maximum a gets s = UE4M3(a / (6 g)), d = s * g,
+ * inv = 1 / d (0 if d = 0) and codes E2M1(x * inv), round to nearest even,
+ * saturating, each step one fp32 operation.
+ *
+ * A pattern keep:group counts PAIRS of adjacent elements: 2:4 is the
+ * hardware's pairwise 4:8, and 4:6, 6:8, 8:10 slide windows of 4 pairs with
+ * a stride of 2 pairs, exactly as the 8-bit patterns slide elements.  A
+ * window of 4 pairs stores its 2 kept pairs (ascending) and the nibble
+ * p0 | p1 << 2.  The sparse tensor-core instruction applies one scale per
+ * 32 lifted K to both operands: 16 stored values of the sparse weight, 32
+ * elements of the dense activation; the dense comparator uses 16.
+ *
+ * Scale storage is tile-major in 512-byte blocks, the source shape of the
+ * tensor-memory copy: scale j (= k / block) of row r is at
+ *   ((r / 128) * (n_blocks / 4) + j / 4) * 512 + (r % 32) * 16
+ *     + ((r % 128) / 32) * 4 + j % 4,      n_blocks = K_lp / block,
+ * rows padded to 128 (padding scales 0).  Sparse metadata is the tile-major
+ * layout of ss_meta_bytes() over K_lp / 2 (16 bytes cover 256 lifted K).
+ * ------------------------------------------------------------------------ */
+
+/* Lifted and padded lengths for NVFP4 under pattern p (counted in pairs):
+ * K_lift = 2 * (the pair slide's lifted length), K_lp = K_lift rounded up
+ * to 256.  Dense: K_lift = K, K_lp = K rounded up to 256. */
+ss_status ss_fp4_shape(ss_pattern p, int64_t K, int64_t *K_lift, int64_t *K_lp);
+
+/* Bytes of a tile-major scale buffer for `rows` rows of K_lp lifted elements
+ * with `block` (16 or 32) elements per scale; 0 for invalid shapes. */
+int64_t ss_fp4_scale_bytes(int64_t rows, int64_t K_lp, int32_t block);
+
+/* NVFP4 weight (offline).  Sparse pattern: prune pairs (keep the 2Nh-2 of
+ * every 2Nh pairs of largest x0^2 + x1^2, ties keep the lower pair), slide
+ * them into windows of 4 pairs (ascending first fit), store 2 pairs per
+ * window, quantise the stored values in blocks of 16 with one global scale
+ * for the tensor (amax of the kept weights).  Outputs: Wv [N, K_lp/4] bytes,
+ * Wm ss_meta_bytes(N, K_lp/2) bytes, Ws ss_fp4_scale_bytes(N, K_lp, 32),
+ * g_w[1].  Dense pattern: Wv [N, K_lp/2], Wm unused, Ws with block 16.
+ * A NaN/Inf weight sets SS_ERR_DATA in the device status. */
+ss_status ss_compress_weight_nvfp4(const void *W, ss_in_dtype in_dtype, int64_t N, int64_t K,
+                                   ss_pattern p, void *Wv, void *Wm, void *Ws, float *g_w,
+                                   ss_stream_t stream);
+
+/* NVFP4 activation: per token, global scale g_x[m] = amax(row) / 2688 (no
+ * calibration set exists, so it is taken from the row), the pair lift of
+ * pattern p, blocks of `block` lifted elements (32 for the sparse product,
+ * 16 for the dense one).  Outputs Xv [M, K_lp/2] bytes, Xs
+ * ss_fp4_scale_bytes(M, K_lp, block), g_x [M]. */
+ss_status ss_quant_lift_act_nvfp4(const void *X, ss_in_dtype in_dtype, int64_t M, int64_t K,
+                                  ss_pattern p, int32_t block, void *Xv, void *Xs, float *g_x,
+                                  ss_stream_t stream);
+
+/* Sparse NVFP4 GEMM (tcgen05.mma.sp kind::mxf4nvf4, block-scaled, single SM
+ * per MMA): Y[m, n] = ((float)acc[m, n] * g_x[m]) * g_w[0], acc the fp32
+ * tensor-core sum of (codes x local scales) products; A = the compressed
+ * weight, B = the lifted activation (block 32).  K_lp a positive multiple
+ * of 256. */
+ss_status ss_sparse_gemm_nvfp4(const void *Wv, const void *Wm, const void *Ws, const float *g_w,
+                               const void *Xv, const void *Xs, const float *g_x, int64_t M,
+                               int64_t N, int64_t K_lp, void *Y, ss_out_dtype out_dtype,
+                               ss_stream_t stream);
+
+/* Dense NVFP4 GEMM of the same construction (kind::mxf4nvf4, blocks of 16
+ * on both operands), the comparator.  K_p a positive multiple of 256. */
+ss_status ss_dense_gemm_nvfp4(const void *Xv, const void *Xs, const float *g_x, const void *Wv,
+                              const void *Ws, const float *g_w, int64_t M, int64_t N,
+                              int64_t K_p, void *Y, ss_out_dtype out_dtype, ss_stream_t stream);
+
 /* Synchronises `stream`, returns the first device-side error recorded since
  * the last call (SS_ERR_TIMEOUT, SS_ERR_DATA) or SS_OK, and clears it. */
 ss_status ss_get_device_status(ss_stream_t stream);

@@ -565,3 +565,20 @@ def dense_gemm_nvfp4(Xv, Xs, g_x, Wv, Ws, g_w, out_dtype: int, m_idx=None):
     g_w = np.ascontiguousarray(g_w, dtype=np.float32)
     return matmul_nvfp4(Xd, g_x, Wd, np.broadcast_to(g_w, (Wd.shape[0],)).copy(), out_dtype,
                         m_idx)
+
+
+def scales_to_tiles(S: np.ndarray, K_lp: int, block: int) -> np.ndarray:
+    """Row-layout UE4M3 scales [rows, K_lp/block] -> the library's tile-major
+    storage: 512-byte blocks of 128 rows x 4 consecutive scales, inside a
+    block byte (r % 32) * 16 + ((r % 128) / 32) * 4 + j % 4 (the source shape
+    of the tensor-memory copy); rows padded to 128 with zeros.  A pure
+    relabelling of bytes."""
+    S = np.ascontiguousarray(S, dtype=np.uint8)
+    rows, nblk = S.shape
+    assert nblk == K_lp // block and nblk % 4 == 0
+    rt = (rows + 127) // 128
+    P = np.zeros((rt * 128, nblk), dtype=np.uint8)
+    P[:rows] = S
+    # [rt, q (row/32 % 4), l (row % 32), kb (j/4), s (j%4)] -> [rt, kb, l, q, s]
+    T = P.reshape(rt, 4, 32, nblk // 4, 4).transpose(0, 3, 2, 1, 4)
+    return np.ascontiguousarray(T).reshape(-1)

@@ -14,10 +14,13 @@ Low-level calls (same names and argument order as the C ABI, outputs
 preallocated by the caller):
     ss_parse_pattern, ss_slide_shape, ss_act_2to4_shape, ss_compress_weight,
     ss_quant_lift_act, ss_prune_act_2to4, ss_sparse_gemm, ss_dense_gemm,
-    ss_get_device_status, ss_status_string, ss_kernel_launches
+    ss_get_device_status, ss_status_string, ss_kernel_launches, ss_meta_bytes,
+    ss_fp4_shape, ss_fp4_scale_bytes, ss_compress_weight_nvfp4,
+    ss_quant_lift_act_nvfp4, ss_sparse_gemm_nvfp4, ss_dense_gemm_nvfp4
 Convenience wrappers that allocate their outputs with torch:
     compress_weight, quant_lift_act, prune_act_2to4, sparse_gemm, dense_gemm,
-    linear
+    linear, and for NVFP4 compress_weight_nvfp4, quant_lift_act_nvfp4,
+    sparse_gemm_nvfp4, dense_gemm_nvfp4, linear_nvfp4
 """
 from __future__ import annotations
 
@@ -80,6 +83,11 @@ def lib() -> ctypes.CDLL:
         "ss_sparse_gemm": [i32, p, p, p, p, p, i64, i64, i64, i32, p, i32, p],
         "ss_dense_gemm": [p, p, p, p, i64, i64, i64, i32, p, i32, p],
         "ss_get_device_status": [p],
+        "ss_fp4_shape": [pat, i64, ctypes.POINTER(i64), ctypes.POINTER(i64)],
+        "ss_compress_weight_nvfp4": [p, i32, i64, i64, pat, p, p, p, p, p],
+        "ss_quant_lift_act_nvfp4": [p, i32, i64, i64, pat, i32, p, p, p, p],
+        "ss_sparse_gemm_nvfp4": [p, p, p, p, p, p, p, i64, i64, i64, p, i32, p],
+        "ss_dense_gemm_nvfp4": [p, p, p, p, p, p, i64, i64, i64, p, i32, p],
     }
     for name, args in sigs.items():
         fn = getattr(L, name)
@@ -91,6 +99,8 @@ def lib() -> ctypes.CDLL:
     L.ss_kernel_launches.restype = i64
     L.ss_meta_bytes.argtypes = [i64, i64]
     L.ss_meta_bytes.restype = i64
+    L.ss_fp4_scale_bytes.argtypes = [i64, i64, i32]
+    L.ss_fp4_scale_bytes.restype = i64
     del f
     _lib = L
     return L
@@ -306,3 +316,117 @@ def linear(X: torch.Tensor, packed, pattern, q, out_dtype=torch.bfloat16, stream
     if _pattern(pattern).group == 0:
         return dense_gemm(Xq, s_x, Wv, s_w, q, out_dtype, stream)
     return sparse_gemm(0, Wv, Wm, s_w, Xq, s_x, M, N, q, out_dtype, stream)
+
+
+# ------------------------------------------------------------------ NVFP4 (pairwise sparse FP4)
+# Patterns count pairs of adjacent elements ("2:4" = the hardware's pairwise
+# 4:8).  Values are packed E2M1 codes (uint8, two per byte), local scales
+# UE4M3 bytes in the tile-major layout of ss_fp4_scale_bytes, global scales
+# fp32 (one per weight tensor, one per token).
+
+def ss_fp4_shape(pattern, K: int) -> tuple[int, int]:
+    a, b = ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().ss_fp4_shape(_pattern(pattern), int(K), ctypes.byref(a), ctypes.byref(b)),
+           "ss_fp4_shape")
+    return a.value, b.value
+
+
+def ss_fp4_scale_bytes(rows: int, K_lp: int, block: int) -> int:
+    return int(lib().ss_fp4_scale_bytes(int(rows), int(K_lp), int(block)))
+
+
+def ss_compress_weight_nvfp4(W, pattern, Wv, Wm, Ws, g_w, stream=None) -> None:
+    N, K = W.shape
+    _check(lib().ss_compress_weight_nvfp4(_dev(W, "W"), _in_dtype(W), N, K, _pattern(pattern),
+                                          _dev(Wv, "Wv"), _dev(Wm, "Wm"), _dev(Ws, "Ws"),
+                                          _dev(g_w, "g_w"), _stream(stream)),
+           "ss_compress_weight_nvfp4")
+
+
+def ss_quant_lift_act_nvfp4(X, pattern, block: int, Xv, Xs, g_x, stream=None) -> None:
+    M, K = X.shape
+    _check(lib().ss_quant_lift_act_nvfp4(_dev(X, "X"), _in_dtype(X), M, K, _pattern(pattern),
+                                         int(block), _dev(Xv, "Xv"), _dev(Xs, "Xs"),
+                                         _dev(g_x, "g_x"), _stream(stream)),
+           "ss_quant_lift_act_nvfp4")
+
+
+def ss_sparse_gemm_nvfp4(Wv, Wm, Ws, g_w, Xv, Xs, g_x, M: int, N: int, K_lp: int, Y,
+                         stream=None) -> None:
+    _check(lib().ss_sparse_gemm_nvfp4(_dev(Wv, "Wv"), _dev(Wm, "Wm"), _dev(Ws, "Ws"),
+                                      _dev(g_w, "g_w"), _dev(Xv, "Xv"), _dev(Xs, "Xs"),
+                                      _dev(g_x, "g_x"), int(M), int(N), int(K_lp), _dev(Y, "Y"),
+                                      _out_dtype(Y), _stream(stream)), "ss_sparse_gemm_nvfp4")
+
+
+def ss_dense_gemm_nvfp4(Xv, Xs, g_x, Wv, Ws, g_w, M: int, N: int, K_p: int, Y,
+                        stream=None) -> None:
+    _check(lib().ss_dense_gemm_nvfp4(_dev(Xv, "Xv"), _dev(Xs, "Xs"), _dev(g_x, "g_x"),
+                                     _dev(Wv, "Wv"), _dev(Ws, "Ws"), _dev(g_w, "g_w"), int(M),
+                                     int(N), int(K_p), _dev(Y, "Y"), _out_dtype(Y),
+                                     _stream(stream)), "ss_dense_gemm_nvfp4")
+
+
+def compress_weight_nvfp4(W: torch.Tensor, pattern, stream=None):
+    """-> (Wv, Wm, Ws, g_w); Wm is None for 'dense' (blocks of 16)."""
+    N, K = W.shape
+    p = _pattern(pattern)
+    _, K_lp = ss_fp4_shape(p, K)
+    dev = W.device
+    if p.group == 0:
+        Wv = torch.empty((N, K_lp // 2), dtype=torch.uint8, device=dev)
+        Wm = None
+        Ws = torch.empty(ss_fp4_scale_bytes(N, K_lp, 16), dtype=torch.uint8, device=dev)
+    else:
+        Wv = torch.empty((N, K_lp // 4), dtype=torch.uint8, device=dev)
+        Wm = torch.empty(meta_shape(N, K_lp // 2), dtype=torch.uint8, device=dev)
+        Ws = torch.empty(ss_fp4_scale_bytes(N, K_lp, 32), dtype=torch.uint8, device=dev)
+    g_w = torch.empty(4, dtype=torch.float32, device=dev)   # [0] is the global scale
+    ss_compress_weight_nvfp4(W, p, Wv, Wm, Ws, g_w, stream)
+    return Wv, Wm, Ws, g_w
+
+
+def quant_lift_act_nvfp4(X: torch.Tensor, pattern, block: int, stream=None, out=None):
+    """-> (Xv [M, K_lp/2] uint8, Xs scale bytes, g_x [M])."""
+    M, K = X.shape
+    p = _pattern(pattern)
+    _, K_lp = ss_fp4_shape(p, K)
+    if out is None:
+        out = (torch.empty((M, K_lp // 2), dtype=torch.uint8, device=X.device),
+               torch.empty(ss_fp4_scale_bytes(M, K_lp, block), dtype=torch.uint8, device=X.device),
+               torch.empty(M, dtype=torch.float32, device=X.device))
+    ss_quant_lift_act_nvfp4(X, p, block, out[0], out[1], out[2], stream)
+    return out
+
+
+def sparse_gemm_nvfp4(packed, act, M: int, N: int, out_dtype=torch.bfloat16, stream=None,
+                      out=None):
+    Wv, Wm, Ws, g_w = packed
+    Xv, Xs, g_x = act
+    K_lp = Xv.shape[1] * 2
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=Xv.device)
+    ss_sparse_gemm_nvfp4(Wv, Wm, Ws, g_w, Xv, Xs, g_x, M, N, K_lp, out, stream)
+    return out
+
+
+def dense_gemm_nvfp4(act, packed, M: int, N: int, out_dtype=torch.bfloat16, stream=None,
+                     out=None):
+    Xv, Xs, g_x = act
+    Wv, _, Ws, g_w = packed
+    K_p = Xv.shape[1] * 2
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=Xv.device)
+    ss_dense_gemm_nvfp4(Xv, Xs, g_x, Wv, Ws, g_w, M, N, K_p, out, stream)
+    return out
+
+
+def linear_nvfp4(X: torch.Tensor, packed, pattern, out_dtype=torch.bfloat16, stream=None):
+    """Y = X W^T in NVFP4: per-token quant + pair lift (blocks of 32 for a
+    sparse weight, 16 for a dense one), then the block-scaled GEMM."""
+    dense = _pattern(pattern).group == 0
+    act = quant_lift_act_nvfp4(X, pattern, 16 if dense else 32, stream)
+    M, N = X.shape[0], packed[0].shape[0]
+    if dense:
+        return dense_gemm_nvfp4(act, packed, M, N, out_dtype, stream)
+    return sparse_gemm_nvfp4(packed, act, M, N, out_dtype, stream)

@@ -15,6 +15,7 @@
 #include "ss.h"
 #include "ss_common.cuh"
 #include "ss_compress.cuh"
+#include "ss_fp4.cuh"
 #include "ss_gemm.cuh"
 #include "ss_gemm_splitk.cuh"
 #include "ss_gemm_wide.cuh"
@@ -160,8 +161,10 @@ bool make_y_map(CUtensorMap* map, void* Y, int64_t M, int64_t N, bool out_bf16, 
 
 template <bool kSparse, int kQ, bool kOutBf16, int kPair>
 ss_status launch_gemm(int dev, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& e,
-                      const CUtensorMap& y, const ss::GemmArgs& args, cudaStream_t stream) {
-    using C = ss::GemmCfg<kSparse, kPair, kQ == ss::kQBf16 ? 2 : 1>;
+                      const CUtensorMap& y, const ss::GemmArgs& args, cudaStream_t stream,
+                      const CUtensorMap* sfa = nullptr, const CUtensorMap* sfb = nullptr) {
+    using C = std::conditional_t<kQ == ss::kQNvfp4, ss::Fp4Cfg<kSparse>,
+                                 ss::GemmCfg<kSparse, kPair, kQ == ss::kQBf16 ? 2 : 1>>;
     auto kern = ss::gemm_kernel<kSparse, kQ, kOutBf16, kPair>;
     static std::once_flag once[kMaxDevices];
     static cudaError_t attr_err[kMaxDevices];
@@ -176,7 +179,7 @@ ss_status launch_gemm(int dev, const CUtensorMap& a, const CUtensorMap& b, const
     const int64_t units = g_num_sms[dev] / kPair;
     const int grid = static_cast<int>((tiles < units ? tiles : units) * kPair);
     return launch_ex(kern, dim3(grid), dim3(ss::kGemmThreads), C::kSmemBytes, stream, kPair, a, b,
-                     e, y, args);
+                     e, y, sfa ? *sfa : a, sfb ? *sfb : a, args);
 }
 
 // q: ss::kQE4M3, kQInt8 or kQBf16; bf16: Y element type.
@@ -689,6 +692,7 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
     args.a_is_w = sparse_operand == 0 ? 1 : 0;
     args.ldy = static_cast<int>(N);
     args.e_chunks = static_cast<int>(K_lp / 128);
+    args.sf_k = 0;
     args.s_a = s_a;
     args.s_b = s_b;
     args.y = Y;
@@ -761,6 +765,7 @@ ss_status ss_dense_gemm(const void* Xq, const float* s_x, const void* Wq, const 
     args.a_is_w = 1;
     args.ldy = static_cast<int>(N);
     args.e_chunks = 0;
+    args.sf_k = 0;
     args.s_a = s_w;
     args.s_b = s_x;
     args.y = Y;
@@ -776,6 +781,192 @@ ss_status ss_dense_gemm(const void* Xq, const float* s_x, const void* Wq, const 
     }
     return pair == 2 ? dispatch_gemm<false, 2>(dev, kq, bf, ta, tb, ta, ty, args, st_)
                      : dispatch_gemm<false, 1>(dev, kq, bf, ta, tb, ta, ty, args, st_);
+}
+
+// ---------------------------------------------------------------- NVFP4
+
+ss_status ss_fp4_shape(ss_pattern p, int64_t K, int64_t* K_lift, int64_t* K_lp) {
+    if (!valid_pattern(p) || K <= 0 || K > (int64_t{1} << 30) || !K_lift || !K_lp)
+        return SS_ERR_INVALID_ARG;
+    if (p.group == 0) {
+        *K_lift = K;
+        *K_lp = round_up(K, 256);
+        return SS_OK;
+    }
+    int64_t kp_pad, kp_lift, kp_lp;
+    const ss_status st = ss_slide_shape(p, (K + 1) / 2, &kp_pad, &kp_lift, &kp_lp);
+    if (st != SS_OK) return st;
+    *K_lift = 2 * kp_lift;
+    *K_lp = 2 * kp_lp;
+    return SS_OK;
+}
+
+int64_t ss_fp4_scale_bytes(int64_t rows, int64_t K_lp, int32_t block) {
+    if (rows < 1 || rows > INT32_MAX || K_lp <= 0 || K_lp % 256 != 0 || K_lp > (int64_t{1} << 30) ||
+        (block != 16 && block != 32))
+        return 0;
+    return (rows + 127) / 128 * 128 * (K_lp / block);
+}
+
+ss_status ss_compress_weight_nvfp4(const void* W, ss_in_dtype in_dtype, int64_t N, int64_t K,
+                                   ss_pattern p, void* Wv, void* Wm, void* Ws, float* g_w,
+                                   ss_stream_t stream) {
+    int64_t K_lift, K_lp;
+    ss_status st = ss_fp4_shape(p, K, &K_lift, &K_lp);
+    if (st != SS_OK) return st;
+    const bool dense = p.group == 0;
+    if (!W || !Wv || !Ws || !g_w || (!dense && !Wm) || N <= 0 || N > INT32_MAX)
+        return SS_ERR_INVALID_ARG;
+    if (in_dtype != SS_IN_F32 && in_dtype != SS_IN_BF16) return SS_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(Wv) || !aligned16(Ws) || !aligned16(g_w) ||
+        (!dense && !aligned16(Wm)))
+        return SS_ERR_ALIGNMENT;
+    const int64_t P_pad = dense ? (K + 1) / 2 : round_up((K + 1) / 2, p.group);
+    const int64_t len = dense ? K_lp : 2 * P_pad;
+    const size_t smem1 = static_cast<size_t>(round_up(2 * P_pad, 4) * 4);
+    const size_t smem2 = static_cast<size_t>(round_up(len, 4) * 4) +
+                         (dense ? 0 : static_cast<size_t>(K_lp / 2 * 4 + 2 * (P_pad / p.group) + 16));
+    if (smem1 > kMaxRowSmem || smem2 > kMaxRowSmem) return SS_ERR_UNSUPPORTED;
+    int dev;
+    if ((st = check_device(&dev)) != SS_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    auto* amax = reinterpret_cast<unsigned int*>(g_w);  // pass 1 leaves the amax bits here
+    if (cudaMemsetAsync(amax, 0, sizeof(unsigned int), s) != cudaSuccess) return SS_ERR_CUDA;
+    const int64_t rows_grid = (N + 127) / 128 * 128;
+    auto* wv = static_cast<uint8_t*>(Wv);
+    auto* wm = static_cast<uint8_t*>(Wm);
+    auto* ws = static_cast<uint8_t*>(Ws);
+#define SS_FP4W(T)                                                                             \
+    do {                                                                                      \
+        auto k1 = ss::fp4_weight_amax_kernel<T>;                                               \
+        auto k2 = ss::compress_weight_nvfp4_kernel<T>;                                         \
+        if ((st = set_smem(k1, dev, smem1)) != SS_OK) return st;                              \
+        if ((st = set_smem(k2, dev, smem2)) != SS_OK) return st;                              \
+        const T* w = static_cast<const T*>(W);                                                \
+        if ((st = launch_ex(k1, dim3(static_cast<unsigned>(N)), dim3(ss::kCompressThreads),   \
+                            smem1, s, 1, w, N, K, p.keep, p.group, amax)) != SS_OK)           \
+            return st;                                                                        \
+        if ((st = launch_ex(k2, dim3(static_cast<unsigned>(rows_grid)),                       \
+                            dim3(ss::kCompressThreads), smem2, s, 1, w, N, K, p.keep,          \
+                            p.group, K_lift, K_lp, amax, wv, wm, ws)) != SS_OK)               \
+            return st;                                                                        \
+    } while (0)
+    if (in_dtype == SS_IN_BF16) SS_FP4W(__nv_bfloat16);
+    else SS_FP4W(float);
+#undef SS_FP4W
+    return launch_ex(ss::fp4_global_kernel, dim3(1), dim3(32), 0, s, 1, g_w);
+}
+
+ss_status ss_quant_lift_act_nvfp4(const void* X, ss_in_dtype in_dtype, int64_t M, int64_t K,
+                                  ss_pattern p, int32_t block, void* Xv, void* Xs, float* g_x,
+                                  ss_stream_t stream) {
+    int64_t K_lift, K_lp;
+    ss_status st = ss_fp4_shape(p, K, &K_lift, &K_lp);
+    if (st != SS_OK) return st;
+    if (!X || !Xv || !Xs || !g_x || M <= 0 || M > INT32_MAX || (block != 16 && block != 32))
+        return SS_ERR_INVALID_ARG;
+    if (in_dtype != SS_IN_F32 && in_dtype != SS_IN_BF16) return SS_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(Xv) || !aligned16(Xs) || !aligned16(g_x))
+        return SS_ERR_ALIGNMENT;
+    int dev;
+    if ((st = check_device(&dev)) != SS_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int warps = ss::kWarpRowThreads / 32;
+    const unsigned grid = static_cast<unsigned>(((M + 127) / 128 * 128 + warps - 1) / warps);
+    const int Nh = p.group / 2;
+    auto* xv = static_cast<uint8_t*>(Xv);
+    auto* xs = static_cast<uint8_t*>(Xs);
+#define SS_FP4X(T, B)                                                                          \
+    return launch_ex(ss::quant_lift_nvfp4_kernel<T, B>, dim3(grid), dim3(ss::kWarpRowThreads), \
+                     0, s, 1, static_cast<const T*>(X), M, K, Nh, static_cast<int>(p.group),   \
+                     K_lift, K_lp, xv, xs, g_x)
+    if (in_dtype == SS_IN_BF16) {
+        if (block == 32) SS_FP4X(__nv_bfloat16, 32);
+        SS_FP4X(__nv_bfloat16, 16);
+    }
+    if (block == 32) SS_FP4X(float, 32);
+    SS_FP4X(float, 16);
+#undef SS_FP4X
+}
+
+}  // extern "C"
+
+namespace {
+
+// Shared by the two NVFP4 GEMMs: single-SM tiles of 128 weight rows x up to
+// 128 tokens (one B tile for small M, else 128 so that every B tile starts a
+// 128-row scale tile).
+template <bool kSparse>
+ss_status gemm_nvfp4(const void* Av, const void* Am, const void* As, const float* g_w,
+                     const void* Bv, const void* Bs, const float* g_x, int64_t M, int64_t N,
+                     int64_t K_lp, void* Y, ss_out_dtype out_dtype, ss_stream_t stream) {
+    if (!Av || (kSparse && !Am) || !As || !g_w || !Bv || !Bs || !g_x || !Y)
+        return SS_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || M > INT32_MAX || N > INT32_MAX || K_lp <= 0 || K_lp % 256 != 0 ||
+        K_lp > (int64_t{1} << 30))
+        return SS_ERR_INVALID_ARG;
+    if (out_dtype != SS_OUT_F32 && out_dtype != SS_OUT_BF16) return SS_ERR_INVALID_ARG;
+    if (!aligned16(Av) || (kSparse && !aligned16(Am)) || !aligned16(As) || !aligned16(Bv) ||
+        !aligned16(Bs) || !aligned16(Y))
+        return SS_ERR_ALIGNMENT;
+    int dev;
+    ss_status st = check_device(&dev);
+    if (st != SS_OK) return st;
+    using C = ss::Fp4Cfg<kSparse>;
+    const int block = kSparse ? 32 : 16;
+    const int bn = M <= C::kBnMax ? static_cast<int>(round_up(M, 32)) : C::kBnMax;
+    const int64_t a_bytes = kSparse ? K_lp / 4 : K_lp / 2;  // bytes per A row
+    const int64_t nblk = K_lp / block;
+    CUtensorMap ta, tb, te, tsa, tsb;
+    if (!make_map_2d(&ta, Av, N, a_bytes, ss::kTileA, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tb, Bv, M, K_lp / 2, bn, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tsa, As, (N + 127) / 128 * nblk, 128, 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map_2d(&tsb, Bs, (M + 127) / 128 * nblk, 128, 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return SS_ERR_CUDA;
+    if (kSparse) {
+        if (!make_map_2d(&te, Am, (N + 127) / 128 * (K_lp / 256) * 16, 128, 16, 128,
+                         CU_TENSOR_MAP_SWIZZLE_NONE))
+            return SS_ERR_CUDA;
+    } else {
+        te = ta;  // unused
+    }
+    ss::GemmArgs args;
+    args.rowsA = static_cast<int>(N);
+    args.rowsB = static_cast<int>(M);
+    args.k_stages = static_cast<int>((K_lp + C::kStageK - 1) / C::kStageK);
+    args.bn = bn;
+    args.a_is_w = 1;
+    args.ldy = static_cast<int>(N);
+    args.e_chunks = static_cast<int>(K_lp / 256);
+    args.sf_k = static_cast<int>(nblk / 4);
+    args.s_a = g_w;
+    args.s_b = g_x;
+    args.y = Y;
+    CUtensorMap ty;
+    args.tma_store = make_y_map(&ty, Y, M, N, out_dtype == SS_OUT_BF16, true) ? 1 : 0;
+    if (!args.tma_store) ty = ta;  // unused
+    cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
+    if (out_dtype == SS_OUT_BF16)
+        return launch_gemm<kSparse, ss::kQNvfp4, true, 1>(dev, ta, tb, te, ty, args, st_, &tsa,
+                                                          &tsb);
+    return launch_gemm<kSparse, ss::kQNvfp4, false, 1>(dev, ta, tb, te, ty, args, st_, &tsa, &tsb);
+}
+
+}  // namespace
+
+extern "C" {
+
+ss_status ss_sparse_gemm_nvfp4(const void* Wv, const void* Wm, const void* Ws, const float* g_w,
+                               const void* Xv, const void* Xs, const float* g_x, int64_t M,
+                               int64_t N, int64_t K_lp, void* Y, ss_out_dtype out_dtype,
+                               ss_stream_t stream) {
+    return gemm_nvfp4<true>(Wv, Wm, Ws, g_w, Xv, Xs, g_x, M, N, K_lp, Y, out_dtype, stream);
+}
+
+ss_status ss_dense_gemm_nvfp4(const void* Xv, const void* Xs, const float* g_x, const void* Wv,
+                              const void* Ws, const float* g_w, int64_t M, int64_t N,
+                              int64_t K_p, void* Y, ss_out_dtype out_dtype, ss_stream_t stream) {
+    return gemm_nvfp4<false>(Wv, nullptr, Ws, g_w, Xv, Xs, g_x, M, N, K_p, Y, out_dtype, stream);
 }
 
 ss_status ss_get_device_status(ss_stream_t stream) {

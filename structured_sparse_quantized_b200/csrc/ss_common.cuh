@@ -306,6 +306,7 @@ __host__ __device__ constexpr uint32_t make_idesc(bool sparse, bool is_int8, uin
 constexpr int kQE4M3 = 0;
 constexpr int kQInt8 = 1;
 constexpr int kQBf16 = 2;
+constexpr int kQNvfp4 = 3;  // E2M1 with UE4M3 block scales (kind::mxf4nvf4)
 
 // Instruction descriptor for kind::f16 with bf16 A and B (format 1 in bits
 // 7-9 and 10-12), fp32 accumulator, both operands K-major.
@@ -314,8 +315,17 @@ __host__ __device__ constexpr uint32_t make_idesc_bf16(bool sparse, uint32_t M, 
            ((M >> 4) << 24);
 }
 
+// Instruction descriptor for kind::mxf4nvf4 (block-scaled): E2M1 A and B
+// (format 1 in bits 7-9 and 10-12), UE4M3 scales (bit 23 clear), scale IDs 0
+// (bits 4-5, 29-30: each MMA's scales start a tensor-memory column), K-major.
+__host__ __device__ constexpr uint32_t make_idesc_fp4(bool sparse, uint32_t M, uint32_t N) {
+    return (sparse ? (1u << 2) : 0u) | (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
 __host__ __device__ constexpr uint32_t make_idesc_q(bool sparse, int q, uint32_t M, uint32_t N) {
-    return q == kQBf16 ? make_idesc_bf16(sparse, M, N) : make_idesc(sparse, q == kQInt8, M, N);
+    return q == kQBf16    ? make_idesc_bf16(sparse, M, N)
+           : q == kQNvfp4 ? make_idesc_fp4(sparse, M, N)
+                          : make_idesc(sparse, q == kQInt8, M, N);
 }
 
 template <bool kInt8>
@@ -585,6 +595,38 @@ __device__ __forceinline__ void mma_sparse_bf16_g(uint32_t d_tmem, uint64_t a_de
                 d_tmem),
             "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
             : "memory");
+}
+
+// Block-scaled FP4 MMAs (single SM): scale factors of A and B in tensor
+// memory, one 32-bit column per 32 rows (4 scales) with the rows of each
+// 32-lane quarter repeated in all four quarters (tcgen05.cp .32x128b.warpx4).
+__device__ __forceinline__ void mma_fp4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], "
+        "[%5], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_fp4_sparse(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t e_tmem, uint32_t idesc, uint32_t sfa,
+                                               uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %7, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, [%3], "
+        "%4, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+        : "memory");
+}
+
+// Shared memory -> tensor memory, 32 lanes x 128 bits copied to all four
+// lane quarters (the scale-factor source: [32 rows][16 B], 512 bytes).
+__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t src_desc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc)
+                 : "memory");
 }
 
 // Two fp32 products in one instruction (mul.rn.f32x2): (a0 * b0, a1 * b1),

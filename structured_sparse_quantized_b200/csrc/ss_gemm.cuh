@@ -40,6 +40,8 @@
 // Every wait is bounded (ss_common.cuh); no load multicasts.
 #pragma once
 
+#include <type_traits>
+
 #include "ss_common.cuh"
 
 namespace ss {
@@ -99,6 +101,48 @@ struct GemmCfg {
     static_assert((2 * kStages + 5) * 8 + 4 <= 256, "barrier area");
 };
 
+// Stage layout of the block-scaled FP4 GEMM (single SM, M = 128): per stage
+// 4 MMAs (sparse: K = 128 lifted each, dense: K = 64), A 128 rows x 128 B,
+// B up to 128 rows x 256 B (sparse) / 128 B (dense), sparse metadata 2 x 2 KB,
+// and the scale factors of A and B, 4 x 512 B each.  Tensor memory: two
+// 128-column accumulators, then a metadata slot (8 columns, sparse) and a
+// scale slot (16 columns for A, 16 for B) per stage.
+template <bool kSparse>
+struct Fp4Cfg {
+    static constexpr int kStageK = kSparse ? 512 : 256;
+    static constexpr int kMmaK = kSparse ? 128 : 64;
+    static constexpr int kMmaPerStage = 4;
+    static constexpr int kARowBytes = 128;
+    static constexpr int kABytes = kTileA * kARowBytes;
+    static constexpr int kBAtoms = kSparse ? 2 : 1;
+    static constexpr int kBnMax = 128;
+    static constexpr int kBRowsMax = kBnMax;
+    static constexpr int kBAtomBytes = kBRowsMax * 128;
+    static constexpr int kBBytes = kBAtoms * kBAtomBytes;
+    static constexpr int kEChunks = kSparse ? 2 : 0;
+    static constexpr int kEBytes = kEChunks * kTileA * 16;
+    static constexpr int kSfBytes = 4 * 512;  // one operand's scales for a stage
+    static constexpr int kBOffset = kABytes;
+    static constexpr int kEOffset = kBOffset + kBBytes;
+    static constexpr int kSfaOffset = kEOffset + kEBytes;
+    static constexpr int kSfbOffset = kSfaOffset + kSfBytes;
+    static constexpr int kStageBytes = (kSfbOffset + kSfBytes + 1023) / 1024 * 1024;
+    static constexpr int kEpiBytes = 32 * kTileA * 2;
+    static constexpr int kSmemBudget = 225 * 1024 - 1024 - 256 - 2 * kEpiBytes;
+    static constexpr int kStagesRaw = kSmemBudget / kStageBytes;
+    static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+    static constexpr int kAccStride = kBnMax;
+    static constexpr int kECol = 2 * kBnMax;
+    static constexpr int kESlotCols = 4 * kEChunks;
+    static constexpr int kESlots = kStages;
+    static constexpr int kSfCol = kECol + kStages * kESlotCols;  // scale slots: 32 columns each
+    static constexpr int kEpiOffset = kStages * kStageBytes;
+    static constexpr int kSmemBytes = kEpiOffset + 2 * kEpiBytes + 1024 + 256;
+    static_assert(kSfCol % 4 == 0 && kSfCol + 32 * kStages <= kTmemCols, "TMEM budget");
+    static_assert(kSmemBytes <= 227 * 1024 && kStages >= 2, "shared memory budget");
+    static_assert((2 * kStages + 5) * 8 + 4 <= 256, "barrier area");
+};
+
 struct GemmArgs {
     int rowsA;        // rows of A
     int rowsB;        // rows of B
@@ -109,6 +153,8 @@ struct GemmArgs {
     int tma_store;    // 1: Y written by TMA tensor stores through shared memory
                       //    (A rows = channels: 128B-swizzled [32][64] halves)
     int e_chunks;     // K_lp / 128: 2 KB metadata tiles per 128 rows (tile-major)
+                      // (block-scaled FP4: K_lp / 256)
+    int sf_k;         // FP4: MMA k-blocks per 128-row scale tile (4 scales each)
     const float* s_a;
     const float* s_b;
     void* y;
@@ -135,14 +181,20 @@ __device__ __forceinline__ float load_scale(const float* s, int i, bool in_range
 }
 
 // kQ: kQE4M3, kQInt8 (kind::f8f6f4 / kind::i8) or kQBf16 (kind::f16).
+// kQ: kQE4M3, kQInt8 (kind::f8f6f4 / kind::i8), kQBf16 (kind::f16) or kQNvfp4
+// (kind::mxf4nvf4, block-scaled; single SM only; tm_sfa / tm_sfb are its
+// scale-factor maps, unused otherwise, and s_a is one global scale).
 template <bool kSparse, int kQ, bool kOutBf16, int kPair>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_e, const __grid_constant__ CUtensorMap tm_y,
-                const GemmArgs args) {
+                const __grid_constant__ CUtensorMap tm_sfa,
+                const __grid_constant__ CUtensorMap tm_sfb, const GemmArgs args) {
     constexpr bool kInt8 = kQ == kQInt8;
     constexpr bool kBf16 = kQ == kQBf16;
-    using C = GemmCfg<kSparse, kPair, kBf16 ? 2 : 1>;
+    constexpr bool kFp4 = kQ == kQNvfp4;
+    static_assert(!kFp4 || kPair == 1, "block-scaled FP4 runs on single SMs");
+    using C = std::conditional_t<kFp4, Fp4Cfg<kSparse>, GemmCfg<kSparse, kPair, kBf16 ? 2 : 1>>;
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -226,8 +278,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         __syncwarp();
         pdl_wait();
-        const uint32_t tx =
-            kPair * (C::kABytes + C::kEBytes + C::kBAtoms * b_rows_cta * 128);
+        const uint32_t tx = kPair * (C::kABytes + C::kEBytes + C::kBAtoms * b_rows_cta * 128) +
+                            (kFp4 ? 2 * 4 * 512 : 0);
         int s = 0;
         uint32_t ph = 0, armed = 0, armed_par = 0;
         bool ok = true;
@@ -266,6 +318,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         for (int u = 0; u < C::kEChunks; ++u)
                             tma_load_2d(st + C::kEOffset + u * kTileA * 16, &tm_e, &full[s], 0,
                                         ((a0 >> 7) * args.e_chunks + kb * C::kEChunks + u) * 16);
+                        if constexpr (kFp4) {
+                            // 4 MMAs' scales of A and of B: 2 KB each, as 16 rows of 128 B
+                            tma_load_2d(st + Fp4Cfg<kSparse>::kSfaOffset, &tm_sfa, &full[s], 0,
+                                        ((a0 >> 7) * args.sf_k + kb * 4) * 4);
+                            tma_load_2d(st + Fp4Cfg<kSparse>::kSfbOffset, &tm_sfb, &full[s], 0,
+                                        ((b0 >> 7) * args.sf_k + kb * 4) * 4);
+                        }
                     }
                 }
                 __syncwarp();
@@ -298,6 +357,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint64_t b_desc0 = smem_desc(base + C::kBOffset, 16, 1024, kSwizzle128B);
             const uint64_t e_desc0 =
                 smem_desc(base + C::kEOffset, 128 * 16, 128, kSwizzleNone);
+            const uint64_t sf_desc0 = smem_desc(base, 512, 128, kSwizzleNone);  // + stage offsets
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -322,7 +382,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         tmem_base + C::kECol + C::kESlotCols * s;
                     const uint32_t d_tmem = tmem_base + buf * C::kAccStride;
                     if (elect_one()) {
-                        if constexpr (kSparse) {
+                        if constexpr (kFp4) {
+                            const uint32_t sf_tmem = tmem_base + Fp4Cfg<kSparse>::kSfCol + 32 * s;
+#pragma unroll
+                            for (int t = 0; t < 4; ++t) {
+                                tc_cp_32x128b_warpx4(
+                                    sf_tmem + 4 * t,
+                                    sf_desc0 + soff + ((Fp4Cfg<kSparse>::kSfaOffset + 512 * t) >> 4));
+                                tc_cp_32x128b_warpx4(
+                                    sf_tmem + 16 + 4 * t,
+                                    sf_desc0 + soff + ((Fp4Cfg<kSparse>::kSfbOffset + 512 * t) >> 4));
+                            }
+                            if constexpr (kSparse) {
+#pragma unroll
+                                for (int u = 0; u < C::kEChunks; ++u)
+                                    tc_cp_128x128b(e_tmem + 4 * u,
+                                                   e_desc0 + soff + ((u * kTileA * 16) >> 4));
+                            }
+#pragma unroll
+                            for (int j = 0; j < C::kMmaPerStage; ++j) {
+                                const uint64_t a_desc = a_desc0 + soff + ((j * 32) >> 4);
+                                const uint32_t accum = (kb > 0 || j > 0) ? 1u : 0u;
+                                if constexpr (kSparse) {
+                                    const uint64_t b_desc =
+                                        b_desc0 + soff +
+                                        (((j >> 1) * C::kBAtomBytes + (j & 1) * 64) >> 4);
+                                    mma_fp4_sparse(d_tmem, a_desc, b_desc, e_tmem + 2 * j, idesc,
+                                                   sf_tmem + 4 * j, sf_tmem + 16 + 4 * j, accum);
+                                } else {
+                                    const uint64_t b_desc = b_desc0 + soff + ((j * 32) >> 4);
+                                    mma_fp4(d_tmem, a_desc, b_desc, idesc, sf_tmem + 4 * j,
+                                            sf_tmem + 16 + 4 * j, accum);
+                                }
+                            }
+                        } else if constexpr (kSparse) {
 #pragma unroll
                             for (int u = 0; u < C::kEChunks; ++u)
                                 tc_cp_128x128b_g<kPair>(e_tmem + 4 * u,
@@ -410,7 +503,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int a_cta0 = a_tile0;
             const int a_row = a_cta0 + lane_row;
             const bool row_ok = a_row < args.rowsA;
-            const float sa = load_scale<kBf16>(args.s_a, a_row, row_ok);
+            const float sa = kFp4 ? __ldg(args.s_a) : load_scale<kBf16>(args.s_a, a_row, row_ok);
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    static_cast<uint32_t>(acc * C::kAccStride);
             if (args.tma_store && args.a_is_w) {
@@ -426,7 +519,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int ch = a_cta0 + q * 32 + 16 * h + t4 + 8 * e;
-                        sa2[h][e] = load_scale<kBf16>(args.s_a, ch, ch < args.rowsA);
+                        sa2[h][e] = kFp4 ? __ldg(args.s_a)
+                                         : load_scale<kBf16>(args.s_a, ch, ch < args.rowsA);
                     }
                 // this thread's stmatrix row: matrix mi, row mj
                 const int mi = lane >> 3, mj = lane & 7;
