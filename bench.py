@@ -177,6 +177,22 @@ class Path:
         self.X_host = synth.make_activation(M, self.K, w["x_kind"], w["in_dtype"])
         self.X = self.X_host.to(device)
         # offline: compress weights (sparse and the dense comparator's)
+        self.fp4 = self.q == "nvfp4"
+        if self.fp4:  # pairwise sparse NVFP4 against dense NVFP4 (patterns count pairs)
+            if self.online:
+                raise ValueError("the NVFP4 path is weight-sparse only")
+            self.dense_w = ss.compress_weight_nvfp4(W, "dense")
+            self.sparse_w = ss.compress_weight_nvfp4(W, self.pat)
+            _, self.K_lp = ss.ss_fp4_shape(self.pat, self.K)
+            _, self.K_p = ss.ss_fp4_shape("dense", self.K)
+            self.act = ss.quant_lift_act_nvfp4(self.X, self.pat, 32)
+            self.dense_act = ss.quant_lift_act_nvfp4(self.X, "dense", 16)
+            self.Y = torch.empty((M, self.N), dtype=self.out_dtype, device=device)
+            del W
+            torch.cuda.synchronize()
+            if ss.ss_get_device_status() != ss.SS_OK:
+                raise RuntimeError("device status not clean after set-up")
+            return
         self.dense_w = ss.compress_weight(W, "dense", self.q)
         if self.online:
             self.K_lp = ss.ss_act_2to4_shape(self.K)
@@ -198,7 +214,12 @@ class Path:
         X = self.X if X is None else X
         if ev:
             ev[0].record()
-        if self.online:
+        if self.fp4:
+            ss.quant_lift_act_nvfp4(X, self.pat, 32, out=self.act)
+            if ev and ev[1] is not None:
+                ev[1].record()
+            ss.sparse_gemm_nvfp4(self.sparse_w, self.act, self.M, self.N, out=self.Y)
+        elif self.online:
             ss.prune_act_2to4(X, self.q, out=self.act)
             if ev and ev[1] is not None:
                 ev[1].record()
@@ -221,7 +242,13 @@ class Path:
         ss = self.ss
         m = r1 - r0
         rows = lambda t: None if t is None else t[r0:r1]  # bf16 tier: no scales
-        if self.online:
+        if self.fp4:
+            Xv, Xs, g_x = self.act
+            nblk = self.K_lp // 32  # tile-major scales: 128-row tiles are contiguous
+            part = (Xv[r0:r1], Xs[r0 * nblk:r1 * nblk], g_x[r0:r1])
+            ss.quant_lift_act_nvfp4(X_rows, self.pat, 32, out=part)
+            ss.sparse_gemm_nvfp4(self.sparse_w, part, m, self.N, out=self.Y[r0:r1])
+        elif self.online:
             Xv, Xm, s_x = self.act
             part = (Xv[r0:r1], Xm[r0 // 128:r1 // 128], rows(s_x))
             ss.prune_act_2to4(X_rows, self.q, out=part)
@@ -240,6 +267,14 @@ class Path:
         ss = self.ss
         if ev:
             ev[0].record()
+        if self.fp4:
+            ss.quant_lift_act_nvfp4(self.X, "dense", 16, out=self.dense_act)
+            if ev and ev[1] is not None:
+                ev[1].record()
+            ss.dense_gemm_nvfp4(self.dense_act, self.dense_w, self.M, self.N, out=self.Y)
+            if ev:
+                ev[2].record()
+            return
         ss.quant_lift_act(self.X, "dense", self.q, out=self.dense_act)
         if ev and ev[1] is not None:
             ev[1].record()
@@ -257,22 +292,29 @@ class Path:
         return 2.0 * self.M * self.N * self.K_lp      # lifted logical MACs x 2
 
     def dense_gemm_ops(self):
+        if self.fp4:
+            return 2.0 * self.M * self.N * self.K_p
         return 2.0 * self.M * self.N * self.dense_w[0].shape[1]
 
     def act_kernel_bytes(self):
         esz = self.X.element_size()
+        if self.fp4:  # codes, one UE4M3 scale per 32, a global scale per token
+            return self.M * (esz * self.K + self.K_lp // 2 + self.K_lp // 32 + 4)
         vb, sb = (2, 0) if self.q == "bf16" else (1, 4)   # value bytes, scale bytes
         if self.online:
             return self.M * (esz * self.K + vb * self.K_lp // 2 + self.K_lp // 8 + sb)
         return self.M * (esz * self.K + vb * self.K_lp + sb)
 
     def dense_act_bytes(self):
+        if self.fp4:
+            return self.M * (self.X.element_size() * self.K + self.K_p // 2 + self.K_p // 16 + 4)
         vb, sb = (2, 0) if self.q == "bf16" else (1, 4)
         return self.M * (self.X.element_size() * self.K + vb * self.dense_act[0].shape[1] + sb)
 
-    # peaks: dense bf16 measured; 8-bit dense = 2x, 2:4 sparse = 2x dense
+    # peaks: dense bf16 measured; 8-bit dense = 2x, FP4 dense = 4x, 2:4 sparse
+    # = 2x dense (NVIDIA's nominal ratios)
     def dense_peak(self, bf16_peak: float) -> float:
-        return bf16_peak * (1.0 if self.q == "bf16" else 2.0)
+        return bf16_peak * {"bf16": 1.0, "nvfp4": 4.0}.get(self.q, 2.0)
 
     def sparse_peak(self, bf16_peak: float) -> float:
         return 2.0 * self.dense_peak(bf16_peak)
@@ -442,18 +484,30 @@ def oracle_sample(name: str, M: int, budget_s: float):
     w = synth.WORKLOADS[name]
     N, K = w["N"], w["K"]
     bf16 = w["qdtype"] == "bf16"
-    q = {"int8": oracle.INT8, "fp8": oracle.FP8_E4M3, "bf16": oracle.BF16}[w["qdtype"]]
+    fp4 = w["qdtype"] == "nvfp4"
+    q = {"int8": oracle.INT8, "fp8": oracle.FP8_E4M3, "bf16": oracle.BF16,
+         "nvfp4": oracle.NVFP4}[w["qdtype"]]
     out = oracle.OUT_F32 if w["out"] == "f32" else oracle.OUT_BF16
     W = synth.make_weight(N, K, w["w_std"], w["in_dtype"])
     online = name.startswith("online")
     pat = "dense" if online else w["pattern"]
-    packed = oracle.compress_weight_bf16(W, pat) if bf16 else oracle.compress_weight(W, pat, q)
+    if fp4:
+        packed = oracle.compress_weight_nvfp4(W, pat)
+    elif bf16:
+        packed = oracle.compress_weight_bf16(W, pat)
+    else:
+        packed = oracle.compress_weight(W, pat, q)
     X = synth.make_activation(M, K, w["x_kind"], w["in_dtype"])
 
     def run(rows):
         Xs = X[rows]
         t0 = time.perf_counter()
-        if bf16 and online:
+        if fp4:
+            Wv, Wm, Ws, g_w = packed
+            Xv, Xsc, g_x = oracle.quant_nvfp4(Xs, pat, 32)
+            oracle.sparse_gemm_nvfp4(Wv, Wm, Ws, g_w, Xv, Xsc, g_x, len(rows), N,
+                                     Xv.shape[1] * 2, out)
+        elif bf16 and online:
             Xv, Xm = oracle.prune_act_2to4_bf16(Xs)
             Wb, _ = packed
             oracle.sparse_gemm_bf16(1, Xv, Xm, Wb, len(rows), N, Wb.shape[1], out)
@@ -533,7 +587,7 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=6.0)
     ap.add_argument("--pattern", default=None, choices=["2:4", "4:6", "6:8", "8:10"],
                     help="override the workload's pattern (the Llama-layer sweep)")
-    ap.add_argument("--qdtype", default=None, choices=["int8", "fp8", "bf16"],
+    ap.add_argument("--qdtype", default=None, choices=["int8", "fp8", "bf16", "nvfp4"],
                     help="override the workload's quantised type")
     args = ap.parse_args()
     if args.pattern or args.qdtype:

@@ -876,6 +876,28 @@ ss_status ss_quant_lift_act_nvfp4(const void* X, ss_in_dtype in_dtype, int64_t M
     const int Nh = p.group / 2;
     auto* xv = static_cast<uint8_t*>(Xv);
     auto* xs = static_cast<uint8_t*>(Xs);
+    // bf16 rows under the identity map with K_lp <= 4096: one read of X, in
+    // registers (two warps per row above 2048, to keep the occupancy up)
+    if (in_dtype == SS_IN_BF16 && Nh <= 2 && K % 8 == 0 && K_lp <= 4096) {
+        const auto* xb = static_cast<const __nv_bfloat16*>(X);
+        const int wpr = K_lp > 2048 ? 2 : 1;
+        const int rows_per_cta = (ss::kWarpRowThreads / 32) / wpr;
+        const unsigned rgrid =
+            static_cast<unsigned>(((M + 127) / 128 * 128 + rows_per_cta - 1) / rows_per_cta);
+        const int chunks = static_cast<int>(K_lp / (256 * wpr));
+#define SS_FP4R(B, C, W)                                                                       \
+    return launch_ex(ss::quant_nvfp4_reg_kernel<B, C, W>, dim3(rgrid),                        \
+                     dim3(ss::kWarpRowThreads), 0, s, 1, xb, M, K, K_lp, xv, xs, g_x)
+        if (block == 32) {
+            if (wpr == 2) SS_FP4R(32, 8, 2);
+            if (chunks <= 4) SS_FP4R(32, 4, 1);
+            SS_FP4R(32, 8, 1);
+        }
+        if (wpr == 2) SS_FP4R(16, 8, 2);
+        if (chunks <= 4) SS_FP4R(16, 4, 1);
+        SS_FP4R(16, 8, 1);
+#undef SS_FP4R
+    }
 #define SS_FP4X(T, B)                                                                          \
     return launch_ex(ss::quant_lift_nvfp4_kernel<T, B>, dim3(grid), dim3(ss::kWarpRowThreads), \
                      0, s, 1, static_cast<const T*>(X), M, K, Nh, static_cast<int>(p.group),   \

@@ -37,8 +37,10 @@ __device__ __forceinline__ uint32_t ue4m3_code(float t) {
 }
 
 __device__ __forceinline__ float ue4m3_value(uint32_t c) {
-    const int e = static_cast<int>((c >> 3) & 15u), m = static_cast<int>(c & 7u);
-    return e == 0 ? ldexpf(static_cast<float>(m), -9) : ldexpf(static_cast<float>(8 + m), e - 10);
+    const uint32_t e = (c >> 3) & 15u, m = c & 7u;
+    // normal: 2^(e - 7) (1 + m / 8) as fp32 bits; subnormal: m 2^-9 (exact)
+    return e == 0 ? __fmul_rn(static_cast<float>(m), 0.001953125f)
+                  : __uint_as_float(((e + 120u) << 23) | (m << 20));
 }
 
 // Tile-major scale offset (512-byte blocks: 128 rows x 4 consecutive scales,
@@ -275,46 +277,155 @@ __global__ void __launch_bounds__(kWarpRowThreads) quant_lift_nvfp4_kernel(
     const float a = warp_row_absmax<T>(x, K, vec, lane);
     const float g = __fdiv_rn(a, 2688.0f);
     if (lane == 0) g_x[m] = g;
-    uint8_t* vrow = Xv + m * (K_lp / 2);
-    for (int64_t b = lane; b < nblk; b += 32) {
-        float v[kBlock];
-        // kBlock / 8 windows of 8 lifted elements, each 8 consecutive inputs
+    // One window of 8 lifted elements per lane; the kBlock / 8 lanes of a
+    // block (adjacent, and always in the same iteration: K_lp / 8 is a
+    // multiple of 32) combine their maxima with shuffles.
+    constexpr int kLanes = kBlock / 8;
+    uint32_t* vrow = reinterpret_cast<uint32_t*>(Xv + m * (K_lp / 2));
+    for (int64_t wi = lane; wi < K_lp / 8; wi += 32) {
+        int64_t src0;
+        if (Nh <= 2) {
+            src0 = 8 * wi;  // dense and pair 2:4: the identity
+        } else if (8 * wi < K_lift) {
+            const int64_t gi = wi / (Nh - 1), j = wi - gi * (Nh - 1);
+            src0 = 2 * (gi * group + 2 * j);
+        } else {
+            src0 = -1;
+        }
+        float v[8];
+        bool done = false;
+        if constexpr (sizeof(T) == 2) {
+            if (src0 >= 0 && src0 + 8 <= K) {
+                const uintptr_t addr = reinterpret_cast<uintptr_t>(x + src0);
+                uint32_t u[4];
+                if ((addr & 15u) == 0) {
+                    const uint4 q = __ldg(reinterpret_cast<const uint4*>(x + src0));
+                    u[0] = q.x, u[1] = q.y, u[2] = q.z, u[3] = q.w;
+                    done = true;
+                } else if ((addr & 3u) == 0) {  // src0 is even; odd K can shift the row
 #pragma unroll
-        for (int wq = 0; wq < kBlock / 8; ++wq) {
-            const int64_t k0 = b * kBlock + 8 * wq;
-            int64_t src0;
-            if (Nh <= 2) {
-                src0 = k0;  // dense and pair 2:4: the identity
-            } else if (k0 < K_lift) {
-                const int64_t wi = k0 >> 3;
-                const int64_t gi = wi / (Nh - 1), j = wi - gi * (Nh - 1);
-                src0 = 2 * (gi * group + 2 * j);
-            } else {
-                src0 = -1;
-            }
-            if constexpr (sizeof(T) == 2) {
-                // whole window in the row and 4-byte aligned (src0 is even, but
-                // a row starts on an odd element when K is odd)
-                if (src0 >= 0 && src0 + 8 <= K &&
-                    (reinterpret_cast<uintptr_t>(x + src0) & 3u) == 0) {
-                    const uint32_t* p = reinterpret_cast<const uint32_t*>(x + src0);
+                    for (int h = 0; h < 4; ++h) u[h] = __ldg(reinterpret_cast<const uint32_t*>(x + src0) + h);
+                    done = true;
+                }
+                if (done) {
 #pragma unroll
                     for (int h = 0; h < 4; ++h) {
-                        const uint32_t u = __ldg(p + h);
-                        v[8 * wq + 2 * h] = __uint_as_float(u << 16);
-                        v[8 * wq + 2 * h + 1] = __uint_as_float(u & 0xFFFF0000u);
+                        v[2 * h] = __uint_as_float(u[h] << 16);
+                        v[2 * h + 1] = __uint_as_float(u[h] & 0xFFFF0000u);
                     }
-                    continue;
                 }
             }
+        }
+        if (!done) {
 #pragma unroll
             for (int t = 0; t < 8; ++t) {
                 const int64_t src = src0 + t;
-                v[8 * wq + t] = (src0 >= 0 && src < K) ? to_f32<T>(x[src]) : 0.0f;
+                v[t] = (src0 >= 0 && src < K) ? to_f32<T>(x[src]) : 0.0f;
             }
         }
-        const uint32_t sc = nvfp4_block<kBlock>(v, g, vrow + b * (kBlock / 2));
-        Xs[fp4_scale_offset(m, b, nblk)] = static_cast<uint8_t>(sc);
+        float a = 0.0f;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) a = fmaxf(a, fabsf(v[t]));
+#pragma unroll
+        for (int o = 1; o < kLanes; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        uint32_t sc = 0;
+        float inv = 0.0f;
+        if (g != 0.0f) {
+            sc = ue4m3_code(__fdiv_rn(a, __fmul_rn(6.0f, g)));
+            const float d = __fmul_rn(ue4m3_value(sc), g);
+            inv = d == 0.0f ? 0.0f : __fdiv_rn(1.0f, d);
+        }
+        uint32_t word = 0;
+        if (inv != 0.0f) {
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+                word |= e2m1x2(__fmul_rn(v[2 * h], inv), __fmul_rn(v[2 * h + 1], inv)) << (8 * h);
+        }
+        __stcs(vrow + wi, word);
+        if ((lane & (kLanes - 1)) == 0)
+            Xs[fp4_scale_offset(m, wi / kLanes, nblk)] = static_cast<uint8_t>(sc);
+    }
+}
+
+// Single-pass variant for bf16 rows with the identity map (dense and pair
+// 2:4) and K_lp <= 256 kChunks kWpr: a row is held by kWpr warps; lane l of
+// warp `sub` keeps the 16-byte chunks (8 inputs = one window) 32 sub + l +
+// 32 kWpr i, so X is read from HBM once; window wi = chunk wi, and the lanes
+// of a block are adjacent as above.  The warps of a row combine their maxima
+// through shared memory (one named barrier per row slot).
+template <int kBlock, int kChunks, int kWpr>
+__global__ void __launch_bounds__(kWarpRowThreads) quant_nvfp4_reg_kernel(
+    const __nv_bfloat16* __restrict__ X, int64_t M, int64_t K64, int64_t K_lp,
+    uint8_t* __restrict__ Xv, uint8_t* __restrict__ Xs, float* __restrict__ g_x) {
+    pdl_trigger();
+    pdl_wait();
+    constexpr int kLanes = kBlock / 8;
+    constexpr int kRowsPerCta = kWarpRowThreads / (32 * kWpr);
+    __shared__ float part[kRowsPerCta][kWpr];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int slot = warp / kWpr, sub = warp % kWpr;
+    const int64_t m = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + slot;
+    const int64_t M_pad = (M + 127) / 128 * 128;
+    const int64_t nblk = K_lp / kBlock;
+    if (m >= M_pad) return;  // whole row slots leave together
+    if (m >= M) {
+        for (int64_t j = sub * 32 + lane; j < nblk; j += 32 * kWpr) Xs[fp4_scale_offset(m, j, nblk)] = 0;
+        return;
+    }
+    const int K = static_cast<int>(K64);
+    const uint4* x = reinterpret_cast<const uint4*>(X + m * K64);  // K % 8 == 0
+    uint4 c[kChunks];
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kChunks; ++i) {
+        const int ch = sub * 32 + lane + 32 * kWpr * i;
+        c[i] = 8 * ch < K ? __ldg(x + ch) : make_uint4(0u, 0u, 0u, 0u);
+        a = fmaxf(a, chunk_absmax<__nv_bfloat16>(c[i]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if constexpr (kWpr > 1) {
+        if (lane == 0) part[slot][sub] = a;
+        named_bar_sync(1 + slot, 32 * kWpr);
+#pragma unroll
+        for (int w = 0; w < kWpr; ++w) a = fmaxf(a, part[slot][w]);
+    }
+    const float g = __fdiv_rn(a, 2688.0f);
+    const float g6 = __fmul_rn(6.0f, g);
+    if (lane == 0 && sub == 0) g_x[m] = g;
+    uint32_t* vrow = reinterpret_cast<uint32_t*>(Xv + m * (K_lp / 2));
+#pragma unroll
+    for (int i = 0; i < kChunks; ++i) {
+        const int64_t wi = sub * 32 + lane + 32 * kWpr * i;
+        if (wi - lane >= K_lp / 8) break;  // the same for every lane (K_lp / 8 % 32 == 0)
+        const uint32_t u[4] = {c[i].x, c[i].y, c[i].z, c[i].w};
+        float v[8];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            v[2 * h] = __uint_as_float(u[h] << 16);
+            v[2 * h + 1] = __uint_as_float(u[h] & 0xFFFF0000u);
+        }
+        float b = 0.0f;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) b = fmaxf(b, fabsf(v[t]));
+#pragma unroll
+        for (int o = 1; o < kLanes; o <<= 1) b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, o));
+        uint32_t sc = 0;
+        float inv = 0.0f;
+        if (g != 0.0f) {
+            sc = ue4m3_code(__fdiv_rn(b, g6));
+            const float d = __fmul_rn(ue4m3_value(sc), g);
+            inv = d == 0.0f ? 0.0f : __frcp_rn(d);
+        }
+        uint32_t word = 0;
+        if (inv != 0.0f) {
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+                word |= e2m1x2(__fmul_rn(v[2 * h], inv), __fmul_rn(v[2 * h + 1], inv)) << (8 * h);
+        }
+        __stcs(vrow + wi, word);
+        if ((lane & (kLanes - 1)) == 0)
+            Xs[fp4_scale_offset(m, wi / kLanes, nblk)] = static_cast<uint8_t>(sc);
     }
 }
 

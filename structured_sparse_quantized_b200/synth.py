@@ -74,6 +74,10 @@ WORKLOADS = {
     # Llama-3.1-8B q_proj shape (compared with dense bf16 and dense FP8)
     "llama_q_2of4_bf16": dict(M=8192, K=4096, N=4096, pattern="2:4", qdtype="bf16",
                               in_dtype="bf16", w_std=0.02, out="bf16", x_kind="outlier"),
+    # Blackwell's sparse FP4: pairwise 4:8 (pattern 2:4 counted in pairs) in
+    # NVFP4 on the Llama-3.1-8B gate/up shape, against dense NVFP4
+    "llama_gateup_4of8_nvfp4": dict(M=8192, K=4096, N=14336, pattern="2:4", qdtype="nvfp4",
+                                    in_dtype="bf16", w_std=0.02, out="bf16", x_kind="gauss"),
 }
 
 # Llama-3.1-8B layer projections (N, K) for the pattern sweep.

@@ -156,3 +156,20 @@ def test_chained_nvfp4_path(pat):
         ref = oracle.sparse_gemm_nvfp4(Wv, Wm, Ws, g_w, Xv, Xs, g_x, M, N, K_lp, oracle.OUT_BF16)
     Y = ss.linear_nvfp4(dev(X), ss.compress_weight_nvfp4(dev(W), pat), pat)
     assert_y_matches(host(Y), ref, "fp8", True)
+
+
+# Many bf16 rows through both activation kernels: the single-pass register
+# kernel (identity map, K_lp <= 4096, with 4, 8 and 16 chunks per lane) and
+# the two-pass kernel (sliding pair patterns and longer rows).
+@pytest.mark.parametrize("pat", ["dense", "2:4", "6:8"])
+@pytest.mark.parametrize("block", [16, 32])
+@pytest.mark.parametrize("M,K", [(3000, 4096), (3000, 3584), (2100, 2048), (2100, 1000),
+                                  (1200, 8192)])
+def test_quant_lift_act_nvfp4_many_rows(pat, block, M, K):
+    X = _x(M, K, "bf16", seed=K + block)
+    Xv, Xs, g_x = ss.quant_lift_act_nvfp4(dev(X), pat, block)
+    Xv_ref, Xs_ref, g_ref = oracle.quant_nvfp4(X, pat, block)
+    _, K_lp = oracle.fp4_shape(pat, K)
+    np.testing.assert_array_equal(host(g_x), g_ref)
+    np.testing.assert_array_equal(host(Xv), Xv_ref)
+    np.testing.assert_array_equal(host(Xs), oracle.scales_to_tiles(Xs_ref, K_lp, block))
