@@ -394,38 +394,44 @@ __global__ void __launch_bounds__(kWarpRowThreads) quant_nvfp4_reg_kernel(
     const float g6 = __fmul_rn(6.0f, g);
     if (lane == 0 && sub == 0) g_x[m] = g;
     uint32_t* vrow = reinterpret_cast<uint32_t*>(Xv + m * (K_lp / 2));
+    // Three passes over the chunks (block maxima, block scales, codes) so that
+    // the chunks' dependency chains (shuffles, divisions, conversions) overlap.
+    float inv[kChunks];
+    uint32_t sc[kChunks];
+#pragma unroll
+    for (int i = 0; i < kChunks; ++i) {
+        float b = chunk_absmax<__nv_bfloat16>(c[i]);
+#pragma unroll
+        for (int o = 1; o < kLanes; o <<= 1) b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, o));
+        inv[i] = b;
+    }
+#pragma unroll
+    for (int i = 0; i < kChunks; ++i) {
+        sc[i] = 0;
+        float r = 0.0f;
+        if (g != 0.0f) {
+            sc[i] = ue4m3_code(__fdiv_rn(inv[i], g6));
+            const float d = __fmul_rn(ue4m3_value(sc[i]), g);
+            r = d == 0.0f ? 0.0f : __frcp_rn(d);
+        }
+        inv[i] = r;
+    }
 #pragma unroll
     for (int i = 0; i < kChunks; ++i) {
         const int64_t wi = sub * 32 + lane + 32 * kWpr * i;
         if (wi - lane >= K_lp / 8) break;  // the same for every lane (K_lp / 8 % 32 == 0)
         const uint32_t u[4] = {c[i].x, c[i].y, c[i].z, c[i].w};
-        float v[8];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            v[2 * h] = __uint_as_float(u[h] << 16);
-            v[2 * h + 1] = __uint_as_float(u[h] & 0xFFFF0000u);
-        }
-        float b = 0.0f;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) b = fmaxf(b, fabsf(v[t]));
-#pragma unroll
-        for (int o = 1; o < kLanes; o <<= 1) b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, o));
-        uint32_t sc = 0;
-        float inv = 0.0f;
-        if (g != 0.0f) {
-            sc = ue4m3_code(__fdiv_rn(b, g6));
-            const float d = __fmul_rn(ue4m3_value(sc), g);
-            inv = d == 0.0f ? 0.0f : __frcp_rn(d);
-        }
         uint32_t word = 0;
-        if (inv != 0.0f) {
+        if (inv[i] != 0.0f) {
 #pragma unroll
             for (int h = 0; h < 4; ++h)
-                word |= e2m1x2(__fmul_rn(v[2 * h], inv), __fmul_rn(v[2 * h + 1], inv)) << (8 * h);
+                word |= e2m1x2(__fmul_rn(__uint_as_float(u[h] << 16), inv[i]),
+                               __fmul_rn(__uint_as_float(u[h] & 0xFFFF0000u), inv[i]))
+                        << (8 * h);
         }
         __stcs(vrow + wi, word);
         if ((lane & (kLanes - 1)) == 0)
-            Xs[fp4_scale_offset(m, wi / kLanes, nblk)] = static_cast<uint8_t>(sc);
+            Xs[fp4_scale_offset(m, wi / kLanes, nblk)] = static_cast<uint8_t>(sc[i]);
     }
 }
 
