@@ -163,7 +163,7 @@ template <bool kSparse, int kQ, bool kOutBf16, int kPair>
 ss_status launch_gemm(int dev, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& e,
                       const CUtensorMap& y, const ss::GemmArgs& args, cudaStream_t stream,
                       const CUtensorMap* sfa = nullptr, const CUtensorMap* sfb = nullptr) {
-    using C = std::conditional_t<kQ == ss::kQNvfp4, ss::Fp4Cfg<kSparse>,
+    using C = std::conditional_t<kQ == ss::kQNvfp4, ss::Fp4Cfg<kSparse, kPair>,
                                  ss::GemmCfg<kSparse, kPair, kQ == ss::kQBf16 ? 2 : 1>>;
     auto kern = ss::gemm_kernel<kSparse, kQ, kOutBf16, kPair>;
     static std::once_flag once[kMaxDevices];
@@ -217,7 +217,7 @@ int splitk_max_clusters(int dev, int S) {
         for (int i = 1; i < 4; ++i) {
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(1 << i);
-            cfg.blockDim = dim3(ss::kGemmThreads);
+            cfg.blockDim = dim3(ss::kSplitKThreads);
             cfg.dynamicSmemBytes = C::kSmemBytes;
             cudaLaunchAttribute attr[1];
             attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -242,7 +242,7 @@ ss_status launch_splitk(int S, int64_t tiles, const CUtensorMap& a, const CUtens
                         const CUtensorMap& e, const ss::GemmArgs& args, cudaStream_t stream) {
     using C = ss::SplitKCfg<kSparse, kQ == ss::kQBf16 ? 2 : 1>;
     return launch_ex(ss::gemm_splitk_kernel<kSparse, kQ, kOutBf16>,
-                     dim3(static_cast<unsigned>(tiles * S)), dim3(ss::kGemmThreads), C::kSmemBytes,
+                     dim3(static_cast<unsigned>(tiles * S)), dim3(ss::kSplitKThreads), C::kSmemBytes,
                      stream, S, a, b, e, args);
 }
 
@@ -915,9 +915,9 @@ ss_status ss_quant_lift_act_nvfp4(const void* X, ss_in_dtype in_dtype, int64_t M
 
 namespace {
 
-// Shared by the two NVFP4 GEMMs: single-SM tiles of 128 weight rows x up to
-// 128 tokens (one B tile for small M, else 128 so that every B tile starts a
-// 128-row scale tile).
+// Shared by the two NVFP4 GEMMs: tiles of 128 weight rows per CTA x up to 128
+// tokens (single SM), or, above 128 weight rows, a CTA pair with MMA M = 256 x
+// up to 256 tokens (two 128-row scale tiles of B).  One B tile covers small M.
 template <bool kSparse>
 ss_status gemm_nvfp4(const void* Av, const void* Am, const void* As, const float* g_w,
                      const void* Bv, const void* Bs, const float* g_x, int64_t M, int64_t N,
@@ -936,12 +936,20 @@ ss_status gemm_nvfp4(const void* Av, const void* Am, const void* As, const float
     if (st != SS_OK) return st;
     using C = ss::Fp4Cfg<kSparse>;
     const int block = kSparse ? 32 : 16;
-    const int bn = M <= C::kBnMax ? static_cast<int>(round_up(M, 32)) : C::kBnMax;
+    // CTA pairs (MMA M = 256, N up to 256 tokens) above one 128-row A tile;
+    // for the sparse product only from K_lp > 2048: with fewer K stages per
+    // tile the pair's single accumulator leaves the MMAs waiting on the
+    // epilogue, and the single-SM form (two accumulators) is faster (measured
+    // at M = 8192, N = 14336: K_lp = 2048 106.6 us single vs 123.0 us pair;
+    // K_lp = 4096 190.7 vs 166.8 us)
+    const int pair = N > ss::kTileA && (!kSparse || K_lp > 2048) ? 2 : 1;
+    const int bn_max = pair == 2 ? ss::Fp4Cfg<kSparse, 2>::kBnMax : C::kBnMax;
+    const int bn = M <= bn_max ? static_cast<int>(round_up(M, 32)) : bn_max;
     const int64_t a_bytes = kSparse ? K_lp / 4 : K_lp / 2;  // bytes per A row
     const int64_t nblk = K_lp / block;
     CUtensorMap ta, tb, te, tsa, tsb;
     if (!make_map_2d(&ta, Av, N, a_bytes, ss::kTileA, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_2d(&tb, Bv, M, K_lp / 2, bn, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tb, Bv, M, K_lp / 2, bn / pair, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&tsa, As, (N + 127) / 128 * nblk, 128, 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_map_2d(&tsb, Bs, (M + 127) / 128 * nblk, 128, 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
         return SS_ERR_CUDA;
@@ -968,10 +976,15 @@ ss_status gemm_nvfp4(const void* Av, const void* Am, const void* As, const float
     args.tma_store = make_y_map(&ty, Y, M, N, out_dtype == SS_OUT_BF16, true) ? 1 : 0;
     if (!args.tma_store) ty = ta;  // unused
     cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
-    if (out_dtype == SS_OUT_BF16)
-        return launch_gemm<kSparse, ss::kQNvfp4, true, 1>(dev, ta, tb, te, ty, args, st_, &tsa,
-                                                          &tsb);
-    return launch_gemm<kSparse, ss::kQNvfp4, false, 1>(dev, ta, tb, te, ty, args, st_, &tsa, &tsb);
+    const bool bf = out_dtype == SS_OUT_BF16;
+    if (pair == 2)
+        return bf ? launch_gemm<kSparse, ss::kQNvfp4, true, 2>(dev, ta, tb, te, ty, args, st_, &tsa,
+                                                               &tsb)
+                  : launch_gemm<kSparse, ss::kQNvfp4, false, 2>(dev, ta, tb, te, ty, args, st_,
+                                                                &tsa, &tsb);
+    return bf ? launch_gemm<kSparse, ss::kQNvfp4, true, 1>(dev, ta, tb, te, ty, args, st_, &tsa, &tsb)
+              : launch_gemm<kSparse, ss::kQNvfp4, false, 1>(dev, ta, tb, te, ty, args, st_, &tsa,
+                                                            &tsb);
 }
 
 }  // namespace

@@ -597,7 +597,7 @@ __device__ __forceinline__ void mma_sparse_bf16_g(uint32_t d_tmem, uint64_t a_de
             : "memory");
 }
 
-// Block-scaled FP4 MMAs (single SM): scale factors of A and B in tensor
+// Block-scaled FP4 MMAs (cta_group::1 form): scale factors of A and B in tensor
 // memory, one 32-bit column per 32 rows (4 scales) with the rows of each
 // 32-lane quarter repeated in all four quarters (tcgen05.cp .32x128b.warpx4).
 __device__ __forceinline__ void mma_fp4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
@@ -623,10 +623,48 @@ __device__ __forceinline__ void mma_fp4_sparse(uint32_t d_tmem, uint64_t a_desc,
 }
 
 // Shared memory -> tensor memory, 32 lanes x 128 bits copied to all four
-// lane quarters (the scale-factor source: [32 rows][16 B], 512 bytes).
-__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t src_desc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc)
-                 : "memory");
+// lane quarters (the scale-factor source: [32 rows][16 B], 512 bytes).  The
+// pair form, issued by the leader, copies each CTA's shared memory into its
+// own tensor memory.
+template <int kPair>
+__device__ __forceinline__ void tc_cp_32x128b_warpx4_g(uint32_t taddr, uint64_t src_desc) {
+    if constexpr (kPair == 2)
+        asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc)
+                     : "memory");
+    else
+        asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc)
+                     : "memory");
+}
+
+// Block-scaled FP4 MMAs in either CTA-group form.
+template <int kPair>
+__device__ __forceinline__ void mma_fp4_g(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                          uint32_t accumulate) {
+    if constexpr (kPair == 2)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, "
+            "[%4], [%5], p;\n\t}" ::"r"(d_tmem),
+            "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+            : "memory");
+    else
+        mma_fp4(d_tmem, a_desc, b_desc, idesc, sfa, sfb, accumulate);
+}
+
+template <int kPair>
+__device__ __forceinline__ void mma_fp4_sparse_g(uint32_t d_tmem, uint64_t a_desc,
+                                                 uint64_t b_desc, uint32_t e_tmem, uint32_t idesc,
+                                                 uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    if constexpr (kPair == 2)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %7, 0;\n\t"
+            "tcgen05.mma.sp.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, "
+            "[%3], %4, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+            "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+            : "memory");
+    else
+        mma_fp4_sparse(d_tmem, a_desc, b_desc, e_tmem, idesc, sfa, sfb, accumulate);
 }
 
 // Two fp32 products in one instruction (mul.rn.f32x2): (a0 * b0, a1 * b1),

@@ -23,7 +23,7 @@
 // one tile while the MMAs of the next fill the other buffer.  (For large
 // problems the sparse GEMM also has a two-B-tile shape, ss_gemm_wide.cuh.)
 //
-// CTA = 6 warps, one CTA per SM, persistent over output tiles:
+// CTA = 10 warps, one CTA per SM, persistent over output tiles:
 //   warp 0       TMA producer (whole warp, one elected lane issues): A tiles,
 //                B atoms and, for the sparse variant, the 128 x 16-byte
 //                metadata chunks of each K stage, into a ring of shared-memory
@@ -33,10 +33,11 @@
 //                whole warp runs the MMA loop and one elected lane issues the
 //                metadata copies into tensor memory, the MMAs, and the commits
 //                that release stages / accumulators in both CTAs.
-//   warps 2-5    epilogue: tcgen05.ld the accumulator (lane = A row, column =
-//                B row), scale, convert, stage a 32-column chunk in shared
-//                memory and write it with one TMA tensor store; release the
-//                accumulator on the leader's barrier.
+//   warps 2-9    epilogue, two groups of four taking alternate 32-column
+//                chunks: tcgen05.ld the accumulator (lane = A row, column =
+//                B row), scale, convert, stage the chunk in the group's
+//                shared-memory buffer and write it with one TMA tensor store;
+//                release the accumulator on the leader's barrier.
 // Every wait is bounded (ss_common.cuh); no load multicasts.
 #pragma once
 
@@ -46,7 +47,8 @@
 
 namespace ss {
 
-constexpr int kGemmThreads = 192;
+constexpr int kGemmEpiWarps = 8;  // two groups of four, one warp per TMEM lane quarter each
+constexpr int kGemmThreads = 64 + 32 * kGemmEpiWarps;
 constexpr int kL2PrefetchStages = 16;  // weight stages a CTA prefetches before pdl_wait
 constexpr int kTileA = 128;  // A rows per CTA per A tile
 constexpr int kTmemCols = 512;
@@ -83,6 +85,8 @@ struct GemmCfg {
     static constexpr int kSmemBudget = 225 * 1024 - 1024 - 256 - 2 * kEpiBytes;
     static constexpr int kStagesRaw = kSmemBudget / kStageBytes;
     static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+    static constexpr int kAccBufs = 2;                     // accumulators in TMEM
+    static constexpr int kSfStageBytes = 0;                // no block scales
     static constexpr int kAccStride = kBnMax;              // TMEM columns between accumulators
     static constexpr int kECol = 2 * kBnMax;               // metadata columns (sparse)
     static constexpr int kESlotCols = 4 * kEChunks;        // columns one stage's metadata takes
@@ -101,13 +105,22 @@ struct GemmCfg {
     static_assert((2 * kStages + 5) * 8 + 4 <= 256, "barrier area");
 };
 
-// Stage layout of the block-scaled FP4 GEMM (single SM, M = 128): per stage
-// 4 MMAs (sparse: K = 128 lifted each, dense: K = 64), A 128 rows x 128 B,
-// B up to 128 rows x 256 B (sparse) / 128 B (dense), sparse metadata 2 x 2 KB,
-// and the scale factors of A and B, 4 x 512 B each.  Tensor memory: two
-// 128-column accumulators, then a metadata slot (8 columns, sparse) and a
-// scale slot (16 columns for A, 16 for B) per stage.
-template <bool kSparse>
+// Stage layout of the block-scaled FP4 GEMM: per stage 4 MMAs (sparse: K =
+// 128 lifted each, dense: K = 64), A 128 rows x 128 B, this CTA's B rows x
+// 256 B (sparse) / 128 B (dense), sparse metadata 2 x 2 KB, the scale factors
+// of A (4 x 512 B) and those of the whole B tile (4 x 512 B per 128-row scale
+// tile).
+//   single SM: MMA M = 128, N = 128; two 128-column accumulators in tensor
+//     memory (the epilogue drains one while the next tile fills the other).
+//   CTA pair:  MMA M = 256, N = 256 (128 B rows per CTA, two scale tiles);
+//     one 256-column accumulator.  An FP4 MMA of N = 128 runs at about half
+//     the rate of one of N = 256, so the pair takes the wide N and gives up
+//     the second accumulator (the epilogue releases it as soon as it has
+//     read it into registers).
+// After the accumulators, tensor memory holds per stage a metadata slot (8
+// columns, sparse) and a scale slot (4 columns per MMA for A, 4 per MMA and
+// scale tile for B).
+template <bool kSparse, int kPair = 1>
 struct Fp4Cfg {
     static constexpr int kStageK = kSparse ? 512 : 256;
     static constexpr int kMmaK = kSparse ? 128 : 64;
@@ -115,31 +128,41 @@ struct Fp4Cfg {
     static constexpr int kARowBytes = 128;
     static constexpr int kABytes = kTileA * kARowBytes;
     static constexpr int kBAtoms = kSparse ? 2 : 1;
-    static constexpr int kBnMax = 128;
-    static constexpr int kBRowsMax = kBnMax;
+    static constexpr int kBnMax = 128 * kPair;
+    static constexpr int kSfbTiles = kBnMax / 128;  // 128-row scale tiles per B tile
+    static constexpr int kAccBufs = kPair == 2 ? 1 : 2;
+    static constexpr int kBRowsMax = kBnMax / kPair;
     static constexpr int kBAtomBytes = kBRowsMax * 128;
     static constexpr int kBBytes = kBAtoms * kBAtomBytes;
     static constexpr int kEChunks = kSparse ? 2 : 0;
     static constexpr int kEBytes = kEChunks * kTileA * 16;
-    static constexpr int kSfBytes = 4 * 512;  // one operand's scales for a stage
+    static constexpr int kSfaBytes = 4 * 512;              // A scales of a stage
+    static constexpr int kSfbBytes = kSfbTiles * 4 * 512;  // B scales of a stage
+    static constexpr int kSfStageBytes = kSfaBytes + kSfbBytes;
     static constexpr int kBOffset = kABytes;
     static constexpr int kEOffset = kBOffset + kBBytes;
     static constexpr int kSfaOffset = kEOffset + kEBytes;
-    static constexpr int kSfbOffset = kSfaOffset + kSfBytes;
-    static constexpr int kStageBytes = (kSfbOffset + kSfBytes + 1023) / 1024 * 1024;
+    static constexpr int kSfbOffset = kSfaOffset + kSfaBytes;
+    static constexpr int kStageBytes = (kSfbOffset + kSfbBytes + 1023) / 1024 * 1024;
     static constexpr int kEpiBytes = 32 * kTileA * 2;
     static constexpr int kSmemBudget = 225 * 1024 - 1024 - 256 - 2 * kEpiBytes;
     static constexpr int kStagesRaw = kSmemBudget / kStageBytes;
-    static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-    static constexpr int kAccStride = kBnMax;
-    static constexpr int kECol = 2 * kBnMax;
     static constexpr int kESlotCols = 4 * kEChunks;
+    static constexpr int kSfaCols = 4 * kMmaPerStage;
+    static constexpr int kSfbCols = 4 * kMmaPerStage * kSfbTiles;
+    static constexpr int kSfSlotCols = kSfaCols + kSfbCols;
+    static constexpr int kStagesTmem =
+        (kTmemCols - kAccBufs * kBnMax) / (kESlotCols + kSfSlotCols);
+    static constexpr int kStagesMin = kStagesRaw < kStagesTmem ? kStagesRaw : kStagesTmem;
+    static constexpr int kStages = kStagesMin > 8 ? 8 : kStagesMin;
+    static constexpr int kAccStride = kBnMax;
+    static constexpr int kECol = kAccBufs * kBnMax;
     static constexpr int kESlots = kStages;
-    static constexpr int kSfCol = kECol + kStages * kESlotCols;  // scale slots: 32 columns each
+    static constexpr int kSfCol = kECol + kStages * kESlotCols;  // scale slots
     static constexpr int kEpiOffset = kStages * kStageBytes;
     static constexpr int kSmemBytes = kEpiOffset + 2 * kEpiBytes + 1024 + 256;
-    static_assert(kSfCol % 4 == 0 && kSfCol + 32 * kStages <= kTmemCols, "TMEM budget");
-    static_assert(kSmemBytes <= 227 * 1024 && kStages >= 2, "shared memory budget");
+    static_assert(kSfCol % 4 == 0 && kSfCol + kSfSlotCols * kStages <= kTmemCols, "TMEM budget");
+    static_assert(kSmemBytes <= 227 * 1024 && kStages >= 3, "shared memory budget");
     static_assert((2 * kStages + 5) * 8 + 4 <= 256, "barrier area");
 };
 
@@ -180,10 +203,9 @@ __device__ __forceinline__ float load_scale(const float* s, int i, bool in_range
     else return in_range ? __ldg(s + i) : 0.0f;
 }
 
-// kQ: kQE4M3, kQInt8 (kind::f8f6f4 / kind::i8) or kQBf16 (kind::f16).
 // kQ: kQE4M3, kQInt8 (kind::f8f6f4 / kind::i8), kQBf16 (kind::f16) or kQNvfp4
-// (kind::mxf4nvf4, block-scaled; single SM only; tm_sfa / tm_sfb are its
-// scale-factor maps, unused otherwise, and s_a is one global scale).
+// (kind::mxf4nvf4, block-scaled; tm_sfa / tm_sfb are its scale-factor maps,
+// unused otherwise, and s_a is one global scale).
 template <bool kSparse, int kQ, bool kOutBf16, int kPair>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -193,8 +215,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     constexpr bool kInt8 = kQ == kQInt8;
     constexpr bool kBf16 = kQ == kQBf16;
     constexpr bool kFp4 = kQ == kQNvfp4;
-    static_assert(!kFp4 || kPair == 1, "block-scaled FP4 runs on single SMs");
-    using C = std::conditional_t<kFp4, Fp4Cfg<kSparse>, GemmCfg<kSparse, kPair, kBf16 ? 2 : 1>>;
+    using C = std::conditional_t<kFp4, Fp4Cfg<kSparse, kPair>, GemmCfg<kSparse, kPair, kBf16 ? 2 : 1>>;
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -229,7 +250,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 4 * kPair);
+            mbar_init(&acc_empty[b], kGemmEpiWarps * kPair);
         }
         mbar_init(drain, 1);
         fence_barrier_init();
@@ -278,8 +299,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         __syncwarp();
         pdl_wait();
-        const uint32_t tx = kPair * (C::kABytes + C::kEBytes + C::kBAtoms * b_rows_cta * 128) +
-                            (kFp4 ? 2 * 4 * 512 : 0);
+        // FP4: each CTA also loads its A scales and the B tile's scales
+        const uint32_t tx = kPair * (C::kABytes + C::kEBytes + C::kBAtoms * b_rows_cta * 128 +
+                                     C::kSfStageBytes);
         int s = 0;
         uint32_t ph = 0, armed = 0, armed_par = 0;
         bool ok = true;
@@ -307,6 +329,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             tma_load_2d_pair_hint(st + C::kEOffset + u * kTileA * 16, &tm_e, fb, 0,
                                                   ((a0 >> 7) * args.e_chunks + kb * C::kEChunks + u) * 16,
                                                   keep);
+                        if constexpr (kFp4) {  // this CTA's A scales, the whole B tile's scales
+                            tma_load_2d_pair_hint(st + C::kSfaOffset, &tm_sfa, fb, 0,
+                                                  ((a0 >> 7) * args.sf_k + kb * 4) * 4, keep);
+                            const int sfb_tile = (t / nA) * args.bn >> 7;
+#pragma unroll
+                            for (int u = 0; u < C::kSfbTiles; ++u)  // past the last: zero fill
+                                tma_load_2d_pair_hint(st + C::kSfbOffset + 2048 * u, &tm_sfb, fb, 0,
+                                                      ((sfb_tile + u) * args.sf_k + kb * 4) * 4,
+                                                      keep);
+                        }
                     } else {
                         mbar_arrive_expect_tx(&full[s], tx);
                         tma_load_2d(st, &tm_a, &full[s], kb * C::kARowBytes, a0);
@@ -320,10 +352,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                         ((a0 >> 7) * args.e_chunks + kb * C::kEChunks + u) * 16);
                         if constexpr (kFp4) {
                             // 4 MMAs' scales of A and of B: 2 KB each, as 16 rows of 128 B
-                            tma_load_2d(st + Fp4Cfg<kSparse>::kSfaOffset, &tm_sfa, &full[s], 0,
+                            tma_load_2d(st + C::kSfaOffset, &tm_sfa, &full[s], 0,
                                         ((a0 >> 7) * args.sf_k + kb * 4) * 4);
-                            tma_load_2d(st + Fp4Cfg<kSparse>::kSfbOffset, &tm_sfb, &full[s], 0,
-                                        ((b0 >> 7) * args.sf_k + kb * 4) * 4);
+#pragma unroll
+                            for (int u = 0; u < C::kSfbTiles; ++u)
+                                tma_load_2d(st + C::kSfbOffset + 2048 * u, &tm_sfb, &full[s], 0,
+                                            (((b0 >> 7) + u) * args.sf_k + kb * 4) * 4);
                         }
                     }
                 }
@@ -363,9 +397,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             bool ok = true;
             int i = 0;
             for (int t = unit; t < n_tiles && ok; t += n_units, ++i) {
-                // double-buffered accumulator: buffer i & 1, one phase per use
-                const int buf = i & 1;
-                const uint32_t aph = (i >> 1) & 1;
+                // accumulator buffer of this tile (two: i & 1; one: 0), one
+                // phase per use
+                const int buf = C::kAccBufs == 2 ? (i & 1) : 0;
+                const uint32_t aph = C::kAccBufs == 2 ? ((i >> 1) & 1) : (i & 1);
                 if (!__all_sync(0xffffffffu, mbar_wait(&acc_empty[buf], aph ^ 1u, abort_flag))) {
                     ok = false;
                     break;
@@ -383,21 +418,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint32_t d_tmem = tmem_base + buf * C::kAccStride;
                     if (elect_one()) {
                         if constexpr (kFp4) {
-                            const uint32_t sf_tmem = tmem_base + Fp4Cfg<kSparse>::kSfCol + 32 * s;
+                            // scale slot: A's 4 columns per MMA, then B's 4
+                            // per MMA and 128-row scale tile
+                            const uint32_t sf_tmem = tmem_base + C::kSfCol + C::kSfSlotCols * s;
+                            const uint32_t sfb_tmem = sf_tmem + C::kSfaCols;
 #pragma unroll
                             for (int t = 0; t < 4; ++t) {
-                                tc_cp_32x128b_warpx4(
-                                    sf_tmem + 4 * t,
-                                    sf_desc0 + soff + ((Fp4Cfg<kSparse>::kSfaOffset + 512 * t) >> 4));
-                                tc_cp_32x128b_warpx4(
-                                    sf_tmem + 16 + 4 * t,
-                                    sf_desc0 + soff + ((Fp4Cfg<kSparse>::kSfbOffset + 512 * t) >> 4));
+                                tc_cp_32x128b_warpx4_g<kPair>(
+                                    sf_tmem + 4 * t, sf_desc0 + soff + ((C::kSfaOffset + 512 * t) >> 4));
+#pragma unroll
+                                for (int u = 0; u < C::kSfbTiles; ++u)
+                                    tc_cp_32x128b_warpx4_g<kPair>(
+                                        sfb_tmem + 4 * (C::kSfbTiles * t + u),
+                                        sf_desc0 + soff +
+                                            ((C::kSfbOffset + 2048 * u + 512 * t) >> 4));
                             }
                             if constexpr (kSparse) {
 #pragma unroll
                                 for (int u = 0; u < C::kEChunks; ++u)
-                                    tc_cp_128x128b(e_tmem + 4 * u,
-                                                   e_desc0 + soff + ((u * kTileA * 16) >> 4));
+                                    tc_cp_128x128b_g<kPair>(e_tmem + 4 * u,
+                                                            e_desc0 + soff + ((u * kTileA * 16) >> 4));
                             }
 #pragma unroll
                             for (int j = 0; j < C::kMmaPerStage; ++j) {
@@ -407,12 +447,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                     const uint64_t b_desc =
                                         b_desc0 + soff +
                                         (((j >> 1) * C::kBAtomBytes + (j & 1) * 64) >> 4);
-                                    mma_fp4_sparse(d_tmem, a_desc, b_desc, e_tmem + 2 * j, idesc,
-                                                   sf_tmem + 4 * j, sf_tmem + 16 + 4 * j, accum);
+                                    mma_fp4_sparse_g<kPair>(d_tmem, a_desc, b_desc, e_tmem + 2 * j,
+                                                            idesc, sf_tmem + 4 * j,
+                                                            sfb_tmem + 4 * C::kSfbTiles * j, accum);
                                 } else {
                                     const uint64_t b_desc = b_desc0 + soff + ((j * 32) >> 4);
-                                    mma_fp4(d_tmem, a_desc, b_desc, idesc, sf_tmem + 4 * j,
-                                            sf_tmem + 16 + 4 * j, accum);
+                                    mma_fp4_g<kPair>(d_tmem, a_desc, b_desc, idesc, sf_tmem + 4 * j,
+                                                     sfb_tmem + 4 * C::kSfbTiles * j, accum);
                                 }
                             }
                         } else if constexpr (kSparse) {
@@ -473,33 +514,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        // Each 32-column chunk of an accumulator is scaled, converted and
-        // written to one of two shared-memory staging buffers laid out as the
-        // chunk's box of Y, then stored by one TMA tensor store (clipped at
-        // the edges of Y).  Without TMA stores (fp32 Y, or Y rows not 16-byte
-        // aligned) the values go straight to global memory.
+        // Two groups of four warps (one warp per TMEM lane quarter in each);
+        // group g takes the 32-column chunks g, g + 2, ... of an accumulator.
+        // A chunk is scaled, converted and written to the group's own
+        // shared-memory staging buffer, laid out as the chunk's box of Y, then
+        // stored by one TMA tensor store (clipped at the edges of Y).  The two
+        // groups' load / convert / store latencies overlap, which is what
+        // keeps the epilogue shorter than the MMAs of a tile when K is short.
+        // Without TMA stores (fp32 Y, or Y rows not 16-byte aligned) the
+        // values go straight to global memory.
+        const int ew = warp - 2;
+        const int grp = ew >> 2;  // chunk parity of this group
+        const uint32_t grp_bar = 1 + static_cast<uint32_t>(grp);
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const int lane_row = q * 32 + lane;
-        const bool issuer = (warp == 2 && lane == 0);
+        const bool issuer = (ew & 3) == 0 && lane == 0;
         const uint32_t acc_empty_leader = kPair == 2 ? map_to_rank(acc_empty, 0) : 0u;
         constexpr int kEsz = 2;  // TMA-store staging is used for bf16 output only
-        uint8_t* stage_y = smem + C::kEpiOffset;
+        uint8_t* sy = smem + C::kEpiOffset + grp * C::kEpiBytes;
         int i = 0;
-        uint32_t chunk_iter = 0;
         bool ok = true;
         for (int t = unit; t < n_tiles && ok; t += n_units, ++i) {
             const int a_tile0 = (t % nA) * tile_a_rows + static_cast<int>(rank) * kTileA;
             const int b0 = (t / nA) * args.bn;
-            const int acc = i & 1;
-            const uint32_t aph = (i >> 1) & 1;
-            // all four epilogue warps take the same decision, so none is left
-            // behind at a named barrier if the wait gives up
+            const int acc = C::kAccBufs == 2 ? (i & 1) : 0;
+            const uint32_t aph = C::kAccBufs == 2 ? ((i >> 1) & 1) : (i & 1);
+            // the four warps of a group take the same decision, so none is
+            // left behind at the group's named barrier if the wait gives up
             const bool got = mbar_wait(&acc_full[acc], aph, abort_flag);
-            if (!named_bar_and(1, 128, got)) {
+            if (!named_bar_and(grp_bar, 128, got)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
+            if (32 * grp >= args.bn) {  // no chunk for this group (bn = 32)
+                __syncwarp();
+                if (lane == 0) {
+                    if constexpr (kPair == 2)
+                        mbar_arrive_cluster(acc_empty_leader + acc * sizeof(uint64_t));
+                    else
+                        mbar_arrive(&acc_empty[acc]);
+                }
+                continue;
+            }
             const int a_cta0 = a_tile0;
             const int a_row = a_cta0 + lane_row;
             const bool row_ok = a_row < args.rowsA;
@@ -524,85 +581,100 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 // this thread's stmatrix row: matrix mi, row mj
                 const int mi = lane >> 3, mj = lane & 7;
-                for (int c = 0; c < args.bn; c += 32) {
-                    uint32_t v[2][16];
-                    tmem_ld_16x256b_x4(t_row + c, v[0]);
-                    tmem_ld_16x256b_x4(t_row + (16u << 16) + c, v[1]);
-                    tmem_ld_wait();
-                    if (c + 32 >= args.bn) {  // last read of this accumulator: release it
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) {
-                            if constexpr (kPair == 2)
-                                mbar_arrive_cluster(acc_empty_leader + acc * sizeof(uint64_t));
-                            else
-                                mbar_arrive(&acc_empty[acc]);
-                        }
-                    }
-                    float sb[4][2];
+                // 1) every chunk of this group into registers as packed bf16
+                //    ([chunk][half][column group r * 2 + channel block])
+                constexpr int kCpg = (C::kBnMax + 63) / 64;  // chunks per group, at most
+                uint32_t pk[kCpg][2][8];
 #pragma unroll
-                    for (int r = 0; r < 4; ++r)
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int tok = b0 + c + 8 * r + 2 * tm + e;
-                            sb[r][e] = load_scale<kBf16>(args.s_b, tok, tok < args.rowsB);
-                        }
-                    uint32_t pk[2][8];  // [half][column group r * 2 + channel block]
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
+                for (int cc = 0; cc < kCpg; ++cc) {
+                    const int c = 32 * grp + 64 * cc;
+                    if (c < args.bn) {
+                        // token scales first: their loads overlap the TMEM reads
+                        float sb[4][2];
 #pragma unroll
                         for (int r = 0; r < 4; ++r)
 #pragma unroll
                             for (int e = 0; e < 2; ++e) {
-                                float y2[2];
-#pragma unroll
-                                for (int k = 0; k < 2; ++k) {
-                                    const uint32_t bits = v[h][4 * r + 2 * e + k];
-                                    const float accv =
-                                        kInt8 ? __int2float_rn(static_cast<int32_t>(bits))
-                                              : __uint_as_float(bits);
-                                    y2[k] = __fmul_rn(__fmul_rn(accv, sb[r][k]), sa2[h][e]);
-                                }
-                                const __nv_bfloat162 b2 = __floats2bfloat162_rn(y2[0], y2[1]);
-                                pk[h][2 * r + e] = *reinterpret_cast<const uint32_t*>(&b2);
+                                const int tok = b0 + c + 8 * r + 2 * tm + e;
+                                sb[r][e] = load_scale<kBf16>(args.s_b, tok, tok < args.rowsB);
                             }
-                    uint8_t* sy = stage_y + (chunk_iter & 1) * C::kEpiBytes;
-                    if (issuer) bulk_wait_read<1>();  // the stores of two chunks ago have read it
-                    named_bar_sync(1, 128);
-                    const uint32_t sy_u32 = smem_u32(sy);
+                        uint32_t v[2][16];
+                        tmem_ld_16x256b_x4(t_row + c, v[0]);
+                        tmem_ld_16x256b_x4(t_row + (16u << 16) + c, v[1]);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int h = 0; h < 2; ++h)
+                        for (int h = 0; h < 2; ++h)
 #pragma unroll
-                        for (int rp = 0; rp < 2; ++rp) {
-                            // matrices: (r = 2rp, e = 0), (2rp, 1), (2rp+1, 0), (2rp+1, 1)
-                            const int r = 2 * rp + (mi >> 1);
-                            const int e = mi & 1;
-                            const int tok = 8 * r + mj;                 // row of the chunk
-                            const int ch = q * 32 + 16 * h + 8 * e;     // 8-channel block
-                            const int half = ch >> 6;
-                            const int blk = (ch & 63) >> 3;
-                            const uint32_t addr = sy_u32 + half * (32 * 128) + tok * 128 +
-                                                  ((blk ^ (tok & 7)) << 4);
-                            stmatrix_x4_trans(addr, pk[h][4 * rp + 0], pk[h][4 * rp + 1],
-                                              pk[h][4 * rp + 2], pk[h][4 * rp + 3]);
-                        }
-                    fence_async_shared();
-                    named_bar_sync(1, 128);
-                    if (issuer) {
-                        const uint64_t stream = l2_policy_evict_first();
-                        tma_store_2d_hint(&tm_y, sy, a_cta0, b0 + c, stream);
-                        tma_store_2d_hint(&tm_y, sy + 32 * 128, a_cta0 + 64, b0 + c, stream);
-                        bulk_commit_group();
+                            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                                for (int e = 0; e < 2; ++e) {
+                                    float y2[2];
+#pragma unroll
+                                    for (int k = 0; k < 2; ++k) {
+                                        const uint32_t bits = v[h][4 * r + 2 * e + k];
+                                        const float accv =
+                                            kInt8 ? __int2float_rn(static_cast<int32_t>(bits))
+                                                  : __uint_as_float(bits);
+                                        y2[k] = __fmul_rn(__fmul_rn(accv, sb[r][k]), sa2[h][e]);
+                                    }
+                                    const __nv_bfloat162 b2 = __floats2bfloat162_rn(y2[0], y2[1]);
+                                    pk[cc][h][2 * r + e] = *reinterpret_cast<const uint32_t*>(&b2);
+                                }
                     }
-                    ++chunk_iter;
+                }
+                // 2) this group's part of the accumulator is read: release it
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if constexpr (kPair == 2)
+                        mbar_arrive_cluster(acc_empty_leader + acc * sizeof(uint64_t));
+                    else
+                        mbar_arrive(&acc_empty[acc]);
+                }
+                // 3) stage and store the chunks while the next tile's MMAs run
+#pragma unroll
+                for (int cc = 0; cc < kCpg; ++cc) {
+                    const int c = 32 * grp + 64 * cc;
+                    if (c < args.bn) {
+                        if (issuer) bulk_wait_read<0>();  // the group's last stores have read it
+                        named_bar_sync(grp_bar, 128);
+                        const uint32_t sy_u32 = smem_u32(sy);
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+#pragma unroll
+                            for (int rp = 0; rp < 2; ++rp) {
+                                // matrices: (r = 2rp, e = 0), (2rp, 1), (2rp+1, 0), (2rp+1, 1)
+                                const int r = 2 * rp + (mi >> 1);
+                                const int e = mi & 1;
+                                const int tok = 8 * r + mj;              // row of the chunk
+                                const int ch = q * 32 + 16 * h + 8 * e;  // 8-channel block
+                                const int half = ch >> 6;
+                                const int blk = (ch & 63) >> 3;
+                                const uint32_t addr = sy_u32 + half * (32 * 128) + tok * 128 +
+                                                      ((blk ^ (tok & 7)) << 4);
+                                stmatrix_x4_trans(addr, pk[cc][h][4 * rp + 0],
+                                                  pk[cc][h][4 * rp + 1], pk[cc][h][4 * rp + 2],
+                                                  pk[cc][h][4 * rp + 3]);
+                            }
+                        fence_async_shared();
+                        named_bar_sync(grp_bar, 128);
+                        if (issuer) {
+                            const uint64_t stream = l2_policy_evict_first();
+                            tma_store_2d_hint(&tm_y, sy, a_cta0, b0 + c, stream);
+                            tma_store_2d_hint(&tm_y, sy + 32 * 128, a_cta0 + 64, b0 + c, stream);
+                            bulk_commit_group();
+                        }
+                    }
                 }
                 continue;
             }
-            for (int c = 0; c < args.bn; c += 32) {
+            for (int c = 32 * grp; c < args.bn; c += 64) {
+                const int bc = b0 + c + lane;  // this lane's B row of the chunk
+                const float sb_lane = load_scale<kBf16>(args.s_b, bc, bc < args.rowsB);
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(t_row + c, r);
                 tmem_ld_wait();
-                if (c + 32 >= args.bn) {  // last read of this accumulator: release it
+                if (c + 64 >= args.bn) {  // this group's last read: release its part
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) {
@@ -612,12 +684,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             mbar_arrive(&acc_empty[acc]);
                     }
                 }
-                const int bc = b0 + c + lane;  // this lane's B row of the chunk
-                const float sb_lane = load_scale<kBf16>(args.s_b, bc, bc < args.rowsB);
                 if (args.tma_store) {
-                    uint8_t* sy = stage_y + (chunk_iter & 1) * C::kEpiBytes;
-                    if (issuer) bulk_wait_read<1>();  // the store of two chunks ago has read it
-                    named_bar_sync(1, 128);
+                    if (issuer) bulk_wait_read<0>();  // the group's last store has read it
+                    named_bar_sync(grp_bar, 128);
                     if (args.a_is_w) {
                         // box [32 B rows][128 A rows]: element (u, lane_row)
 #pragma unroll
@@ -653,7 +722,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                                 packed[4 * w + 2], packed[4 * w + 3]);
                     }
                     fence_async_shared();
-                    named_bar_sync(1, 128);
+                    named_bar_sync(grp_bar, 128);
                     if (issuer) {
                         const uint64_t stream = l2_policy_evict_first();
                         if (args.a_is_w)
@@ -662,7 +731,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             tma_store_2d_hint(&tm_y, sy, b0 + c, a_cta0, stream);
                         bulk_commit_group();
                     }
-                    ++chunk_iter;
                 } else {
 #pragma unroll
                     for (int u = 0; u < 32; ++u) {

@@ -26,6 +26,7 @@
 
 namespace ss {
 
+constexpr int kSplitKThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2-5 epilogue
 constexpr int kSkBn = 64;  // tokens (B rows) at most
 
 template <bool kSparse, int kEb>
@@ -61,7 +62,7 @@ struct SplitKCfg {
 // args.k_stages: stages of the whole K; args.bn: B rows (a multiple of 32,
 // <= kSkBn, covering every B row); args.a_is_w must be 1.
 template <bool kSparse, int kQ, bool kOutBf16>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kSplitKThreads, 1)
     gemm_splitk_kernel(const __grid_constant__ CUtensorMap tm_a,
                        const __grid_constant__ CUtensorMap tm_b,
                        const __grid_constant__ CUtensorMap tm_e, const GemmArgs args) {

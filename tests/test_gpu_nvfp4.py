@@ -120,6 +120,25 @@ def test_sparse_gemm_nvfp4_many_tiles(M, N, K, pat, nrows):
     assert_y_matches(Y[rows], Y_ref, "fp8", True)
 
 
+# Sparse CTA-pair tiles (more than 128 weight rows and K_lp > 2048): M = 256
+# MMAs over 256-token B tiles with two scale tiles each, ragged in M, N and K.
+@pytest.mark.parametrize("M,N,K,pat", [(700, 520, 4096, "2:4"), (300, 300, 3000, "6:8"),
+                                       (2100, 1000, 2560, "4:6"), (33, 4096, 4096, "8:10")])
+def test_sparse_gemm_nvfp4_pair_tiles(M, N, K, pat):
+    Wv, Wm, Ws, g_w, Xv, Xs, g_x, K_lp = _sparse_operands(M, N, K, pat)
+    assert K_lp > 2048 and N > 128
+    rows = synth.sample_rows(M, seed=6, middle=200) if M > 600 else None
+    Y_ref = oracle.sparse_gemm_nvfp4(Wv, Wm, Ws, g_w, Xv, Xs, g_x, M, N, K_lp, oracle.OUT_BF16,
+                                     m_idx=rows)
+    packed = (dev(Wv), dev(oracle.meta_to_tiles(Wm, K_lp // 2)),
+              dev(oracle.scales_to_tiles(Ws, K_lp, 32)),
+              dev(np.array([g_w, 0, 0, 0], dtype=np.float32)))
+    act = (dev(Xv), dev(oracle.scales_to_tiles(Xs, K_lp, 32)), dev(g_x))
+    Y = host(ss.sparse_gemm_nvfp4(packed, act, M, N))
+    assert ss.ss_get_device_status() == ss.SS_OK
+    assert_y_matches(Y if rows is None else Y[rows], Y_ref, "fp8", True)
+
+
 @pytest.mark.parametrize("M,N,K", [(16, 64, 64), (1, 130, 300), (300, 257, 1000),
                                    (1000, 2000, 768)])
 def test_dense_gemm_nvfp4(M, N, K):
