@@ -59,7 +59,9 @@ struct GemmCfg {
     // 128 (4 MMAs of K=32) and sparse 256 (4 MMAs of K=64); for bf16 (kEb = 2
     // bytes) half of that, 4 MMAs of K=16 / K=32.  Either way an A row holds
     // 128 bytes of the stage (128B swizzle) and each MMA reads 32 bytes of an
-    // A row and 32 (dense) or 64 (sparse) bytes of a B row.
+    // A row and 32 (dense) or 64 (sparse) bytes of a B row.  (Stages of half
+    // the K, with 64-byte A rows, measured slower: twice the handshakes per
+    // byte cost more than the deeper ring gains.)
     static constexpr int kStageK = (kSparse ? 256 : 128) / kEb;
     static constexpr int kMmaK = (kSparse ? 64 : 32) / kEb;
     static constexpr int kMmaPerStage = kStageK / kMmaK;
@@ -108,8 +110,8 @@ struct GemmCfg {
 // Stage layout of the block-scaled FP4 GEMM: per stage 4 MMAs (sparse: K =
 // 128 lifted each, dense: K = 64), A 128 rows x 128 B, this CTA's B rows x
 // 256 B (sparse) / 128 B (dense), sparse metadata 2 x 2 KB, the scale factors
-// of A (4 x 512 B) and those of the whole B tile (4 x 512 B per 128-row scale
-// tile).
+// of A (512 B per MMA) and those of the whole B tile (512 B per MMA and
+// 128-row scale tile).
 //   single SM: MMA M = 128, N = 128; two 128-column accumulators in tensor
 //     memory (the epilogue drains one while the next tile fills the other).
 //   CTA pair:  MMA M = 256, N = 256 (128 B rows per CTA, two scale tiles);
@@ -124,7 +126,7 @@ template <bool kSparse, int kPair = 1>
 struct Fp4Cfg {
     static constexpr int kStageK = kSparse ? 512 : 256;
     static constexpr int kMmaK = kSparse ? 128 : 64;
-    static constexpr int kMmaPerStage = 4;
+    static constexpr int kMmaPerStage = kStageK / kMmaK;
     static constexpr int kARowBytes = 128;
     static constexpr int kABytes = kTileA * kARowBytes;
     static constexpr int kBAtoms = kSparse ? 2 : 1;
@@ -136,8 +138,9 @@ struct Fp4Cfg {
     static constexpr int kBBytes = kBAtoms * kBAtomBytes;
     static constexpr int kEChunks = kSparse ? 2 : 0;
     static constexpr int kEBytes = kEChunks * kTileA * 16;
-    static constexpr int kSfaBytes = 4 * 512;              // A scales of a stage
-    static constexpr int kSfbBytes = kSfbTiles * 4 * 512;  // B scales of a stage
+    static constexpr int kSfaBytes = kMmaPerStage * 512;   // A scales of a stage
+    static constexpr int kSfbTileBytes = kMmaPerStage * 512;  // per 128-row scale tile
+    static constexpr int kSfbBytes = kSfbTiles * kSfbTileBytes;  // B scales of a stage
     static constexpr int kSfStageBytes = kSfaBytes + kSfbBytes;
     static constexpr int kBOffset = kABytes;
     static constexpr int kEOffset = kBOffset + kBBytes;
@@ -330,14 +333,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                                   ((a0 >> 7) * args.e_chunks + kb * C::kEChunks + u) * 16,
                                                   keep);
                         if constexpr (kFp4) {  // this CTA's A scales, the whole B tile's scales
-                            tma_load_2d_pair_hint(st + C::kSfaOffset, &tm_sfa, fb, 0,
-                                                  ((a0 >> 7) * args.sf_k + kb * 4) * 4, keep);
+                            tma_load_2d_pair_hint(
+                                st + C::kSfaOffset, &tm_sfa, fb, 0,
+                                ((a0 >> 7) * args.sf_k + kb * C::kMmaPerStage) * 4, keep);
                             const int sfb_tile = (t / nA) * args.bn >> 7;
 #pragma unroll
                             for (int u = 0; u < C::kSfbTiles; ++u)  // past the last: zero fill
-                                tma_load_2d_pair_hint(st + C::kSfbOffset + 2048 * u, &tm_sfb, fb, 0,
-                                                      ((sfb_tile + u) * args.sf_k + kb * 4) * 4,
-                                                      keep);
+                                tma_load_2d_pair_hint(
+                                    st + C::kSfbOffset + C::kSfbTileBytes * u, &tm_sfb, fb, 0,
+                                    ((sfb_tile + u) * args.sf_k + kb * C::kMmaPerStage) * 4, keep);
                         }
                     } else {
                         mbar_arrive_expect_tx(&full[s], tx);
@@ -353,11 +357,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         if constexpr (kFp4) {
                             // 4 MMAs' scales of A and of B: 2 KB each, as 16 rows of 128 B
                             tma_load_2d(st + C::kSfaOffset, &tm_sfa, &full[s], 0,
-                                        ((a0 >> 7) * args.sf_k + kb * 4) * 4);
+                                        ((a0 >> 7) * args.sf_k + kb * C::kMmaPerStage) * 4);
 #pragma unroll
                             for (int u = 0; u < C::kSfbTiles; ++u)
-                                tma_load_2d(st + C::kSfbOffset + 2048 * u, &tm_sfb, &full[s], 0,
-                                            (((b0 >> 7) + u) * args.sf_k + kb * 4) * 4);
+                                tma_load_2d(st + C::kSfbOffset + C::kSfbTileBytes * u, &tm_sfb,
+                                            &full[s], 0,
+                                            (((b0 >> 7) + u) * args.sf_k + kb * C::kMmaPerStage) * 4);
                         }
                     }
                 }
@@ -423,7 +428,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             const uint32_t sf_tmem = tmem_base + C::kSfCol + C::kSfSlotCols * s;
                             const uint32_t sfb_tmem = sf_tmem + C::kSfaCols;
 #pragma unroll
-                            for (int t = 0; t < 4; ++t) {
+                            for (int t = 0; t < C::kMmaPerStage; ++t) {
                                 tc_cp_32x128b_warpx4_g<kPair>(
                                     sf_tmem + 4 * t, sf_desc0 + soff + ((C::kSfaOffset + 512 * t) >> 4));
 #pragma unroll
@@ -431,7 +436,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                     tc_cp_32x128b_warpx4_g<kPair>(
                                         sfb_tmem + 4 * (C::kSfbTiles * t + u),
                                         sf_desc0 + soff +
-                                            ((C::kSfbOffset + 2048 * u + 512 * t) >> 4));
+                                            ((C::kSfbOffset + C::kSfbTileBytes * u + 512 * t) >> 4));
                             }
                             if constexpr (kSparse) {
 #pragma unroll
@@ -581,88 +586,102 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 // this thread's stmatrix row: matrix mi, row mj
                 const int mi = lane >> 3, mj = lane & 7;
-                // 1) every chunk of this group into registers as packed bf16
-                //    ([chunk][half][column group r * 2 + channel block])
+                // Chunks go through registers in batches: with two accumulators
+                // one chunk at a time (its stores overlap the next chunk's
+                // reads); with one accumulator the whole group's part is read
+                // first, so that it is released before any store is waited for.
                 constexpr int kCpg = (C::kBnMax + 63) / 64;  // chunks per group, at most
-                uint32_t pk[kCpg][2][8];
+                constexpr int kBatch = C::kAccBufs == 1 ? kCpg : 1;
 #pragma unroll
-                for (int cc = 0; cc < kCpg; ++cc) {
-                    const int c = 32 * grp + 64 * cc;
-                    if (c < args.bn) {
-                        // token scales first: their loads overlap the TMEM reads
-                        float sb[4][2];
+                for (int cb = 0; cb < kCpg; cb += kBatch) {
+                    // 1) the batch's chunks into registers as packed bf16
+                    //    ([chunk][half][column group r * 2 + channel block])
+                    uint32_t pk[kBatch][2][8];
 #pragma unroll
-                        for (int r = 0; r < 4; ++r)
-#pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const int tok = b0 + c + 8 * r + 2 * tm + e;
-                                sb[r][e] = load_scale<kBf16>(args.s_b, tok, tok < args.rowsB);
-                            }
-                        uint32_t v[2][16];
-                        tmem_ld_16x256b_x4(t_row + c, v[0]);
-                        tmem_ld_16x256b_x4(t_row + (16u << 16) + c, v[1]);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int h = 0; h < 2; ++h)
+                    for (int cc = 0; cc < kBatch; ++cc) {
+                        const int c = 32 * grp + 64 * (cb + cc);
+                        if (c < args.bn) {
+                            // token scales first: their loads overlap the TMEM reads
+                            float sb[4][2];
 #pragma unroll
                             for (int r = 0; r < 4; ++r)
 #pragma unroll
                                 for (int e = 0; e < 2; ++e) {
-                                    float y2[2];
-#pragma unroll
-                                    for (int k = 0; k < 2; ++k) {
-                                        const uint32_t bits = v[h][4 * r + 2 * e + k];
-                                        const float accv =
-                                            kInt8 ? __int2float_rn(static_cast<int32_t>(bits))
-                                                  : __uint_as_float(bits);
-                                        y2[k] = __fmul_rn(__fmul_rn(accv, sb[r][k]), sa2[h][e]);
-                                    }
-                                    const __nv_bfloat162 b2 = __floats2bfloat162_rn(y2[0], y2[1]);
-                                    pk[cc][h][2 * r + e] = *reinterpret_cast<const uint32_t*>(&b2);
+                                    const int tok = b0 + c + 8 * r + 2 * tm + e;
+                                    sb[r][e] = load_scale<kBf16>(args.s_b, tok, tok < args.rowsB);
                                 }
+                            uint32_t v[2][16];
+                            tmem_ld_16x256b_x4(t_row + c, v[0]);
+                            tmem_ld_16x256b_x4(t_row + (16u << 16) + c, v[1]);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                                    for (int e = 0; e < 2; ++e) {
+                                        float y2[2];
+#pragma unroll
+                                        for (int k = 0; k < 2; ++k) {
+                                            const uint32_t bits = v[h][4 * r + 2 * e + k];
+                                            const float accv =
+                                                kInt8 ? __int2float_rn(static_cast<int32_t>(bits))
+                                                      : __uint_as_float(bits);
+                                            y2[k] = __fmul_rn(__fmul_rn(accv, sb[r][k]), sa2[h][e]);
+                                        }
+                                        const __nv_bfloat162 b2 =
+                                            __floats2bfloat162_rn(y2[0], y2[1]);
+                                        pk[cc][h][2 * r + e] =
+                                            *reinterpret_cast<const uint32_t*>(&b2);
+                                    }
+                        }
                     }
-                }
-                // 2) this group's part of the accumulator is read: release it
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    if constexpr (kPair == 2)
-                        mbar_arrive_cluster(acc_empty_leader + acc * sizeof(uint64_t));
-                    else
-                        mbar_arrive(&acc_empty[acc]);
-                }
-                // 3) stage and store the chunks while the next tile's MMAs run
+                    // 2) after the group's last read of the accumulator: release its part
+                    if (32 * grp + 64 * (cb + kBatch) >= args.bn &&
+                        32 * grp + 64 * cb < args.bn) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) {
+                            if constexpr (kPair == 2)
+                                mbar_arrive_cluster(acc_empty_leader + acc * sizeof(uint64_t));
+                            else
+                                mbar_arrive(&acc_empty[acc]);
+                        }
+                    }
+                    // 3) stage and store the batch
 #pragma unroll
-                for (int cc = 0; cc < kCpg; ++cc) {
-                    const int c = 32 * grp + 64 * cc;
-                    if (c < args.bn) {
-                        if (issuer) bulk_wait_read<0>();  // the group's last stores have read it
-                        named_bar_sync(grp_bar, 128);
-                        const uint32_t sy_u32 = smem_u32(sy);
+                    for (int cc = 0; cc < kBatch; ++cc) {
+                        const int c = 32 * grp + 64 * (cb + cc);
+                        if (c < args.bn) {
+                            if (issuer) bulk_wait_read<0>();  // the group's last stores have read it
+                            named_bar_sync(grp_bar, 128);
+                            const uint32_t sy_u32 = smem_u32(sy);
 #pragma unroll
-                        for (int h = 0; h < 2; ++h)
+                            for (int h = 0; h < 2; ++h)
 #pragma unroll
-                            for (int rp = 0; rp < 2; ++rp) {
-                                // matrices: (r = 2rp, e = 0), (2rp, 1), (2rp+1, 0), (2rp+1, 1)
-                                const int r = 2 * rp + (mi >> 1);
-                                const int e = mi & 1;
-                                const int tok = 8 * r + mj;              // row of the chunk
-                                const int ch = q * 32 + 16 * h + 8 * e;  // 8-channel block
-                                const int half = ch >> 6;
-                                const int blk = (ch & 63) >> 3;
-                                const uint32_t addr = sy_u32 + half * (32 * 128) + tok * 128 +
-                                                      ((blk ^ (tok & 7)) << 4);
-                                stmatrix_x4_trans(addr, pk[cc][h][4 * rp + 0],
-                                                  pk[cc][h][4 * rp + 1], pk[cc][h][4 * rp + 2],
-                                                  pk[cc][h][4 * rp + 3]);
+                                for (int rp = 0; rp < 2; ++rp) {
+                                    // matrices: (r = 2rp, e = 0), (2rp, 1), (2rp+1, 0), (2rp+1, 1)
+                                    const int r = 2 * rp + (mi >> 1);
+                                    const int e = mi & 1;
+                                    const int tok = 8 * r + mj;              // row of the chunk
+                                    const int ch = q * 32 + 16 * h + 8 * e;  // 8-channel block
+                                    const int half = ch >> 6;
+                                    const int blk = (ch & 63) >> 3;
+                                    const uint32_t addr = sy_u32 + half * (32 * 128) + tok * 128 +
+                                                          ((blk ^ (tok & 7)) << 4);
+                                    stmatrix_x4_trans(addr, pk[cc][h][4 * rp + 0],
+                                                      pk[cc][h][4 * rp + 1], pk[cc][h][4 * rp + 2],
+                                                      pk[cc][h][4 * rp + 3]);
+                                }
+                            fence_async_shared();
+                            named_bar_sync(grp_bar, 128);
+                            if (issuer) {
+                                const uint64_t stream = l2_policy_evict_first();
+                                tma_store_2d_hint(&tm_y, sy, a_cta0, b0 + c, stream);
+                                tma_store_2d_hint(&tm_y, sy + 32 * 128, a_cta0 + 64, b0 + c,
+                                                  stream);
+                                bulk_commit_group();
                             }
-                        fence_async_shared();
-                        named_bar_sync(grp_bar, 128);
-                        if (issuer) {
-                            const uint64_t stream = l2_policy_evict_first();
-                            tma_store_2d_hint(&tm_y, sy, a_cta0, b0 + c, stream);
-                            tma_store_2d_hint(&tm_y, sy + 32 * 128, a_cta0 + 64, b0 + c, stream);
-                            bulk_commit_group();
                         }
                     }
                 }
