@@ -232,8 +232,8 @@ ss_status ss_quant_lift_act_nvfp4(const void *X, ss_in_dtype in_dtype, int64_t M
                                   ss_pattern p, int32_t block, void *Xv, void *Xs, float *g_x,
                                   ss_stream_t stream);
 
-/* Sparse NVFP4 GEMM (tcgen05.mma.sp kind::mxf4nvf4, block-scaled, single SM
- * per MMA): Y[m, n] = ((float)acc[m, n] * g_x[m]) * g_w[0], acc the fp32
+/* Sparse NVFP4 GEMM (tcgen05.mma.sp kind::mxf4nvf4, block-scaled; one SM or a
+ * CTA pair per MMA): Y[m, n] = ((float)acc[m, n] * g_x[m]) * g_w[0], acc the fp32
  * tensor-core sum of (codes x local scales) products; A = the compressed
  * weight, B = the lifted activation (block 32).  K_lp a positive multiple
  * of 256. */
