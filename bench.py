@@ -51,9 +51,12 @@ IDEAL = {"2:4": 2.0, "4:6": 1.5, "6:8": 4.0 / 3.0, "8:10": 1.25}
 
 # DRAM bytes per launch of the dominant kernel (dram__bytes_read.sum +
 # dram__bytes_write.sum of one sparse-GEMM launch) from one ncu capture of the
-# same kernel build; absent when not captured for this build.
+# same kernel build; absent when not captured for this build.  Keyed by
+# (workload, M, pattern, qdtype) as run.
 TRAFFIC = {
-    ("llama_q_2of4_int8", 8192): 44.21e6 + 16.07e6,
+    ("llama_q_2of4_int8", 8192, "2:4", "int8"): 44.21e6 + 16.07e6,
+    ("llama_q_2of4_bf16", 8192, "2:4", "bf16"): 86.13e6 + 38.76e6,
+    ("llama_gateup_4of8_nvfp4", 8192, "2:4", "nvfp4"): 38.83e6 + 178.86e6,
 }
 
 
@@ -611,7 +614,8 @@ def main():
     n = dist.world
     value = n * path.dense_equiv_ops() / (r["t_step_ms"] * 1e-3) / 1e12
     line = base_line(args, args.workload, args.m, n)
-    tr = TRAFFIC.get((args.workload, args.m))
+    wl = synth.WORKLOADS[args.workload]
+    tr = TRAFFIC.get((args.workload, args.m, wl["pattern"], wl["qdtype"]))
     line.update({
         "value": value, "ms_per_step": r["t_step_ms"],
         "dtype": path.q,
