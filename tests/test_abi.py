@@ -129,6 +129,70 @@ def test_argument_errors_return_before_any_launch(L):
         == ss.SS_ERR_UNSUPPORTED
 
 
+@pytest.mark.parametrize("pat", ["dense", "2:4", "4:6", "6:8", "8:10"])
+def test_fp4_shape_matches_oracle(pat):
+    for K in [1, 2, 7, 64, 300, 1000, 4096, 4097, 14336]:
+        assert ss.ss_fp4_shape(pat, K) == oracle.fp4_shape(pat, K)
+
+
+def test_fp4_scale_bytes(L):
+    """Tile-major scales: 128-row tiles, one byte per block of 16 or 32."""
+    assert ss.ss_fp4_scale_bytes(1, 256, 16) == 128 * 16
+    assert ss.ss_fp4_scale_bytes(129, 512, 32) == 256 * 16
+    assert ss.ss_fp4_scale_bytes(300, 4096, 32) == 384 * 128
+    for rows, K_lp, block in [(0, 256, 16), (1, 100, 16), (1, 128, 16), (1, 256, 8),
+                              (-1, 256, 32)]:
+        assert ss.ss_fp4_scale_bytes(rows, K_lp, block) == 0
+
+
+def test_nvfp4_argument_errors_return_before_any_launch(L):
+    """The NVFP4 calls validate shapes, pointers, dtypes and alignment before
+    the device is touched."""
+    vp = ctypes.c_void_p
+    good = vp(0x10000)          # never dereferenced: every call below fails first
+    odd = vp(0x10008)
+    pat = ss.ss_pattern(6, 8)
+    dense = ss.ss_pattern(0, 0)
+    # weight: Wm required unless dense, bad dtype, bad size, misaligned
+    assert L.ss_compress_weight_nvfp4(good, 1, 64, 64, pat, good, None, good, good, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_compress_weight_nvfp4(good, 2, 64, 64, pat, good, good, good, good, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_compress_weight_nvfp4(good, 1, 0, 64, dense, good, None, good, good, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_compress_weight_nvfp4(odd, 1, 64, 64, pat, good, good, good, good, None) \
+        == ss.SS_ERR_ALIGNMENT
+    assert L.ss_compress_weight_nvfp4(good, 1, 64, 64, ss.ss_pattern(3, 4), good, good, good,
+                                      good, None) == ss.SS_ERR_INVALID_ARG
+    # activation: block 16 or 32 only, NULL outputs, misaligned
+    assert L.ss_quant_lift_act_nvfp4(good, 1, 16, 64, pat, 8, good, good, good, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_quant_lift_act_nvfp4(good, 1, 16, 64, pat, 32, good, None, good, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_quant_lift_act_nvfp4(good, 1, 0, 64, pat, 32, good, good, good, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_quant_lift_act_nvfp4(good, 1, 16, 64, pat, 32, good, good, odd, None) \
+        == ss.SS_ERR_ALIGNMENT
+    # GEMMs: K_lp a positive multiple of 256, metadata required for the sparse
+    # one, out dtype, alignment
+    assert L.ss_sparse_gemm_nvfp4(good, good, good, good, good, good, good, 16, 64, 128, good, 1,
+                                  None) == ss.SS_ERR_INVALID_ARG
+    assert L.ss_sparse_gemm_nvfp4(good, None, good, good, good, good, good, 16, 64, 256, good, 1,
+                                  None) == ss.SS_ERR_INVALID_ARG
+    assert L.ss_sparse_gemm_nvfp4(good, good, good, good, good, good, good, 0, 64, 256, good, 1,
+                                  None) == ss.SS_ERR_INVALID_ARG
+    assert L.ss_sparse_gemm_nvfp4(good, good, good, good, good, good, good, 16, 64, 256, good, 2,
+                                  None) == ss.SS_ERR_INVALID_ARG
+    assert L.ss_sparse_gemm_nvfp4(good, good, good, good, odd, good, good, 16, 64, 256, good, 1,
+                                  None) == ss.SS_ERR_ALIGNMENT
+    assert L.ss_dense_gemm_nvfp4(good, good, good, good, good, good, 16, 64, 384, good, 1, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_dense_gemm_nvfp4(good, good, None, good, good, good, 16, 64, 256, good, 1, None) \
+        == ss.SS_ERR_INVALID_ARG
+    assert L.ss_dense_gemm_nvfp4(good, good, good, good, good, good, 16, 64, 256, odd, 1, None) \
+        == ss.SS_ERR_ALIGNMENT
+
+
 @pytest.mark.parametrize("rows,K_lp", [(1, 128), (130, 384), (256, 1024), (300, 128)])
 def test_metadata_storage_layout(L, rows, K_lp):
     """Tile-major selector storage: every byte sits where ss.h's formula puts
