@@ -58,7 +58,8 @@ def lib() -> ctypes.CDLL:
             "ssref_fp4_shape": [i32, i32, i64, p, p],
             "ssref_prune_pairs": [p, i64, i64, i32, i32, p],
             "ssref_compress_weight_nvfp4": [p, i64, i64, i32, i32, p, p, p, p],
-            "ssref_quant_nvfp4": [p, i64, i64, i32, i32, i32, i32, p, p, p],
+            "ssref_quant_nvfp4": [p, i64, i64, i32, i32, i32, p, p, p],
+            "ssref_nvfp4_act_page": [p, i64, i64, i32, i32, p, p],
             "ssref_decode_sparse_nvfp4": [p, p, p, i64, i64, p],
             "ssref_decode_dense_nvfp4": [p, p, i64, i64, i32, p],
             "ssref_matmul_nvfp4": [p, p, p, p, i64, i64, i64, p, i64, i32, p],
@@ -499,19 +500,35 @@ def compress_weight_nvfp4(W, p: str):
     return Wv, Wm, Ws, float(g[0])
 
 
-def quant_nvfp4(X, p: str, block: int, per_row: bool = True):
-    """Dense NVFP4 rows (lifted on pairs for a pattern) -> (Xv [rows, K_lp/2]
-    bytes, Xs [rows, K_lp/block] UE4M3, g [rows])."""
+def quant_nvfp4(X, p: str, block: int):
+    """Dense NVFP4 matrix (lifted on pairs for a pattern) with one global
+    scale for the whole tensor -> (Xv [rows, K_lp/2] bytes, Xs [rows,
+    K_lp/block] UE4M3, g [1])."""
     X = _f32(X)
     rows, K = X.shape
     keep, group = pattern(p)
     _, K_lp = fp4_shape(p, K)
     Xv = np.zeros((rows, K_lp // 2), dtype=np.uint8)
     Xs = np.zeros((rows, K_lp // block), dtype=np.uint8)
-    g = np.zeros(rows, dtype=np.float32)
-    _check(lib().ssref_quant_nvfp4(_ptr(X), rows, K, keep, group, block, 1 if per_row else 0,
-                                   _ptr(Xv), _ptr(Xs), _ptr(g)), "quant_nvfp4")
+    g = np.zeros(1, dtype=np.float32)
+    _check(lib().ssref_quant_nvfp4(_ptr(X), rows, K, keep, group, block, _ptr(Xv), _ptr(Xs),
+                                   _ptr(g)), "quant_nvfp4")
     return Xv, Xs, g
+
+
+def nvfp4_act_page(X, p: str):
+    """The activation as the NVFP4 definition has it (16-element groups along
+    the original K, one global scale), decoded without the global scale and
+    lifted to K_lp -> (Xlift [rows, K_lp] float64, g [1])."""
+    X = _f32(X)
+    rows, K = X.shape
+    keep, group = pattern(p)
+    _, K_lp = fp4_shape(p, K)
+    Xl = np.zeros((rows, K_lp), dtype=np.float64)
+    g = np.zeros(1, dtype=np.float32)
+    _check(lib().ssref_nvfp4_act_page(_ptr(X), rows, K, keep, group, _ptr(Xl), _ptr(g)),
+           "nvfp4_act_page")
+    return Xl, g
 
 
 def decode_sparse_nvfp4(Av, Am, As, K_lp: int) -> np.ndarray:
@@ -534,12 +551,13 @@ def decode_dense_nvfp4(Xv, Xs, K_lp: int, block: int) -> np.ndarray:
 
 
 def matmul_nvfp4(Xd, g_x, Wd, g_w, out_dtype: int, m_idx=None):
-    """Y = ((float)(Xd . Wd^T) * g_x[m]) * g_w[n] over decoded operands."""
+    """Y = ((float)(Xd . Wd^T) * g_x) * g_w[n] over decoded operands (g_x one
+    value for the tensor, or one per row)."""
     Xd = np.ascontiguousarray(Xd, dtype=np.float64)
     Wd = np.ascontiguousarray(Wd, dtype=np.float64)
-    g_x = np.ascontiguousarray(g_x, dtype=np.float32)
-    g_w = np.ascontiguousarray(g_w, dtype=np.float32)
     M, K = Xd.shape
+    g_x = np.ascontiguousarray(np.broadcast_to(np.asarray(g_x, dtype=np.float32).reshape(-1), (M,)))
+    g_w = np.ascontiguousarray(g_w, dtype=np.float32)
     N = Wd.shape[0]
     m_idx, R = _rows(m_idx, M)
     Y = _out(R, N, out_dtype)
@@ -555,6 +573,16 @@ def sparse_gemm_nvfp4(Wv, Wm, Ws, g_w: float, Xv, Xs, g_x, M: int, N: int, K_lp:
     Wd = decode_sparse_nvfp4(Wv, Wm, Ws, K_lp)
     Xd = decode_dense_nvfp4(Xv, Xs, K_lp, 32)
     return matmul_nvfp4(Xd, g_x, Wd, np.full(N, g_w, dtype=np.float32), out_dtype, m_idx)
+
+
+def sparse_gemm_nvfp4_page(Wv, Wm, Ws, g_w: float, X, p: str, out_dtype: int, m_idx=None):
+    """The same product with the activation quantised as the NVFP4 definition
+    has it (nvfp4_act_page: 16-element groups along the original K)."""
+    N = Wv.shape[0]
+    K_lp = Wv.shape[1] * 4
+    Xl, g_x = nvfp4_act_page(X, p)
+    Wd = decode_sparse_nvfp4(Wv, Wm, Ws, K_lp)
+    return matmul_nvfp4(Xl, g_x, Wd, np.full(N, g_w, dtype=np.float32), out_dtype, m_idx)
 
 
 def dense_gemm_nvfp4(Xv, Xs, g_x, Wv, Ws, g_w, out_dtype: int, m_idx=None):

@@ -59,8 +59,10 @@
  *        g = amax / (6 * 448) in fp32; a block with amax a gets
  *        s = UE4M3(a / (6 g)), divisor d = s * g, inv = 1 / d (0 if d = 0)
  *        and codes E2M1(x * inv), every step one fp32 operation;
- *      - weights: one global scale per tensor; activations: one per token
- *        (no calibration set exists here, so it is taken from the row);
+ *      - one global scale per tensor, for weights and activations alike
+ *        ([LC] NVFP4 row); the page calibrates the activation's global scale
+ *        on a data set, and with none here it is taken dynamically from the
+ *        amax of the whole activation tensor of the call;
  *      - sparsity is on pairs of adjacent elements: a pattern keep:group
  *        counts pairs (2:4 is the hardware's pairwise 4:8), pairs are ranked
  *        by x0^2 + x1^2 (ties keep the lower pair) and slid as units, and a
@@ -69,7 +71,10 @@
  *      - block size: 16 stored values of a sparse operand (= 32 lifted
  *        elements), 32 lifted elements of the dense operand of a sparse
  *        product, 16 elements in a dense product -- the sparse FP4 tensor-core
- *        instruction applies one scale per 32 lifted K to both operands.
+ *        instruction applies one scale per 32 lifted K to both operands.  The
+ *        page's own definition (16-element groups of the activation, along
+ *        its original K) is computed too, by ssref_nvfp4_act_page, so that
+ *        the tests can bound what the 32-element blocks cost.
  */
 #include <math.h>
 #include <stdint.h>
@@ -916,35 +921,39 @@ int ssref_compress_weight_nvfp4(const float *W, int64_t N, int64_t K, int keep, 
     return SSREF_OK;
 }
 
+/* Source element of lifted position k under the pair slide of a pattern
+ * with `group` pairs per group (window i of 4 pairs, element t of its 8):
+ * [OM] 3.2's window map, base = 2Nh * (i / (Nh - 1)) + 2 * (i % (Nh - 1)),
+ * applied to pairs.  -1 past the lifted length (zero padding). */
+static int64_t pair_lift_src(int64_t k, int group, int64_t K_lift) {
+    if (group == 0) return k;
+    if (k >= K_lift) return -1;
+    int64_t Nh = group / 2;
+    int64_t wi = k / 8, t = k % 8;
+    int64_t gi = wi / (Nh - 1), j = wi % (Nh - 1);
+    return 2 * (gi * group + 2 * j) + t;
+}
+
 /* Dense NVFP4 matrix (the comparator's operands, or the dense operand of a
  * sparse product): rows of K (lifted on pairs for a pattern), zero-padded to
- * K_lp, blocks of `block` elements, global scale per row (per_row) or one for
- * the whole matrix.  Xv [rows, K_lp/2] bytes, Xs [rows, K_lp/block], g[rows]. */
+ * K_lp, blocks of `block` lifted elements, ONE global scale for the whole
+ * matrix ([LC] NVFP4 row: a global scale per tensor), from the amax of all
+ * its elements.  Xv [rows, K_lp/2] bytes, Xs [rows, K_lp/block], g_out[0]. */
 int ssref_quant_nvfp4(const float *X, int64_t rows, int64_t K, int keep, int group, int block,
-                      int per_row, uint8_t *Xv, uint8_t *Xs, float *g_out) {
+                      uint8_t *Xv, uint8_t *Xs, float *g_out) {
     int64_t K_lift, K_lp;
     int st = ssref_fp4_shape(keep, group, K, &K_lift, &K_lp);
     if (st || (block != 16 && block != 32)) return SSREF_EINVAL;
-    int Nh = group / 2;
-    float amax_all = 0.0f;
-    for (int64_t i = 0; i < rows * K; i++) amax_all = fmaxf(amax_all, fabsf(X[i]));
+    float amax = 0.0f;
+    for (int64_t i = 0; i < rows * K; i++) amax = fmaxf(amax, fabsf(X[i]));
+    float g = ssref_nvfp4_global(amax);
+    g_out[0] = g;
     float *lifted = (float *)malloc((size_t)K_lp * sizeof(float));
     memset(Xv, 0, (size_t)(rows * K_lp / 2));
     for (int64_t r = 0; r < rows; r++) {
         const float *x = &X[r * K];
-        float amax = 0.0f;
-        for (int64_t k = 0; k < K; k++) amax = fmaxf(amax, fabsf(x[k]));
-        float g = ssref_nvfp4_global(per_row ? amax : amax_all);
-        g_out[r] = g;
         for (int64_t k = 0; k < K_lp; k++) {
-            int64_t src = -1;
-            if (group == 0) {
-                src = k;
-            } else if (k < K_lift) {           /* window i of 4 pairs, element t */
-                int64_t wi = k / 8, t = k % 8;
-                int64_t gi = wi / (Nh - 1), j = wi % (Nh - 1);
-                src = 2 * (gi * group + 2 * j) + t;
-            }
+            int64_t src = pair_lift_src(k, group, K_lift);
             lifted[k] = (src >= 0 && src < K) ? x[src] : 0.0f;
         }
         for (int64_t b = 0; b < K_lp / block; b++) {
@@ -954,6 +963,45 @@ int ssref_quant_nvfp4(const float *X, int64_t rows, int64_t K, int keep, int gro
         }
     }
     free(lifted);
+    return SSREF_OK;
+}
+
+/* The activation of a sparse NVFP4 product as the [LC] NVFP4 row defines
+ * it: one global scale for the tensor, local scales per group of 16
+ * elements along the ORIGINAL K (no lift, no padding to the lifted blocks).
+ * The decoded values (codes times local scale, global scale not applied)
+ * are then lifted to K_lp positions by the same pair window map, since
+ * lifting only copies elements (the lossless decomposition, [SS] and
+ * [OM] 2.3): Xlift [rows, K_lp] doubles, g_out[0].  The tensor-core path
+ * cannot take this form (its sparse instruction scales 32 lifted K at a
+ * time); the tests use it to measure what that costs. */
+int ssref_nvfp4_act_page(const float *X, int64_t rows, int64_t K, int keep, int group,
+                         double *Xlift, float *g_out) {
+    int64_t K_lift, K_lp;
+    int st = ssref_fp4_shape(keep, group, K, &K_lift, &K_lp);
+    if (st) return st;
+    float amax = 0.0f;
+    for (int64_t i = 0; i < rows * K; i++) amax = fmaxf(amax, fabsf(X[i]));
+    float g = ssref_nvfp4_global(amax);
+    g_out[0] = g;
+    int64_t K16 = round_up(K, 16);
+    float *row = (float *)malloc((size_t)K16 * sizeof(float));
+    double *dec = (double *)malloc((size_t)K16 * sizeof(double));
+    for (int64_t r = 0; r < rows; r++) {
+        for (int64_t k = 0; k < K16; k++) row[k] = k < K ? X[r * K + k] : 0.0f;
+        for (int64_t b = 0; b < K16 / 16; b++) {
+            uint8_t codes[16], sc;
+            nvfp4_block(&row[16 * b], 16, g, codes, &sc);
+            double s = ssref_e4m3_to_double(sc);
+            for (int i = 0; i < 16; i++) dec[16 * b + i] = ssref_e2m1_to_double(codes[i]) * s;
+        }
+        for (int64_t k = 0; k < K_lp; k++) {
+            int64_t src = pair_lift_src(k, group, K_lift);
+            Xlift[r * K_lp + k] = (src >= 0 && src < K) ? dec[src] : 0.0;
+        }
+    }
+    free(row);
+    free(dec);
     return SSREF_OK;
 }
 

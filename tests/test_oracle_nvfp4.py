@@ -50,8 +50,10 @@ def test_nvfp4_block_scaling_closed_forms():
     Xv, Xs, g = oracle.quant_nvfp4(X, "dense", 16)
     K_lp = Xv.shape[1] * 2
     D = oracle.decode_dense_nvfp4(Xv, Xs, K_lp, 16)
+    # one global scale for the tensor (the NVFP4 row of the LLM-Compressor
+    # compression-schemes page), from the amax of all its elements
+    assert g.shape == (1,) and g[0] == np.float32(np.abs(X).max()) / np.float32(2688.0)
     for r in range(40):
-        assert g[r] == np.float32(np.abs(X[r]).max()) / np.float32(2688.0)
         for b in range(4):
             blk = X[r, 16 * b:16 * b + 16].astype(np.float64)
             dq = D[r, 16 * b:16 * b + 16]
@@ -62,7 +64,7 @@ def test_nvfp4_block_scaling_closed_forms():
             s = dq[i] / 6.0 if dq[i] != 0 else 0.0
             assert abs(abs(dq[i]) - 6.0 * abs(s)) < 1e-12 and s != 0
             d = abs(s)                                   # block divisor without g
-            for x, y in zip(blk / g[r], dq):
+            for x, y in zip(blk / g[0], dq):
                 step = 0.5 if abs(y) <= 2.0 else (1.0 if abs(y) <= 4.0 else 2.0)
                 assert abs(x - y / d * d) <= 0.5 * step * d * (1 + 2 ** -3) + 1e-9 or abs(x / d) > 6
     assert not Xv[3].any() and not Xs[3].any()
@@ -118,7 +120,7 @@ def test_lifted_activation_follows_the_pair_window_map(pat):
     block = 16 if pat == "dense" else 32
     Xv, Xs, g = oracle.quant_nvfp4(X, pat, block)
     K_lift, K_lp = oracle.fp4_shape(pat, K)
-    D = oracle.decode_dense_nvfp4(Xv, Xs, K_lp, block) * g[:, None]
+    D = oracle.decode_dense_nvfp4(Xv, Xs, K_lp, block) * g[0]
     for k in range(K_lp):
         if pat == "dense":
             src = k if k < K else -1
@@ -133,7 +135,7 @@ def test_lifted_activation_follows_the_pair_window_map(pat):
         if src < 0:
             assert not D[:, k].any()
         else:
-            amax = np.abs(X).max(axis=1)
+            amax = np.abs(X).max()
             assert np.all(np.abs(D[:, k] - X[:, src]) <= np.abs(X[:, src]) * 0.26 + 0.05 * amax + 1e-9)
 
 
@@ -166,8 +168,93 @@ def test_sparse_nvfp4_product_approximates_pruned_matmul(pat):
     # operand (measured 0.09-0.10 here); the product carries both
     assert rel < 0.2
     # and the dense comparator on unpruned W approximates X W^T
-    Wd_v, Wd_s, gwd = oracle.quant_nvfp4(W, "dense", 16, per_row=False)
+    Wd_v, Wd_s, gwd = oracle.quant_nvfp4(W, "dense", 16)
     Xd_v, Xd_s, gxd = oracle.quant_nvfp4(X, "dense", 16)
     Yd = oracle.dense_gemm_nvfp4(Xd_v, Xd_s, gxd, Wd_v, Wd_s, gwd[0], oracle.OUT_F32)
     full = X.astype(np.float64) @ W.T.astype(np.float64)
     assert np.linalg.norm(Yd - full) / np.linalg.norm(full) < 0.2
+
+
+def _src(pat, k, K, K_lift):
+    """Source of lifted position k: window i of 4 pairs reads 8 elements from
+    2 * (2Nh * (i // (Nh - 1)) + 2 * (i % (Nh - 1))) (the SlideSparse
+    write-up's window map, 3.2, on pairs); -1 for padding."""
+    if pat == "dense":
+        return k if k < K else -1
+    if k >= K_lift:
+        return -1
+    _, group = oracle.pattern(pat)
+    wi, t = divmod(k, 8)
+    gi, j = divmod(wi, group // 2 - 1)
+    src = 2 * (gi * group + 2 * j) + t
+    return src if src < K else -1
+
+
+@pytest.mark.parametrize("pat", ["dense"] + PAIR_PATTERNS)
+def test_page_activation_is_the_dense_group16_quantiser_then_the_lift(pat):
+    """The NVFP4 definition's activation (16-element groups along the original
+    K, one global scale) is the dense 16-block quantiser -- pinned above by
+    its closed forms -- followed by the window map: every lifted position
+    holds exactly the decoded value of its source element."""
+    rng = np.random.default_rng(17)
+    K = 512
+    X = (rng.standard_normal((5, K)) * rng.uniform(0.1, 4, (5, 1))).astype(np.float32)
+    Xl, g = oracle.nvfp4_act_page(X, pat)
+    Dv, Ds, gd = oracle.quant_nvfp4(X, "dense", 16)
+    D = oracle.decode_dense_nvfp4(Dv, Ds, K, 16)
+    assert g[0] == gd[0] == np.float32(np.abs(X).max()) / np.float32(2688.0)
+    K_lift, K_lp = oracle.fp4_shape(pat, K)
+    assert Xl.shape == (5, K_lp)
+    for k in range(K_lp):
+        src = _src(pat, k, K, K_lift)
+        if src < 0:
+            assert not Xl[:, k].any()
+        else:
+            np.testing.assert_array_equal(Xl[:, k], D[:, src])
+
+
+def _block_cost(X, W, pat):
+    """Normwise errors of the two activation forms against the exact product
+    of X with the (common) quantised sparse weight."""
+    M, K = X.shape
+    N = W.shape[0]
+    Wv, Wm, Ws, g_w = oracle.compress_weight_nvfp4(W, pat)
+    K_lift, K_lp = oracle.fp4_shape(pat, K)
+    Wd = oracle.decode_sparse_nvfp4(Wv, Wm, Ws, K_lp) * np.float64(g_w)
+    Xlift = np.zeros((M, K_lp))
+    for k in range(K_lp):
+        src = _src(pat, k, K, K_lift)
+        if src >= 0:
+            Xlift[:, k] = X[:, src]
+    exact = Xlift @ Wd.T                                   # = X . dequant(prune(W))^T
+    Xv, Xs, g_x = oracle.quant_nvfp4(X, pat, 32)
+    Y32 = oracle.sparse_gemm_nvfp4(Wv, Wm, Ws, g_w, Xv, Xs, g_x, M, N, K_lp, oracle.OUT_F32)
+    Y16 = oracle.sparse_gemm_nvfp4_page(Wv, Wm, Ws, g_w, X, pat, oracle.OUT_F32)
+    nrm = np.linalg.norm(exact)
+    return (np.linalg.norm(Y16 - exact) / nrm, np.linalg.norm(Y32 - exact) / nrm,
+            np.linalg.norm(Y32 - Y16) / nrm)
+
+
+@pytest.mark.parametrize("kind", ["gauss", "outlier"])
+@pytest.mark.parametrize("pat", ["2:4", "6:8"])
+def test_block32_activation_cost_against_the_group16_definition(pat, kind):
+    """The sparse FP4 instruction scales the dense operand per 32 lifted K, the
+    NVFP4 definition per 16 elements.  Against the exact product with the
+    (common) quantised weight, the 32-block activation error stays within 1.4x
+    of the definition's on Gaussian activations and with 1% of channels x20.
+    Measured here (normwise): 16-block 0.091-0.096, 32-block 0.100 (Gaussian)
+    and 0.117-0.121 (outliers: a x20 channel coarsens the scale of 31 other
+    elements instead of 15), distance between the two 0.089-0.095.  A
+    Gaussian block of 32 has a larger expected maximum than one of 16
+    (about 2.4 against 2.1 standard deviations), so its E2M1 steps are ~1.1x
+    coarser; that is the Gaussian ratio."""
+    rng = np.random.default_rng(18)
+    M, N, K = 48, 40, 1024
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    X = rng.standard_normal((M, K)).astype(np.float32)
+    if kind == "outlier":
+        X[:, rng.choice(K, K // 100, replace=False)] *= 20.0
+    e16, e32, dist = _block_cost(X, W, pat)
+    assert 0.0 < e16 < 0.11
+    assert e16 <= e32 <= 1.4 * e16
+    assert dist < 0.11
