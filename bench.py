@@ -43,21 +43,46 @@ from structured_sparse_quantized_b200 import synth  # noqa: E402
 
 METRIC = "dense-equiv TOPS & speedup vs own dense GEMM at prefill M; % sparse TC peak"
 UNIT = "TOPS (dense-equivalent)"
-DEFAULT_WORKLOAD = "llama_q_2of4_int8"
-DEFAULT_M = 8192
-ALSO_WORKLOAD = ("qwen_gateup_6of8_fp8", 8192)  # the SlideSparse 6:8 headline shape
+# The default line: the largest single-GPU configuration, one Llama-3.1-8B
+# gate/up projection (N = 14336, K = 4096) at M = 16384 tokens, 6:8 INT8.
+DEFAULT_WORKLOAD = "llama_layer_gate_up"
+# Side lines on the same run: 2:4 INT8 on the q_proj shape and the SlideSparse
+# 6:8 FP8 headline shape (Qwen2.5-7B gate/up), both at M = 8192.
+ALSO_WORKLOADS = (("llama_q_2of4_int8", 8192), ("qwen_gateup_6of8_fp8", 8192))
 FLUSH_BYTES = 256 << 20
 IDEAL = {"2:4": 2.0, "4:6": 1.5, "6:8": 4.0 / 3.0, "8:10": 1.25}
 
 # DRAM bytes per launch of the dominant kernel (dram__bytes_read.sum +
-# dram__bytes_write.sum of one sparse-GEMM launch) from one ncu capture of the
-# same kernel build; absent when not captured for this build.  Keyed by
-# (workload, M, pattern, qdtype) as run.
-TRAFFIC = {
-    ("llama_q_2of4_int8", 8192, "2:4", "int8"): 44.21e6 + 16.07e6,
-    ("llama_q_2of4_bf16", 8192, "2:4", "bf16"): 86.13e6 + 38.76e6,
-    ("llama_gateup_4of8_nvfp4", 8192, "2:4", "nvfp4"): 38.83e6 + 178.86e6,
-}
+# dram__bytes_write.sum of one sparse-GEMM launch) from one ncu capture.
+# Keyed by (workload, M, pattern, qdtype) as run; each entry names the
+# profile summary it comes from and the hash of the kernel sources
+# (csrc_hash()) it was captured with.  A stored figure is reported only while
+# the sources still hash the same; otherwise "traffic" is null.
+TRAFFIC = {}
+
+
+def csrc_hash() -> str:
+    """sha256 (first 16 hex digits) of the library's CUDA sources."""
+    import hashlib
+    d = os.path.join(HERE, "structured_sparse_quantized_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(d, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 def load_peaks():
@@ -190,6 +215,10 @@ class Path:
             _, self.K_p = ss.ss_fp4_shape("dense", self.K)
             self.act = ss.quant_lift_act_nvfp4(self.X, self.pat, 32)
             self.dense_act = ss.quant_lift_act_nvfp4(self.X, "dense", 16)
+            # row blocks of the end-to-end run are separate calls, each with
+            # its own tensor-wide global scale (16-byte aligned slots)
+            self.g_blocks = torch.zeros(4 * ((M + 127) // 128), dtype=torch.float32,
+                                        device=device)
             self.Y = torch.empty((M, self.N), dtype=self.out_dtype, device=device)
             del W
             torch.cuda.synchronize()
@@ -246,9 +275,10 @@ class Path:
         m = r1 - r0
         rows = lambda t: None if t is None else t[r0:r1]  # bf16 tier: no scales
         if self.fp4:
-            Xv, Xs, g_x = self.act
+            Xv, Xs, _ = self.act
             nblk = self.K_lp // 32  # tile-major scales: 128-row tiles are contiguous
-            part = (Xv[r0:r1], Xs[r0 * nblk:r1 * nblk], g_x[r0:r1])
+            g = self.g_blocks[4 * (r0 // 128):4 * (r0 // 128) + 4]
+            part = (Xv[r0:r1], Xs[r0 * nblk:r1 * nblk], g)
             ss.quant_lift_act_nvfp4(X_rows, self.pat, 32, out=part)
             ss.sparse_gemm_nvfp4(self.sparse_w, part, m, self.N, out=self.Y[r0:r1])
         elif self.online:
@@ -301,8 +331,8 @@ class Path:
 
     def act_kernel_bytes(self):
         esz = self.X.element_size()
-        if self.fp4:  # codes, one UE4M3 scale per 32, a global scale per token
-            return self.M * (esz * self.K + self.K_lp // 2 + self.K_lp // 32 + 4)
+        if self.fp4:  # codes, one UE4M3 scale per 32, one global scale (X read once)
+            return self.M * (esz * self.K + self.K_lp // 2 + self.K_lp // 32) + 4
         vb, sb = (2, 0) if self.q == "bf16" else (1, 4)   # value bytes, scale bytes
         if self.online:
             return self.M * (esz * self.K + vb * self.K_lp // 2 + self.K_lp // 8 + sb)
@@ -310,7 +340,7 @@ class Path:
 
     def dense_act_bytes(self):
         if self.fp4:
-            return self.M * (self.X.element_size() * self.K + self.K_p // 2 + self.K_p // 16 + 4)
+            return self.M * (self.X.element_size() * self.K + self.K_p // 2 + self.K_p // 16) + 4
         vb, sb = (2, 0) if self.q == "bf16" else (1, 4)
         return self.M * (self.X.element_size() * self.K + vb * self.dense_act[0].shape[1] + sb)
 
@@ -569,6 +599,7 @@ def run_reference(args, dist: Dist):
     line.update({"impl": "reference", "value": v, "ms_per_step": secs * 1e3,
                  "dtype": synth.WORKLOADS[args.workload]["qdtype"],
                  "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                  "cpu_model": cpu_model(),
                                   "sample": f"{rows} of {M} token rows per step (quant/lift or "
                                             f"online prune + sparse GEMM rows); weight "
                                             f"compression offline, untimed"},
@@ -585,7 +616,7 @@ def main():
     ap.add_argument("--impl", default="ss", choices=["ss", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--m", type=int, default=None)
-    ap.add_argument("--no-also", action="store_true", help="skip the 6:8 FP8 side measurement")
+    ap.add_argument("--no-also", action="store_true", help="skip the side measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--ref-budget", type=float, default=6.0)
     ap.add_argument("--pattern", default=None, choices=["2:4", "4:6", "6:8", "8:10"],
@@ -599,7 +630,7 @@ def main():
         w["qdtype"] = args.qdtype or w["qdtype"]
         synth.WORKLOADS[args.workload] = w
     if args.m is None:
-        args.m = DEFAULT_M if args.workload != "linear_6of8_int8_m16" else 16
+        args.m = synth.WORKLOADS[args.workload]["M"]
     args.warmup = max(args.warmup, 3)
     dist = Dist()
     if args.impl == "reference":
@@ -616,6 +647,8 @@ def main():
     line = base_line(args, args.workload, args.m, n)
     wl = synth.WORKLOADS[args.workload]
     tr = TRAFFIC.get((args.workload, args.m, wl["pattern"], wl["qdtype"]))
+    src_hash = csrc_hash()
+    traffic = tr["bytes"] if tr and tr["csrc_hash"] == src_hash else None
     line.update({
         "value": value, "ms_per_step": r["t_step_ms"],
         "dtype": path.q,
@@ -638,7 +671,9 @@ def main():
                      "peak_source": f"{peaks['source']} bf16 burst x"
                                     f"{r['sparse_peak'] / peaks['bf16_tflops']:.0f}"
                                     + (" (2:4 x2)" if path.q == "bf16" else " (8-bit x2, 2:4 x2)"),
-                     "traffic": tr},
+                     "traffic": traffic,
+                     "traffic_source": ({"profile": tr["profile"], "csrc_hash": tr["csrc_hash"]}
+                                        if traffic is not None else None)},
         "e2e": {"value": n * path.dense_equiv_ops() / (t_e2e * 1e-3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": r["launches"],
@@ -649,27 +684,35 @@ def main():
                                 "gemm_speedup": r["t_fp8_gemm_ms"] / r["t_gemm_ms"],
                                 "fp8_step_us": r["t_fp8_step_ms"] * 1e3,
                                 "fp8_gemm_us": r["t_fp8_gemm_ms"] * 1e3}
-    if not args.no_also and dist.world == 1 and args.workload != ALSO_WORKLOAD[0]:
+    if not args.no_also and dist.world == 1:
         del path
         torch.cuda.empty_cache()
-        p2 = Path(ALSO_WORKLOAD[0], ALSO_WORKLOAD[1], torch.device("cuda", dist.local))
-        r2 = measure(p2, max(5, args.steps // 2), args.warmup, dist, peaks)
-        line["also"] = {
-            "workload": ALSO_WORKLOAD[0], "M": ALSO_WORKLOAD[1],
-            "value": p2.dense_equiv_ops() / (r2["t_step_ms"] * 1e-3) / 1e12,
-            "speedup_vs_own_dense": r2["t_dense_step_ms"] / r2["t_step_ms"],
-            "gemm_speedup_vs_own_dense": r2["t_dense_gemm_ms"] / r2["t_gemm_ms"],
-            "ideal_speedup": IDEAL[p2.pat],
-            "pct_sparse_tc_peak": 100.0 * r2["sparse_gemm_tflops"] / r2["sparse_peak"],
-            "act_gbs": r2["act_gbs"], "act_frac_hbm": r2["act_gbs"] / peaks["hbm_gbs"],
-            "sparse_gemm_us": r2["t_gemm_ms"] * 1e3, "dense_gemm_us": r2["t_dense_gemm_ms"] * 1e3,
-        }
-        del p2
+        line["also"] = []
+        for name, m in ALSO_WORKLOADS:
+            if name == args.workload:
+                continue
+            p2 = Path(name, m, torch.device("cuda", dist.local))
+            r2 = measure(p2, max(5, args.steps // 2), args.warmup, dist, peaks)
+            line["also"].append({
+                "workload": name, "M": m, "pattern": p2.pat, "qdtype": p2.q,
+                "value": p2.dense_equiv_ops() / (r2["t_step_ms"] * 1e-3) / 1e12,
+                "speedup_vs_own_dense": r2["t_dense_step_ms"] / r2["t_step_ms"],
+                "gemm_speedup_vs_own_dense": r2["t_dense_gemm_ms"] / r2["t_gemm_ms"],
+                "ideal_speedup": IDEAL[p2.pat],
+                "pct_sparse_tc_peak": 100.0 * r2["sparse_gemm_tflops"] / r2["sparse_peak"],
+                "act_gbs": r2["act_gbs"], "act_frac_hbm": r2["act_gbs"] / peaks["hbm_gbs"],
+                "sparse_gemm_us": r2["t_gemm_ms"] * 1e3,
+                "dense_gemm_us": r2["t_dense_gemm_ms"] * 1e3,
+            })
+            del p2
+            torch.cuda.empty_cache()
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
         tops, rows, secs, cores = oracle_sample(args.workload, args.m, budget_s=10.0)
         line["cpu_baseline"] = {"value": tops, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "cpu_model": cpu_model(),
                                 "sample": f"{rows} of {args.m} token rows of the same workload "
-                                          f"({secs:.1f} s)"}
+                                          f"({secs:.1f} s; weight compression offline, "
+                                          f"untimed)"}
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     dist.close()

@@ -223,17 +223,22 @@ ss_status ss_compress_weight_nvfp4(const void *W, ss_in_dtype in_dtype, int64_t 
                                    ss_pattern p, void *Wv, void *Wm, void *Ws, float *g_w,
                                    ss_stream_t stream);
 
-/* NVFP4 activation: per token, global scale g_x[m] = amax(row) / 2688 (no
- * calibration set exists, so it is taken from the row), the pair lift of
- * pattern p, blocks of `block` lifted elements (32 for the sparse product,
- * 16 for the dense one).  Outputs Xv [M, K_lp/2] bytes, Xs
- * ss_fp4_scale_bytes(M, K_lp, block), g_x [M]. */
+/* NVFP4 activation: ONE global scale for the tensor, g_x[0] = amax(X) / 2688
+ * (the NVFP4 row: a global scale per tensor; the page calibrates it on a
+ * data set, and with none here it is taken from this call's X, so the call
+ * first reduces |X| over all M x K elements), the pair lift of pattern p,
+ * blocks of `block` lifted elements (32 for the sparse product -- the sparse
+ * FP4 instruction scales 32 lifted K at a time, where the page's groups are
+ * 16 -- and 16 for the dense one).  Outputs Xv [M, K_lp/2] bytes, Xs
+ * ss_fp4_scale_bytes(M, K_lp, block), g_x [1].  g_x also serves as the
+ * reduction's accumulator while the call runs (four launches: zero, amax,
+ * quantise, g = amax / 2688). */
 ss_status ss_quant_lift_act_nvfp4(const void *X, ss_in_dtype in_dtype, int64_t M, int64_t K,
                                   ss_pattern p, int32_t block, void *Xv, void *Xs, float *g_x,
                                   ss_stream_t stream);
 
 /* Sparse NVFP4 GEMM (tcgen05.mma.sp kind::mxf4nvf4, block-scaled; one SM or a
- * CTA pair per MMA): Y[m, n] = ((float)acc[m, n] * g_x[m]) * g_w[0], acc the fp32
+ * CTA pair per MMA): Y[m, n] = ((float)acc[m, n] * g_x[0]) * g_w[0], acc the fp32
  * tensor-core sum of (codes x local scales) products; A = the compressed
  * weight, B = the lifted activation (block 32).  K_lp a positive multiple
  * of 256. */
@@ -248,9 +253,29 @@ ss_status ss_dense_gemm_nvfp4(const void *Xv, const void *Xs, const float *g_x, 
                               const void *Ws, const float *g_w, int64_t M, int64_t N,
                               int64_t K_p, void *Y, ss_out_dtype out_dtype, ss_stream_t stream);
 
-/* Synchronises `stream`, returns the first device-side error recorded since
- * the last call (SS_ERR_TIMEOUT, SS_ERR_DATA) or SS_OK, and clears it. */
+/* Returns the first device-side error recorded since the last call
+ * (SS_ERR_TIMEOUT, SS_ERR_DATA) or SS_OK, and clears it.  The status word is
+ * one per device, shared by every stream: a kernel on `stream` takes it and
+ * leaves zero in one atomic exchange after all work queued on `stream`
+ * before the call, then the call waits for `stream`.  An error raised by a
+ * kernel still running on ANOTHER stream is not lost -- it stays for the
+ * next call -- but it is reported only if that kernel finished first, so
+ * quiesce every stream that runs this library's kernels before relying on
+ * the answer. */
 ss_status ss_get_device_status(ss_stream_t stream);
+
+/* Test hooks for the bounded waits (no counterpart in the pages).
+ * ss_debug_set_wait_limit: every device-side wait gives up after `ns`
+ *   nanoseconds (1 ms .. 60 s; 4 s by default) and records SS_ERR_TIMEOUT.
+ * ss_debug_skip_stage: when kb >= 0, the producers of the 8-bit and bf16
+ *   GEMM kernels issue no copies for K stage kb of their first output tile,
+ *   so the MMA warp's bounded wait for that stage runs out: a wait that
+ *   nothing satisfies, with no copy or MMA aimed at it.  The kernel then
+ *   unwinds (lets issued copies land, drains issued MMAs, frees tensor
+ *   memory) and the next call runs normally.  kb = -1 turns it off.
+ * Both synchronise the device and set a device-wide value. */
+ss_status ss_debug_set_wait_limit(uint64_t ns);
+ss_status ss_debug_skip_stage(int32_t kb);
 
 /* Human-readable name of a status code (static storage). */
 const char *ss_status_string(ss_status s);

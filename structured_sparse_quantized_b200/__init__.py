@@ -15,6 +15,7 @@ preallocated by the caller):
     ss_parse_pattern, ss_slide_shape, ss_act_2to4_shape, ss_compress_weight,
     ss_quant_lift_act, ss_prune_act_2to4, ss_sparse_gemm, ss_dense_gemm,
     ss_get_device_status, ss_status_string, ss_kernel_launches, ss_meta_bytes,
+    ss_debug_set_wait_limit, ss_debug_skip_stage (test hooks),
     ss_fp4_shape, ss_fp4_scale_bytes, ss_compress_weight_nvfp4,
     ss_quant_lift_act_nvfp4, ss_sparse_gemm_nvfp4, ss_dense_gemm_nvfp4
 Convenience wrappers that allocate their outputs with torch:
@@ -83,6 +84,8 @@ def lib() -> ctypes.CDLL:
         "ss_sparse_gemm": [i32, p, p, p, p, p, i64, i64, i64, i32, p, i32, p],
         "ss_dense_gemm": [p, p, p, p, i64, i64, i64, i32, p, i32, p],
         "ss_get_device_status": [p],
+        "ss_debug_set_wait_limit": [ctypes.c_uint64],
+        "ss_debug_skip_stage": [i32],
         "ss_fp4_shape": [pat, i64, ctypes.POINTER(i64), ctypes.POINTER(i64)],
         "ss_compress_weight_nvfp4": [p, i32, i64, i64, pat, p, p, p, p, p],
         "ss_quant_lift_act_nvfp4": [p, i32, i64, i64, pat, i32, p, p, p, p],
@@ -236,6 +239,16 @@ def ss_get_device_status(stream=None) -> int:
     return int(lib().ss_get_device_status(_stream(stream)))
 
 
+def ss_debug_set_wait_limit(ns: int) -> None:
+    """Test hook: device-side waits give up after `ns` nanoseconds (4 s default)."""
+    _check(lib().ss_debug_set_wait_limit(int(ns)), "ss_debug_set_wait_limit")
+
+
+def ss_debug_skip_stage(kb: int) -> None:
+    """Test hook: GEMM producers skip K stage `kb` of their first tile (-1: off)."""
+    _check(lib().ss_debug_skip_stage(int(kb)), "ss_debug_skip_stage")
+
+
 # ------------------------------------------------------------------ allocating wrappers
 # Stored values are uint8 codes for the 8-bit tiers and bfloat16 for the bf16
 # tier, which has no scales (its s_* entries are None).
@@ -387,14 +400,14 @@ def compress_weight_nvfp4(W: torch.Tensor, pattern, stream=None):
 
 
 def quant_lift_act_nvfp4(X: torch.Tensor, pattern, block: int, stream=None, out=None):
-    """-> (Xv [M, K_lp/2] uint8, Xs scale bytes, g_x [M])."""
+    """-> (Xv [M, K_lp/2] uint8, Xs scale bytes, g_x: [0] is the tensor's global scale)."""
     M, K = X.shape
     p = _pattern(pattern)
     _, K_lp = ss_fp4_shape(p, K)
     if out is None:
         out = (torch.empty((M, K_lp // 2), dtype=torch.uint8, device=X.device),
                torch.empty(ss_fp4_scale_bytes(M, K_lp, block), dtype=torch.uint8, device=X.device),
-               torch.empty(M, dtype=torch.float32, device=X.device))
+               torch.empty(4, dtype=torch.float32, device=X.device))
     ss_quant_lift_act_nvfp4(X, p, block, out[0], out[1], out[2], stream)
     return out
 
@@ -422,8 +435,9 @@ def dense_gemm_nvfp4(act, packed, M: int, N: int, out_dtype=torch.bfloat16, stre
 
 
 def linear_nvfp4(X: torch.Tensor, packed, pattern, out_dtype=torch.bfloat16, stream=None):
-    """Y = X W^T in NVFP4: per-token quant + pair lift (blocks of 32 for a
-    sparse weight, 16 for a dense one), then the block-scaled GEMM."""
+    """Y = X W^T in NVFP4: quantisation with one global scale for X + pair
+    lift (blocks of 32 for a sparse weight, 16 for a dense one), then the
+    block-scaled GEMM."""
     dense = _pattern(pattern).group == 0
     act = quant_lift_act_nvfp4(X, pattern, 16 if dense else 32, stream)
     M, N = X.shape[0], packed[0].shape[0]

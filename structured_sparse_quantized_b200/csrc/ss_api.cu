@@ -871,44 +871,53 @@ ss_status ss_quant_lift_act_nvfp4(const void* X, ss_in_dtype in_dtype, int64_t M
     int dev;
     if ((st = check_device(&dev)) != SS_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const int warps = ss::kWarpRowThreads / 32;
-    const unsigned grid = static_cast<unsigned>(((M + 127) / 128 * 128 + warps - 1) / warps);
+    // g_x[0] first accumulates the amax bits of X (zeroed, then atomicMax
+    // over the tensor), pass 2 derives g from it, and the last launch turns
+    // it into g = amax / 2688 in place.
+    auto* amax = reinterpret_cast<unsigned int*>(g_x);
+    if ((st = launch_ex(ss::zero_word_kernel, dim3(1), dim3(32), 0, s, 1, amax)) != SS_OK) return st;
+    const int64_t n = M * K;
+    const int64_t esz = in_dtype == SS_IN_BF16 ? 2 : 4;
+    const int64_t nv = n * esz / 16;
+    const unsigned agrid = static_cast<unsigned>(
+        std::max<int64_t>(1, std::min<int64_t>((nv + 255) / 256, 148 * 8)));
+    if (in_dtype == SS_IN_BF16)
+        st = launch_ex(ss::fp4_act_amax_kernel<__nv_bfloat16>, dim3(agrid), dim3(256), 0, s, 1,
+                       static_cast<const __nv_bfloat16*>(X), n, amax);
+    else
+        st = launch_ex(ss::fp4_act_amax_kernel<float>, dim3(agrid), dim3(256), 0, s, 1,
+                       static_cast<const float*>(X), n, amax);
+    if (st != SS_OK) return st;
+    if (K_lp > INT32_MAX / 2 || M > (int64_t{1} << 30)) return SS_ERR_UNSUPPORTED;
+    // one warp per row at a time: up to 8 row slots per SM
+    const int64_t M_pad = (M + 127) / 128 * 128;
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>((M_pad + 7) / 8, 148 * 8));
+    const int Mi = static_cast<int>(M), Ki = static_cast<int>(K);
+    const int Kl = static_cast<int>(K_lift), Kp = static_cast<int>(K_lp);
     const int Nh = p.group / 2;
     auto* xv = static_cast<uint8_t*>(Xv);
     auto* xs = static_cast<uint8_t*>(Xs);
-    // bf16 rows under the identity map with K_lp <= 4096: one read of X, in
-    // registers (two warps per row above 2048, to keep the occupancy up)
-    if (in_dtype == SS_IN_BF16 && Nh <= 2 && K % 8 == 0 && K_lp <= 4096) {
-        const auto* xb = static_cast<const __nv_bfloat16*>(X);
-        const int wpr = K_lp > 2048 ? 2 : 1;
-        const int rows_per_cta = (ss::kWarpRowThreads / 32) / wpr;
-        const unsigned rgrid =
-            static_cast<unsigned>(((M + 127) / 128 * 128 + rows_per_cta - 1) / rows_per_cta);
-        const int chunks = static_cast<int>(K_lp / (256 * wpr));
-#define SS_FP4R(B, C, W)                                                                       \
-    return launch_ex(ss::quant_nvfp4_reg_kernel<B, C, W>, dim3(rgrid),                        \
-                     dim3(ss::kWarpRowThreads), 0, s, 1, xb, M, K, K_lp, xv, xs, g_x)
-        if (block == 32) {
-            if (wpr == 2) SS_FP4R(32, 8, 2);
-            if (chunks <= 4) SS_FP4R(32, 4, 1);
-            SS_FP4R(32, 8, 1);
-        }
-        if (wpr == 2) SS_FP4R(16, 8, 2);
-        if (chunks <= 4) SS_FP4R(16, 4, 1);
-        SS_FP4R(16, 8, 1);
-#undef SS_FP4R
+#define SS_FP4X(T, B, NH)                                                                     \
+    st = launch_ex(ss::quant_nvfp4_act_kernel<T, B, NH>, dim3(grid), dim3(256), 0, s, 1,     \
+                   static_cast<const T*>(X), Mi, Ki, Kl, Kp, amax, xv, xs)
+#define SS_FP4NH(T, B)                                                                        \
+    switch (Nh) {                                                                             \
+        case 3: SS_FP4X(T, B, 3); break;                                                      \
+        case 4: SS_FP4X(T, B, 4); break;                                                      \
+        case 5: SS_FP4X(T, B, 5); break;                                                      \
+        default: SS_FP4X(T, B, 2); break;                                                     \
     }
-#define SS_FP4X(T, B)                                                                          \
-    return launch_ex(ss::quant_lift_nvfp4_kernel<T, B>, dim3(grid), dim3(ss::kWarpRowThreads), \
-                     0, s, 1, static_cast<const T*>(X), M, K, Nh, static_cast<int>(p.group),   \
-                     K_lift, K_lp, xv, xs, g_x)
     if (in_dtype == SS_IN_BF16) {
-        if (block == 32) SS_FP4X(__nv_bfloat16, 32);
-        SS_FP4X(__nv_bfloat16, 16);
+        if (block == 32) { SS_FP4NH(__nv_bfloat16, 32) }
+        else { SS_FP4NH(__nv_bfloat16, 16) }
+    } else {
+        if (block == 32) { SS_FP4NH(float, 32) }
+        else { SS_FP4NH(float, 16) }
     }
-    if (block == 32) SS_FP4X(float, 32);
-    SS_FP4X(float, 16);
+#undef SS_FP4NH
 #undef SS_FP4X
+    if (st != SS_OK) return st;
+    return launch_ex(ss::fp4_global_kernel, dim3(1), dim3(32), 0, s, 1, g_x);
 }
 
 }  // extern "C"
@@ -1009,13 +1018,36 @@ ss_status ss_get_device_status(ss_stream_t stream) {
     ss_status st = check_device(&dev);
     if (st != SS_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (cudaStreamSynchronize(s) != cudaSuccess) return SS_ERR_CUDA;
+    // one thread takes the word and leaves zero in one atomic exchange, after
+    // everything queued on `s` before it (plain launch: full serialisation)
+    ss::status_exchange_kernel<<<1, 1, 0, s>>>();
+    if (cudaGetLastError() != cudaSuccess) return SS_ERR_CUDA;
     int code = 0;
-    const int zero = 0;
-    if (cudaMemcpyFromSymbol(&code, ss::g_status, sizeof(int)) != cudaSuccess) return SS_ERR_CUDA;
-    if (code != 0 && cudaMemcpyToSymbol(ss::g_status, &zero, sizeof(int)) != cudaSuccess)
+    if (cudaMemcpyFromSymbolAsync(&code, ss::g_status_taken, sizeof(int), 0,
+                                  cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
         return SS_ERR_CUDA;
     return static_cast<ss_status>(code);
+}
+
+ss_status ss_debug_set_wait_limit(uint64_t ns) {
+    int dev;
+    ss_status st = check_device(&dev);
+    if (st != SS_OK) return st;
+    if (ns < 1000000ull || ns > 60000000000ull) return SS_ERR_INVALID_ARG;  // 1 ms .. 60 s
+    if (cudaDeviceSynchronize() != cudaSuccess) return SS_ERR_CUDA;
+    if (cudaMemcpyToSymbol(ss::g_wait_limit_ns, &ns, sizeof(ns)) != cudaSuccess) return SS_ERR_CUDA;
+    return SS_OK;
+}
+
+ss_status ss_debug_skip_stage(int32_t kb) {
+    int dev;
+    ss_status st = check_device(&dev);
+    if (st != SS_OK) return st;
+    if (kb < -1) return SS_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return SS_ERR_CUDA;
+    if (cudaMemcpyToSymbol(ss::g_skip_stage, &kb, sizeof(kb)) != cudaSuccess) return SS_ERR_CUDA;
+    return SS_OK;
 }
 
 }  // extern "C"

@@ -13,15 +13,27 @@ namespace ss {
 
 // Device status word: the first device-side error since the last read.
 __device__ int g_status;
+// Written by ss_get_device_status()'s exchange kernel: the status it took.
+__device__ int g_status_taken;
 
 __device__ __forceinline__ void record_status(int code) { atomicCAS(&g_status, 0, code); }
 
+// Take the status word and leave zero, in one atomic exchange, so that an
+// error recorded concurrently is either taken now or left for the next read.
+__global__ void status_exchange_kernel() { g_status_taken = atomicExch(&g_status, 0); }
+
 // ---------------------------------------------------------------------------
 // Time and bounded waits.  Every spin in these kernels gives up after
-// kWaitLimitNs (or when the CTA-wide abort flag is raised), records
-// SS_ERR_TIMEOUT and lets the caller unwind; nothing traps or hangs.
+// g_wait_limit_ns (4 s unless a test shortens it through
+// ss_debug_set_wait_limit) or when the CTA-wide abort flag is raised,
+// records SS_ERR_TIMEOUT and lets the caller unwind; nothing traps or hangs.
 // ---------------------------------------------------------------------------
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s
+__device__ uint64_t g_wait_limit_ns = kWaitLimitNs;
+// Test hook (ss_debug_skip_stage): when >= 0, the GEMM producers issue no
+// copies for K stage g_skip_stage of their first tile, so the MMA warp's wait
+// for that stage can only run out.  -1 (off) in normal use.
+__device__ int g_skip_stage = -1;
 constexpr int kErrTimeout = 6;                    // SS_ERR_TIMEOUT
 constexpr int kErrData = 7;                       // SS_ERR_DATA
 
@@ -71,7 +83,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
         if (mbar_try_wait(b, parity)) return true;
         if ((i & 255u) == 0) {
             if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
+            if (global_timer_ns() - t0 > *reinterpret_cast<volatile uint64_t*>(&g_wait_limit_ns)) {
                 record_status(kErrTimeout);
                 *abort_flag = 1;
                 return false;

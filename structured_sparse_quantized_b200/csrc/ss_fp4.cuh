@@ -251,187 +251,195 @@ __global__ void __launch_bounds__(kCompressThreads) compress_weight_nvfp4_kernel
     }
 }
 
-// NVFP4 activation: one warp per token row.  Pass 1: row absmax, g = a / 2688.
-// Pass 2: each lane takes whole blocks of kBlock lifted elements (gathered
-// through the pair window map), quantises them and writes kBlock / 2 bytes
-// and one scale.  Warps past M zero the scales of the padding rows.
-template <typename T, int kBlock>
-__global__ void __launch_bounds__(kWarpRowThreads) quant_lift_nvfp4_kernel(
-    const T* __restrict__ X, int64_t M, int64_t K64, int Nh, int group, int64_t K_lift,
-    int64_t K_lp, uint8_t* __restrict__ Xv, uint8_t* __restrict__ Xs, float* __restrict__ g_x) {
+// L2 cache policies for the two passes over X: pass 1 keeps it resident for
+// pass 2 (evict_last), pass 2 is its last use (evict_first).
+__device__ __forceinline__ uint4 ldg_policy(const void* p, uint64_t pol) {
+    uint4 v;
+    asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p), "l"(pol));
+    return v;
+}
+
+__device__ __forceinline__ uint2 ldg_policy2(const void* p, uint64_t pol) {
+    uint2 v;
+    asm volatile("ld.global.nc.L2::cache_hint.v2.u32 {%0, %1}, [%2], %3;"
+                 : "=r"(v.x), "=r"(v.y)
+                 : "l"(p), "l"(pol));
+    return v;
+}
+
+// NVFP4 activation, pass 1: the absolute maximum of the whole tensor X
+// (M * K elements, contiguous), combined with atomicMax on the float bits
+// into *amax_bits, which the caller has zeroed.  The global scale is per
+// tensor (LLM-Compressor compression schemes, NVFP4 row); with no
+// calibration set it is taken from this call's activation.
+template <typename T>
+__global__ void __launch_bounds__(256) fp4_act_amax_kernel(const T* __restrict__ X, int64_t n,
+                                                           unsigned int* __restrict__ amax_bits) {
     pdl_trigger();
     pdl_wait();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t m = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp;
-    const int64_t M_pad = (M + 127) / 128 * 128;
-    const int64_t nblk = K_lp / kBlock;
-    if (m >= M_pad) return;
-    if (m >= M) {
-        for (int64_t j = lane; j < nblk; j += 32) Xs[fp4_scale_offset(m, j, nblk)] = 0;
-        return;
+    __shared__ float red[8];
+    constexpr int kPer = 16 / sizeof(T);  // elements per 16-byte load
+    constexpr int kUnroll = 8;            // loads in flight per thread
+    const int64_t nv = n / kPer;
+    const uint4* xv = reinterpret_cast<const uint4*>(X);  // X is 16-byte aligned
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    const uint64_t keep = l2_policy_evict_last();
+    float a = 0.0f;
+    int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    for (; i + (kUnroll - 1) * stride < nv; i += kUnroll * stride) {
+        uint4 v[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) v[u] = ldg_policy(xv + i + u * stride, keep);
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) a = fmaxf(a, chunk_absmax<T>(v[u]));
     }
-    const int K = static_cast<int>(K64);
-    const T* x = X + m * K64;
-    const bool vec = (K * static_cast<int>(sizeof(T))) % 16 == 0 &&
-                     (reinterpret_cast<uintptr_t>(X) & 15) == 0;
-    const float a = warp_row_absmax<T>(x, K, vec, lane);
-    const float g = __fdiv_rn(a, 2688.0f);
-    if (lane == 0) g_x[m] = g;
-    // One window of 8 lifted elements per lane; the kBlock / 8 lanes of a
-    // block (adjacent, and always in the same iteration: K_lp / 8 is a
-    // multiple of 32) combine their maxima with shuffles.
-    constexpr int kLanes = kBlock / 8;
-    uint32_t* vrow = reinterpret_cast<uint32_t*>(Xv + m * (K_lp / 2));
-    for (int64_t wi = lane; wi < K_lp / 8; wi += 32) {
-        int64_t src0;
-        if (Nh <= 2) {
-            src0 = 8 * wi;  // dense and pair 2:4: the identity
-        } else if (8 * wi < K_lift) {
-            const int64_t gi = wi / (Nh - 1), j = wi - gi * (Nh - 1);
-            src0 = 2 * (gi * group + 2 * j);
-        } else {
-            src0 = -1;
-        }
-        float v[8];
-        bool done = false;
-        if constexpr (sizeof(T) == 2) {
-            if (src0 >= 0 && src0 + 8 <= K) {
-                const uintptr_t addr = reinterpret_cast<uintptr_t>(x + src0);
-                uint32_t u[4];
-                if ((addr & 15u) == 0) {
-                    const uint4 q = __ldg(reinterpret_cast<const uint4*>(x + src0));
-                    u[0] = q.x, u[1] = q.y, u[2] = q.z, u[3] = q.w;
-                    done = true;
-                } else if ((addr & 3u) == 0) {  // src0 is even; odd K can shift the row
+    for (; i < nv; i += stride) a = fmaxf(a, chunk_absmax<T>(ldg_policy(xv + i, keep)));
+    const int64_t t = nv * kPer + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (t < n) a = fmaxf(a, fabsf(to_f32<T>(X[t])));  // the tail (< kPer elements)
 #pragma unroll
-                    for (int h = 0; h < 4; ++h) u[h] = __ldg(reinterpret_cast<const uint32_t*>(x + src0) + h);
-                    done = true;
-                }
-                if (done) {
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        a = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
 #pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        v[2 * h] = __uint_as_float(u[h] << 16);
-                        v[2 * h + 1] = __uint_as_float(u[h] & 0xFFFF0000u);
-                    }
-                }
-            }
-        }
-        if (!done) {
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                const int64_t src = src0 + t;
-                v[t] = (src0 >= 0 && src < K) ? to_f32<T>(x[src]) : 0.0f;
-            }
-        }
-        float a = 0.0f;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) a = fmaxf(a, fabsf(v[t]));
-#pragma unroll
-        for (int o = 1; o < kLanes; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-        uint32_t sc = 0;
-        float inv = 0.0f;
-        if (g != 0.0f) {
-            sc = ue4m3_code(__fdiv_rn(a, __fmul_rn(6.0f, g)));
-            const float d = __fmul_rn(ue4m3_value(sc), g);
-            inv = d == 0.0f ? 0.0f : __fdiv_rn(1.0f, d);
-        }
-        uint32_t word = 0;
-        if (inv != 0.0f) {
-#pragma unroll
-            for (int h = 0; h < 4; ++h)
-                word |= e2m1x2(__fmul_rn(v[2 * h], inv), __fmul_rn(v[2 * h + 1], inv)) << (8 * h);
-        }
-        __stcs(vrow + wi, word);
-        if ((lane & (kLanes - 1)) == 0)
-            Xs[fp4_scale_offset(m, wi / kLanes, nblk)] = static_cast<uint8_t>(sc);
+        for (int o = 4; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        if (threadIdx.x == 0) atomicMax(amax_bits, __float_as_uint(a));
     }
 }
 
-// Single-pass variant for bf16 rows with the identity map (dense and pair
-// 2:4) and K_lp <= 256 kChunks kWpr: a row is held by kWpr warps; lane l of
-// warp `sub` keeps the 16-byte chunks (8 inputs = one window) 32 sub + l +
-// 32 kWpr i, so X is read from HBM once; window wi = chunk wi, and the lanes
-// of a block are adjacent as above.  The warps of a row combine their maxima
-// through shared memory (one named barrier per row slot).
-template <int kBlock, int kChunks, int kWpr>
-__global__ void __launch_bounds__(kWarpRowThreads) quant_nvfp4_reg_kernel(
-    const __nv_bfloat16* __restrict__ X, int64_t M, int64_t K64, int64_t K_lp,
-    uint8_t* __restrict__ Xv, uint8_t* __restrict__ Xs, float* __restrict__ g_x) {
+// Zero one 32-bit word (the amax accumulator of the next pass).
+__global__ void zero_word_kernel(unsigned int* p) {
     pdl_trigger();
     pdl_wait();
-    constexpr int kLanes = kBlock / 8;
-    constexpr int kRowsPerCta = kWarpRowThreads / (32 * kWpr);
-    __shared__ float part[kRowsPerCta][kWpr];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int slot = warp / kWpr, sub = warp % kWpr;
-    const int64_t m = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + slot;
-    const int64_t M_pad = (M + 127) / 128 * 128;
-    const int64_t nblk = K_lp / kBlock;
-    if (m >= M_pad) return;  // whole row slots leave together
-    if (m >= M) {
-        for (int64_t j = sub * 32 + lane; j < nblk; j += 32 * kWpr) Xs[fp4_scale_offset(m, j, nblk)] = 0;
-        return;
-    }
-    const int K = static_cast<int>(K64);
-    const uint4* x = reinterpret_cast<const uint4*>(X + m * K64);  // K % 8 == 0
-    uint4 c[kChunks];
-    float a = 0.0f;
+    if (threadIdx.x == 0 && blockIdx.x == 0) *p = 0u;
+}
+
+// The 8 lifted elements of window wi (8 consecutive inputs from src0; zero
+// past K and for padding windows, src0 < 0).
+template <typename T>
+__device__ __forceinline__ void load_window8(const T* __restrict__ x, int src0, int K,
+                                             uint64_t pol, float (&v)[8]) {
+    bool done = false;
+    if (src0 >= 0 && src0 + 8 <= K) {
+        const uintptr_t addr = reinterpret_cast<uintptr_t>(x + src0);
+        if constexpr (sizeof(T) == 2) {
+            uint32_t u[4];
+            if ((addr & 15u) == 0) {
+                const uint4 q = ldg_policy(x + src0, pol);
+                u[0] = q.x, u[1] = q.y, u[2] = q.z, u[3] = q.w;
+                done = true;
+            } else if ((addr & 7u) == 0) {
+                const uint2 q0 = ldg_policy2(x + src0, pol);
+                const uint2 q1 = ldg_policy2(x + src0 + 4, pol);
+                u[0] = q0.x, u[1] = q0.y, u[2] = q1.x, u[3] = q1.y;
+                done = true;
+            }
+            if (done) {
 #pragma unroll
-    for (int i = 0; i < kChunks; ++i) {
-        const int ch = sub * 32 + lane + 32 * kWpr * i;
-        c[i] = 8 * ch < K ? __ldg(x + ch) : make_uint4(0u, 0u, 0u, 0u);
-        a = fmaxf(a, chunk_absmax<__nv_bfloat16>(c[i]));
+                for (int h = 0; h < 4; ++h) {
+                    v[2 * h] = __uint_as_float(u[h] << 16);
+                    v[2 * h + 1] = __uint_as_float(u[h] & 0xFFFF0000u);
+                }
+            }
+        } else {
+            if ((addr & 15u) == 0) {
+                const uint4 q0 = ldg_policy(x + src0, pol);
+                const uint4 q1 = ldg_policy(x + src0 + 4, pol);
+                v[0] = __uint_as_float(q0.x), v[1] = __uint_as_float(q0.y);
+                v[2] = __uint_as_float(q0.z), v[3] = __uint_as_float(q0.w);
+                v[4] = __uint_as_float(q1.x), v[5] = __uint_as_float(q1.y);
+                v[6] = __uint_as_float(q1.z), v[7] = __uint_as_float(q1.w);
+                done = true;
+            }
+        }
     }
+    if (!done) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    if constexpr (kWpr > 1) {
-        if (lane == 0) part[slot][sub] = a;
-        named_bar_sync(1 + slot, 32 * kWpr);
-#pragma unroll
-        for (int w = 0; w < kWpr; ++w) a = fmaxf(a, part[slot][w]);
+        for (int t = 0; t < 8; ++t) {
+            const int src = src0 + t;
+            v[t] = (src0 >= 0 && src < K) ? to_f32<T>(x[src]) : 0.0f;
+        }
     }
-    const float g = __fdiv_rn(a, 2688.0f);
+}
+
+// NVFP4 activation, pass 2: one warp per token row at a time, lane l taking
+// the blocks of kBlock lifted elements l, l + 32, ... (kBlock / 8 windows of
+// 8 lifted elements each).  g = amax / 2688 from pass 1; the block scale
+// s = UE4M3(a / (6 g)), d = s g, codes E2M1(x * (1 / d)) (the reciprocal
+// correctly rounded, as 1 / d).  kNh: the pattern's half group (pair windows
+// slide by 2 pairs, Nh - 1 windows per group of 2 Nh pairs); 0 or 2 for the
+// identity map (dense, pair 2:4).  Warps of the padding rows
+// (M <= m < M_pad) only zero their scales.
+template <typename T, int kBlock, int kNh>
+__global__ void __launch_bounds__(256) quant_nvfp4_act_kernel(
+    const T* __restrict__ X, int M, int K, int K_lift, int K_lp,
+    const unsigned int* __restrict__ amax_bits, uint8_t* __restrict__ Xv,
+    uint8_t* __restrict__ Xs) {
+    pdl_trigger();
+    pdl_wait();
+    constexpr int kWin = kBlock / 8;  // windows per block
+    const int lane = threadIdx.x & 31;
+    const int warps = static_cast<int>(gridDim.x * (blockDim.x >> 5));
+    const int M_pad = (M + 127) / 128 * 128;
+    const int nblk = K_lp / kBlock;
+    const float g = __fdiv_rn(__uint_as_float(__ldg(amax_bits)), 2688.0f);
     const float g6 = __fmul_rn(6.0f, g);
-    if (lane == 0 && sub == 0) g_x[m] = g;
-    uint32_t* vrow = reinterpret_cast<uint32_t*>(Xv + m * (K_lp / 2));
-    // Three passes over the chunks (block maxima, block scales, codes) so that
-    // the chunks' dependency chains (shuffles, divisions, conversions) overlap.
-    float inv[kChunks];
-    uint32_t sc[kChunks];
-#pragma unroll
-    for (int i = 0; i < kChunks; ++i) {
-        float b = chunk_absmax<__nv_bfloat16>(c[i]);
-#pragma unroll
-        for (int o = 1; o < kLanes; o <<= 1) b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, o));
-        inv[i] = b;
-    }
-#pragma unroll
-    for (int i = 0; i < kChunks; ++i) {
-        sc[i] = 0;
-        float r = 0.0f;
-        if (g != 0.0f) {
-            sc[i] = ue4m3_code(__fdiv_rn(inv[i], g6));
-            const float d = __fmul_rn(ue4m3_value(sc[i]), g);
-            r = d == 0.0f ? 0.0f : __frcp_rn(d);
+    const uint64_t last = l2_policy_evict_first();
+    for (int m = static_cast<int>(blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)); m < M_pad;
+         m += warps) {
+        if (m >= M) {
+            for (int j = lane; j < nblk; j += 32) Xs[fp4_scale_offset(m, j, nblk)] = 0;
+            continue;
         }
-        inv[i] = r;
-    }
+        const T* x = X + static_cast<int64_t>(m) * K;
+        uint8_t* vrow = Xv + static_cast<int64_t>(m) * (K_lp / 2);
+        for (int b = lane; b < nblk; b += 32) {
+            float v[kWin][8];
 #pragma unroll
-    for (int i = 0; i < kChunks; ++i) {
-        const int64_t wi = sub * 32 + lane + 32 * kWpr * i;
-        if (wi - lane >= K_lp / 8) break;  // the same for every lane (K_lp / 8 % 32 == 0)
-        const uint32_t u[4] = {c[i].x, c[i].y, c[i].z, c[i].w};
-        uint32_t word = 0;
-        if (inv[i] != 0.0f) {
+            for (int q = 0; q < kWin; ++q) {
+                const int wi = b * kWin + q;
+                int src0;
+                if constexpr (kNh <= 2) {
+                    src0 = 8 * wi;
+                } else {
+                    const int gi = wi / (kNh - 1), j = wi - gi * (kNh - 1);
+                    src0 = 8 * wi < K_lift ? 2 * (gi * 2 * kNh + 2 * j) : -1;
+                }
+                load_window8<T>(x, src0, K, last, v[q]);
+            }
+            float a = 0.0f;
 #pragma unroll
-            for (int h = 0; h < 4; ++h)
-                word |= e2m1x2(__fmul_rn(__uint_as_float(u[h] << 16), inv[i]),
-                               __fmul_rn(__uint_as_float(u[h] & 0xFFFF0000u), inv[i]))
-                        << (8 * h);
+            for (int q = 0; q < kWin; ++q)
+#pragma unroll
+                for (int t = 0; t < 8; ++t) a = fmaxf(a, fabsf(v[q][t]));
+            uint32_t sc = 0;
+            float inv = 0.0f;
+            if (g != 0.0f) {
+                sc = ue4m3_code(__fdiv_rn(a, g6));
+                const float d = __fmul_rn(ue4m3_value(sc), g);
+                inv = d == 0.0f ? 0.0f : __frcp_rn(d);
+            }
+            uint32_t w[kWin];
+#pragma unroll
+            for (int q = 0; q < kWin; ++q) {
+                uint32_t word = 0;
+                if (inv != 0.0f) {
+#pragma unroll
+                    for (int h = 0; h < 4; ++h)
+                        word |= e2m1x2(__fmul_rn(v[q][2 * h], inv), __fmul_rn(v[q][2 * h + 1], inv))
+                                << (8 * h);
+                }
+                w[q] = word;
+            }
+            if constexpr (kWin == 4)
+                __stcs(reinterpret_cast<uint4*>(vrow) + b, make_uint4(w[0], w[1], w[2], w[3]));
+            else
+                __stcs(reinterpret_cast<uint2*>(vrow) + b, make_uint2(w[0], w[1]));
+            Xs[fp4_scale_offset(m, b, nblk)] = static_cast<uint8_t>(sc);
         }
-        __stcs(vrow + wi, word);
-        if ((lane & (kLanes - 1)) == 0)
-            Xs[fp4_scale_offset(m, wi / kLanes, nblk)] = static_cast<uint8_t>(sc[i]);
     }
 }
 

@@ -206,6 +206,14 @@ __device__ __forceinline__ float load_scale(const float* s, int i, bool in_range
     else return in_range ? __ldg(s + i) : 0.0f;
 }
 
+// Scale of B row i: per row, 1 for the bf16 tier, or the one global scale
+// of the NVFP4 activation tensor.
+template <int kQ>
+__device__ __forceinline__ float load_b_scale(const float* s, int i, bool in_range) {
+    if constexpr (kQ == kQNvfp4) return in_range ? __ldg(s) : 0.0f;
+    else return load_scale<kQ == kQBf16>(s, i, in_range);
+}
+
 // kQ: kQE4M3, kQInt8 (kind::f8f6f4 / kind::i8), kQBf16 (kind::f16) or kQNvfp4
 // (kind::mxf4nvf4, block-scaled; tm_sfa / tm_sfb are its scale-factor maps,
 // unused otherwise, and s_a is one global scale).
@@ -308,10 +316,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int s = 0;
         uint32_t ph = 0, armed = 0, armed_par = 0;
         bool ok = true;
+        const int skip_kb = g_skip_stage;  // test hook, -1 in normal use
         for (int t = unit; t < n_tiles && ok; t += n_units) {
             const int a0 = (t % nA) * tile_a_rows + static_cast<int>(rank) * kTileA;
             const int b0 = (t / nA) * args.bn + static_cast<int>(rank) * b_rows_cta;
             for (int kb = 0; kb < args.k_stages; ++kb) {
+                if (t == unit && kb == skip_kb) {  // this stage is never loaded
+                    ok = false;
+                    break;
+                }
                 if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u, abort_flag))) {
                     ok = false;
                     break;
@@ -608,7 +621,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                                 for (int e = 0; e < 2; ++e) {
                                     const int tok = b0 + c + 8 * r + 2 * tm + e;
-                                    sb[r][e] = load_scale<kBf16>(args.s_b, tok, tok < args.rowsB);
+                                    sb[r][e] = load_b_scale<kQ>(args.s_b, tok, tok < args.rowsB);
                                 }
                             uint32_t v[2][16];
                             tmem_ld_16x256b_x4(t_row + c, v[0]);
@@ -689,7 +702,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             for (int c = 32 * grp; c < args.bn; c += 64) {
                 const int bc = b0 + c + lane;  // this lane's B row of the chunk
-                const float sb_lane = load_scale<kBf16>(args.s_b, bc, bc < args.rowsB);
+                const float sb_lane = load_b_scale<kQ>(args.s_b, bc, bc < args.rowsB);
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(t_row + c, r);
                 tmem_ld_wait();

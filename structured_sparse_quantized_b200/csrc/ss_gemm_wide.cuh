@@ -166,11 +166,16 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         int s = 0;
         uint32_t ph = 0, armed = 0, armed_par = 0;
         bool ok = true;
+        const int skip_kb = g_skip_stage;  // test hook, -1 in normal use
         for (int k = 0, t = snake_tile(0, unit, n_units); t < n_tiles && ok;
              ++k, t = snake_tile(k, unit, n_units)) {
             const int a0 = (t % nA) * kPairRows + static_cast<int>(rank) * kTileA;
             const int b0 = (t / nA) * tile_b_rows + static_cast<int>(rank) * b_rows_cta;
             for (int kb = 0; kb < args.k_stages; ++kb) {
+                if (k == 0 && kb == skip_kb) {  // this stage is never loaded
+                    ok = false;
+                    break;
+                }
                 if (!__all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u, abort_flag))) {
                     ok = false;
                     break;

@@ -119,3 +119,46 @@ def test_pattern_sweep_llama_q_o(pat, q):
     rows = _rows(M)
     Y_ref = oracle.dense_gemm(Xq_ref, s_x_ref, Wq_ref, s_w_ref, Q[q], oracle.OUT_BF16, m_idx=rows)
     assert_y_matches(host(Y)[rows], Y_ref, q, True)
+
+
+# The Llama-3.1-8B layer sweep at the benchmark's M = 16384: every projection
+# shape other than q/o, every pattern, INT8 and FP8.  Quantised activations,
+# packed weights and metadata are compared in full; Y on the first and last
+# 32 rows plus 64 seeded rows.  down with 8:10 INT8 (K_lp = 22944) is the
+# widest int32 accumulation of the build and must be bit-exact.
+_LAYER_CACHE = {}
+
+
+def _layer_inputs(proj, M):
+    N, K = synth.LLAMA_LAYER[proj]
+    key_w, key_x = ("W", proj), ("X", M, K)
+    if key_w not in _LAYER_CACHE:
+        _LAYER_CACHE[key_w] = synth.make_weight(N, K, 0.02, "bf16")
+    if key_x not in _LAYER_CACHE:   # two activations (K = 4096 and 14336): 0.6 GB bf16
+        _LAYER_CACHE[key_x] = synth.make_activation(M, K, "gauss", "bf16")
+    return _LAYER_CACHE[key_w], _LAYER_CACHE[key_x]
+
+
+@pytest.mark.parametrize("proj", ["gate_up", "k_v", "down"])
+@pytest.mark.parametrize("pat", ["dense", "2:4", "4:6", "6:8", "8:10"])
+@pytest.mark.parametrize("q", ["int8", "fp8"])
+def test_llama_layer_sweep_m16384(proj, pat, q):
+    M = 16384
+    W, X = _layer_inputs(proj, M)
+    N = W.shape[0]
+    if pat != "dense":
+        _weight_sparse_case(W, X, pat, q)
+        return
+    Wq_ref, _, s_w_ref = oracle.compress_weight(W, "dense", Q[q])
+    Xq_ref, s_x_ref = oracle.quant_lift_act(X, "dense", Q[q])
+    Wq, _, s_w = ss.compress_weight(dev(W), "dense", q)
+    Xq, s_x = ss.quant_lift_act(dev(X), "dense", q)
+    np.testing.assert_array_equal(host(Wq), Wq_ref)
+    np.testing.assert_array_equal(host(s_w), s_w_ref)
+    np.testing.assert_array_equal(host(Xq), Xq_ref)
+    np.testing.assert_array_equal(host(s_x), s_x_ref)
+    Y = ss.dense_gemm(Xq, s_x, Wq, s_w, q)
+    assert ss.ss_get_device_status() == ss.SS_OK
+    rows = _rows(M)
+    Y_ref = oracle.dense_gemm(Xq_ref, s_x_ref, Wq_ref, s_w_ref, Q[q], oracle.OUT_BF16, m_idx=rows)
+    assert_y_matches(host(Y)[rows], Y_ref, q, True)
