@@ -633,6 +633,48 @@ ss_status ss_prune_act_2to4(const void* X, ss_in_dtype in_dtype, int64_t M, int6
     const int warps = ss::kWarpRowThreads / 32;
     // warps past M zero the padding rows of the last 128-row metadata tile
     const unsigned grid = static_cast<unsigned>(((M + 127) / 128 * 128 + warps - 1) / warps);
+    // 8-bit tiers, bf16 rows split into 1, 2 or 4 chunks of up to 4096
+    // elements (a multiple of 32): X streams through shared memory once, the
+    // kept half of the row stays in registers
+    const int wpr = K <= ss::kPruneChunkMax ? 1 : (K <= 2 * ss::kPruneChunkMax ? 2 : 4);
+    if (in_dtype == SS_IN_BF16 && kq != ss::kQBf16 && K % (32 * wpr) == 0 &&
+        K <= 4 * ss::kPruneChunkMax && M <= (int64_t{1} << 30)) {
+        const int chunk_steps = static_cast<int>(K / wpr / 32);
+        const int last_steps = static_cast<int>(K_lp / 32) - (wpr - 1) * chunk_steps;
+        const int need = (std::max(chunk_steps, last_steps) + 31) / 32;
+        int dev_sms = 148;
+        cudaDeviceGetAttribute(&dev_sms, cudaDevAttrMultiProcessorCount, dev);
+        const int rows_per_cta = (ss::kWarpRowThreads / 32) / wpr;
+        const int64_t M_pad = (M + 127) / 128 * 128;
+        const unsigned pgrid = static_cast<unsigned>(
+            std::min<int64_t>(dev_sms, (M_pad + rows_per_cta - 1) / rows_per_cta));
+        const auto* xb = static_cast<const __nv_bfloat16*>(X);
+        const int Mi = static_cast<int>(M), Ki = static_cast<int>(K), Kl = static_cast<int>(K_lp);
+#define SS_PRUNE_ST(Q, S, W)                                                                  \
+    do {                                                                                      \
+        auto kern = ss::prune_act_stream_kernel<Q, S, W>;                                     \
+        if ((st = set_smem(kern, dev, ss::kPruneSmem)) != SS_OK) return st;                   \
+        return launch_ex(kern, dim3(pgrid), dim3(ss::kWarpRowThreads), ss::kPruneSmem, s, 1,  \
+                         xb, Mi, Ki, Kl, xv, xm, s_x);                                        \
+    } while (0)
+#define SS_PRUNE_ST_W(Q, W)                                                                   \
+    do {                                                                                      \
+        if (need <= 2) SS_PRUNE_ST(Q, 2, W);                                                  \
+        if (need <= 4) SS_PRUNE_ST(Q, 4, W);                                                  \
+        SS_PRUNE_ST(Q, 5, W);                                                                 \
+    } while (0)
+#define SS_PRUNE_ST_Q(Q)                                                                      \
+    do {                                                                                      \
+        if (wpr == 1) SS_PRUNE_ST_W(Q, 1);                                                    \
+        if (wpr == 2) SS_PRUNE_ST_W(Q, 2);                                                    \
+        SS_PRUNE_ST_W(Q, 4);                                                                  \
+    } while (0)
+        if (kq == ss::kQInt8) SS_PRUNE_ST_Q(ss::kQInt8);
+        SS_PRUNE_ST_Q(ss::kQE4M3);
+#undef SS_PRUNE_ST_Q
+#undef SS_PRUNE_ST_W
+#undef SS_PRUNE_ST
+    }
 #define SS_PRUNE(T, Q)                                                                         \
     do {                                                                                      \
         st = launch_ex(ss::prune_act_warp_kernel<T, Q>, dim3(grid), dim3(ss::kWarpRowThreads), \

@@ -388,6 +388,157 @@ __global__ void __launch_bounds__(kWarpRowThreads) prune_act_warp_kernel(
     }
 }
 
+// Single-pass online 2:4 prune of bf16 rows (8-bit tiers), streamed through
+// shared memory.  A row is split into kWpr chunks of C = K / kWpr elements
+// (C a multiple of 32, at most kChunkMax); the kWpr warps of a row slot each
+// take one chunk.  Each warp owns kSlots shared-memory slots and keeps the
+// 1-D bulk copies of its next chunks in flight while it works on the current
+// one, so X is read from HBM once at full overlap:
+//   - select: lane l takes the 32-element steps l, l + 32, ... of the chunk
+//     (8 groups of 4 each) from shared memory, keeps the top-2 of every group
+//     in registers as bf16 pairs, and the nibbles;
+//   - the row absmax is the largest kept magnitude (the largest element of
+//     every group is kept), combined across the row's warps through shared
+//     memory;
+//   - quantise the kept values from registers and store values and nibbles.
+// Steps past K up to K_lp are groups of zeros: values 0, nibble 0x4.  Rows
+// are taken in a grid-stride loop; padding rows (M <= m < M_pad) only zero
+// their metadata.
+constexpr int kPruneChunkMax = 4096;  // elements per chunk (8 KB of bf16)
+constexpr int kPruneSlots = 3;
+constexpr int kPruneSmem = 8 * kPruneSlots * kPruneChunkMax * 2;  // 8 warps
+
+template <int kQ, int kSteps, int kWpr>
+__global__ void __launch_bounds__(kWarpRowThreads, 1) prune_act_stream_kernel(
+    const __nv_bfloat16* __restrict__ X, int M, int K, int K_lp, uint8_t* __restrict__ Xv,
+    uint8_t* __restrict__ Xm, float* __restrict__ s_x) {
+    constexpr bool kInt8 = kQ == kQInt8;
+    constexpr int kRowsPerCta = kWarpRowThreads / (32 * kWpr);
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    __shared__ uint64_t full[8][kPruneSlots];
+    __shared__ float part[2][kRowsPerCta][kWpr];
+    __shared__ int abort_flag_storage;
+    volatile int* abort_flag = &abort_flag_storage;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int slot = warp / kWpr, sub = warp % kWpr;
+    const int chunk = K / kWpr;           // elements of this warp's chunk
+    const int chunk_steps = chunk / 32;   // full steps in the chunk
+    const int n_steps = K_lp / 32;        // steps of a row (K and its padding)
+    const int M_pad = (M + 127) / 128 * 128;
+    const int rows_total = static_cast<int>(gridDim.x) * kRowsPerCta;
+    uint8_t* my_smem = smem_raw + warp * (kPruneSlots * kPruneChunkMax * 2);
+    if (threadIdx.x == 0) *abort_flag = 0;
+    if (lane == 0) {
+        for (int b = 0; b < kPruneSlots; ++b) mbar_init(&full[warp][b], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    pdl_trigger();
+    pdl_wait();
+    const int m0 = static_cast<int>(blockIdx.x) * kRowsPerCta + slot;
+    // the copy of this warp's chunk of row m into buffer b
+    uint32_t pending = 0;  // buffers with a copy in flight (lane 0's view)
+    bool ok = true;
+    auto issue = [&](int m, int b) {
+        if (m < M && ok && lane == 0) {
+            fence_async_shared();  // this warp's reads of the buffer come first
+            pending |= 1u << b;
+            mbar_arrive_expect_tx(&full[warp][b], static_cast<uint32_t>(chunk * 2));
+            bulk_load_1d(my_smem + b * (kPruneChunkMax * 2),
+                         X + static_cast<int64_t>(m) * K + static_cast<int64_t>(sub) * chunk,
+                         static_cast<uint32_t>(chunk * 2), &full[warp][b]);
+        }
+    };
+#pragma unroll
+    for (int b = 0; b < kPruneSlots - 1; ++b) issue(m0 + b * rows_total, b);
+    int it = 0;
+    for (int m = m0; m < M_pad; m += rows_total, ++it) {
+        const int b = it % kPruneSlots;
+        // the slot of item it + kPruneSlots - 1 was last read in iteration it - 1
+        __syncwarp();
+        issue(m + (kPruneSlots - 1) * rows_total, (it + kPruneSlots - 1) % kPruneSlots);
+        if (m >= M) {  // padding row of the last 128-row metadata tile
+            for (int st = sub * 32 + lane; st < n_steps; st += 32 * kWpr)
+                __stcs(reinterpret_cast<uint32_t*>(Xm + meta_offset(m, 4 * st, K_lp)), 0u);
+            continue;
+        }
+        const bool got = ok && mbar_wait(&full[warp][b],
+                                         static_cast<uint32_t>((it / kPruneSlots) & 1), abort_flag);
+        if (!__all_sync(0xffffffffu, got)) ok = false;
+        if (got) pending &= ~(1u << b);
+        const uint4* c4 = reinterpret_cast<const uint4*>(my_smem + b * (kPruneChunkMax * 2));
+        uint32_t kept[kSteps][8];
+        uint32_t nib[kSteps];
+        uint32_t amax_bits = 0;  // |bf16| bit patterns order as the magnitudes
+#pragma unroll
+        for (int i = 0; i < kSteps; ++i) {
+            const int ls = 32 * i + lane;  // step within the chunk
+            uint32_t w[16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint4 v = (ok && ls < chunk_steps) ? c4[4 * ls + j] : make_uint4(0u, 0u, 0u, 0u);
+                w[4 * j] = v.x, w[4 * j + 1] = v.y, w[4 * j + 2] = v.z, w[4 * j + 3] = v.w;
+            }
+            uint32_t nibs = 0;
+#pragma unroll
+            for (int gi = 0; gi < 8; ++gi) {
+                int i0, i1;
+                const uint32_t k = top2_of4_bf16(w[2 * gi], w[2 * gi + 1], i0, i1);
+                kept[i][gi] = k;
+                amax_bits = max(amax_bits, max(k & 0x7FFFu, (k >> 16) & 0x7FFFu));
+                nibs |= static_cast<uint32_t>(i0 | (i1 << 2)) << (4 * gi);
+            }
+            nib[i] = nibs;  // steps past the chunk: zeros, indices 0, 1
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            amax_bits = max(amax_bits, __shfl_xor_sync(0xffffffffu, amax_bits, o));
+        float a = __uint_as_float(amax_bits << 16);
+        if constexpr (kWpr > 1) {
+            if (lane == 0) part[it & 1][slot][sub] = a;
+            named_bar_sync(1 + slot, 32 * kWpr);
+#pragma unroll
+            for (int w = 0; w < kWpr; ++w) a = fmaxf(a, part[it & 1][slot][w]);
+        }
+        float inv, s;
+        scale_from_absmax<kInt8>(a, inv, s);
+        if (lane == 0 && sub == 0) s_x[m] = s;
+        uint4* vout = reinterpret_cast<uint4*>(Xv + static_cast<int64_t>(m) * (K_lp / 2));
+#pragma unroll
+        for (int i = 0; i < kSteps; ++i) {
+            // the chunk's steps, then (last warp of the row) the padding steps
+            const int ls = 32 * i + lane;
+            const int st = sub * chunk_steps + ls;
+            const bool mine = ls < chunk_steps || (sub == kWpr - 1 && st < n_steps);
+            if (mine) {
+                uint32_t vals[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const uint32_t q0 = quantize_pair<kInt8>(
+                        __uint_as_float(kept[i][2 * h] << 16),
+                        __uint_as_float(kept[i][2 * h] & 0xFFFF0000u), inv);
+                    const uint32_t q1 = quantize_pair<kInt8>(
+                        __uint_as_float(kept[i][2 * h + 1] << 16),
+                        __uint_as_float(kept[i][2 * h + 1] & 0xFFFF0000u), inv);
+                    vals[h] = q0 | (q1 << 16);
+                }
+                __stcs(vout + st, make_uint4(vals[0], vals[1], vals[2], vals[3]));
+                __stcs(reinterpret_cast<uint32_t*>(Xm + meta_offset(m, 4 * st, K_lp)), nib[i]);
+            }
+        }
+    }
+    // after a wait that ran out: copies still in flight land before exit
+    __syncwarp();
+    if (lane == 0 && pending) {
+        for (int b = 0; b < kPruneSlots; ++b)
+            if ((pending >> b) & 1u) {
+                const uint64_t t0 = global_timer_ns();
+                while (global_timer_ns() - t0 < 1000000ull) {  // 1 ms
+                }
+            }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Single-pass variants for bf16 rows of up to kRegK elements: the whole row
 // sits in registers (16 bytes x 2 x 8 per lane), so X is read from HBM once.

@@ -75,6 +75,21 @@ def test_prune_act_2to4_many_rows(q, M, K):
     np.testing.assert_array_equal(host(Xv), Xv_ref)
 
 
+# The single-pass prune kernel (bf16 rows, K % 32 == 0): 1 warp per row with
+# 1, 4 and 8 steps of 32 elements per lane, 2 warps with 7 and 8, 4 warps
+# with 8; K = 96 and 160 leave zero-filled padding steps up to K_lp.
+@pytest.mark.parametrize("q", ["int8", "fp8"])
+@pytest.mark.parametrize("M,K", [(300, 96), (257, 160), (2000, 1024), (3000, 4096),
+                                 (1000, 8192), (700, 14336), (600, 16384), (200, 32768)])
+def test_prune_act_2to4_register_rows(q, M, K):
+    X = synth.gaussian_with_heavy_tails(M, K, seed=K + 1)
+    Xv_ref, Xm_ref, s_ref = oracle.prune_act_2to4(X, Q[q])
+    Xv, Xm, s_x = ss.prune_act_2to4(dev(X), q)
+    np.testing.assert_array_equal(host(s_x), s_ref)
+    np.testing.assert_array_equal(host(Xm), oracle.meta_to_tiles(Xm_ref, Xv_ref.shape[1] * 2))
+    np.testing.assert_array_equal(host(Xv), Xv_ref)
+
+
 @pytest.mark.parametrize("pat", ["dense"] + PATTERNS)
 @pytest.mark.parametrize("q", ["int8", "fp8"])
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
