@@ -608,47 +608,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                 for (int cb = 0; cb < kCpg; cb += kBatch) {
                     // 1) the batch's chunks into registers as packed bf16
-                    //    ([chunk][half][column group r * 2 + channel block])
+                    //    ([chunk][half][column group r * 2 + channel block]):
+                    //    every tensor-memory read of the batch is issued first and
+                    //    waited for once; with one accumulator it is released right
+                    //    then (2), before the conversion, so the next tile's MMAs
+                    //    need not wait for it
                     uint32_t pk[kBatch][2][8];
+                    uint32_t v[kBatch][2][16];
 #pragma unroll
                     for (int cc = 0; cc < kBatch; ++cc) {
                         const int c = 32 * grp + 64 * (cb + cc);
                         if (c < args.bn) {
-                            // token scales first: their loads overlap the TMEM reads
-                            float sb[4][2];
-#pragma unroll
-                            for (int r = 0; r < 4; ++r)
-#pragma unroll
-                                for (int e = 0; e < 2; ++e) {
-                                    const int tok = b0 + c + 8 * r + 2 * tm + e;
-                                    sb[r][e] = load_b_scale<kQ>(args.s_b, tok, tok < args.rowsB);
-                                }
-                            uint32_t v[2][16];
-                            tmem_ld_16x256b_x4(t_row + c, v[0]);
-                            tmem_ld_16x256b_x4(t_row + (16u << 16) + c, v[1]);
-                            tmem_ld_wait();
-#pragma unroll
-                            for (int h = 0; h < 2; ++h)
-#pragma unroll
-                                for (int r = 0; r < 4; ++r)
-#pragma unroll
-                                    for (int e = 0; e < 2; ++e) {
-                                        float y2[2];
-#pragma unroll
-                                        for (int k = 0; k < 2; ++k) {
-                                            const uint32_t bits = v[h][4 * r + 2 * e + k];
-                                            const float accv =
-                                                kInt8 ? __int2float_rn(static_cast<int32_t>(bits))
-                                                      : __uint_as_float(bits);
-                                            y2[k] = __fmul_rn(__fmul_rn(accv, sb[r][k]), sa2[h][e]);
-                                        }
-                                        const __nv_bfloat162 b2 =
-                                            __floats2bfloat162_rn(y2[0], y2[1]);
-                                        pk[cc][h][2 * r + e] =
-                                            *reinterpret_cast<const uint32_t*>(&b2);
-                                    }
+                            tmem_ld_16x256b_x4(t_row + c, v[cc][0]);
+                            tmem_ld_16x256b_x4(t_row + (16u << 16) + c, v[cc][1]);
                         }
                     }
+                    tmem_ld_wait();
                     // 2) after the group's last read of the accumulator: release its part
                     if (32 * grp + 64 * (cb + kBatch) >= args.bn &&
                         32 * grp + 64 * cb < args.bn) {
@@ -659,6 +634,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                 mbar_arrive_cluster(acc_empty_leader + acc * sizeof(uint64_t));
                             else
                                 mbar_arrive(&acc_empty[acc]);
+                        }
+                    }
+#pragma unroll
+                    for (int cc = 0; cc < kBatch; ++cc) {
+                        const int c = 32 * grp + 64 * (cb + cc);
+                        if (c < args.bn) {
+                            float sb[4][2];  // the chunk's token scales
+#pragma unroll
+                            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                                for (int e = 0; e < 2; ++e) {
+                                    const int tok = b0 + c + 8 * r + 2 * tm + e;
+                                    sb[r][e] = load_b_scale<kQ>(args.s_b, tok, tok < args.rowsB);
+                                }
+#pragma unroll
+                            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                                    for (int e = 0; e < 2; ++e) {
+                                        float y2[2];
+#pragma unroll
+                                        for (int k = 0; k < 2; ++k) {
+                                            const uint32_t bits = v[cc][h][4 * r + 2 * e + k];
+                                            const float accv =
+                                                kInt8 ? __int2float_rn(static_cast<int32_t>(bits))
+                                                      : __uint_as_float(bits);
+                                            y2[k] = __fmul_rn(__fmul_rn(accv, sb[r][k]), sa2[h][e]);
+                                        }
+                                        const __nv_bfloat162 b2 =
+                                            __floats2bfloat162_rn(y2[0], y2[1]);
+                                        pk[cc][h][2 * r + e] =
+                                            *reinterpret_cast<const uint32_t*>(&b2);
+                                    }
                         }
                     }
                     // 3) stage and store the batch
