@@ -421,7 +421,8 @@ def measure(path: Path, steps: int, warmup: int, dist: Dist, peaks: dict):
     launches0 = ss.ss_kernel_launches()
     with ClockSampler(torch.cuda.current_device()) as clk:
         sp_total, _, _ = time_loop(path.sparse_step, steps, warmup, flush, split=False)
-    launches = ss.ss_kernel_launches() - launches0 - 2 * warmup
+    # every step (warm-up or timed) launches the same kernels
+    launches = (ss.ss_kernel_launches() - launches0) * steps // (steps + warmup)
     dn_total, _, _ = time_loop(path.dense_step, steps, warmup, flush, split=False)
     # the per-kernel split (an event between the two kernels) in separate runs
     _, sp_act, sp_gemm = time_loop(path.sparse_step, steps, warmup, flush)
@@ -670,7 +671,8 @@ def main():
                      "unit": "TFLOP/s", "frac": r["sparse_gemm_tflops"] / r["sparse_peak"],
                      "peak_source": f"{peaks['source']} bf16 burst x"
                                     f"{r['sparse_peak'] / peaks['bf16_tflops']:.0f}"
-                                    + (" (2:4 x2)" if path.q == "bf16" else " (8-bit x2, 2:4 x2)"),
+                                    + {"bf16": " (2:4 x2)", "nvfp4": " (FP4 x4, 2:4 x2)"}.get(
+                                        path.q, " (8-bit x2, 2:4 x2)"),
                      "traffic": traffic,
                      "traffic_source": ({"profile": tr["profile"], "csrc_hash": tr["csrc_hash"]}
                                         if traffic is not None else None)},
