@@ -1073,20 +1073,20 @@ ss_status ss_get_device_status(ss_stream_t stream) {
 }
 
 ss_status ss_debug_set_wait_limit(uint64_t ns) {
+    if (ns < 1000000ull || ns > 60000000000ull) return SS_ERR_INVALID_ARG;  // 1 ms .. 60 s
     int dev;
     ss_status st = check_device(&dev);
     if (st != SS_OK) return st;
-    if (ns < 1000000ull || ns > 60000000000ull) return SS_ERR_INVALID_ARG;  // 1 ms .. 60 s
     if (cudaDeviceSynchronize() != cudaSuccess) return SS_ERR_CUDA;
     if (cudaMemcpyToSymbol(ss::g_wait_limit_ns, &ns, sizeof(ns)) != cudaSuccess) return SS_ERR_CUDA;
     return SS_OK;
 }
 
 ss_status ss_debug_skip_stage(int32_t kb) {
+    if (kb < -1) return SS_ERR_INVALID_ARG;
     int dev;
     ss_status st = check_device(&dev);
     if (st != SS_OK) return st;
-    if (kb < -1) return SS_ERR_INVALID_ARG;
     if (cudaDeviceSynchronize() != cudaSuccess) return SS_ERR_CUDA;
     if (cudaMemcpyToSymbol(ss::g_skip_stage, &kb, sizeof(kb)) != cudaSuccess) return SS_ERR_CUDA;
     return SS_OK;

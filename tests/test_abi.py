@@ -242,3 +242,26 @@ def test_meta_bytes_rejects_bad_shapes(L):
     assert ss.ss_meta_bytes(0, 128) == 0
     assert ss.ss_meta_bytes(5, 100) == 0
     assert ss.ss_meta_bytes(5, 0) == 0
+
+
+def test_debug_hooks_reject_bad_arguments_before_the_device(L):
+    """The test hooks validate their argument before touching the device:
+    a wait limit outside 1 ms .. 60 s and a stage below -1 are refused."""
+    assert L.ss_debug_set_wait_limit(999_999) == ss.SS_ERR_INVALID_ARG
+    assert L.ss_debug_set_wait_limit(60_000_000_001) == ss.SS_ERR_INVALID_ARG
+    assert L.ss_debug_skip_stage(-2) == ss.SS_ERR_INVALID_ARG
+
+
+def test_stored_traffic_is_tied_to_the_sources():
+    """bench.py reports a stored DRAM-traffic figure only while the CUDA
+    sources hash as they did when it was captured."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    h = bench.csrc_hash()
+    assert len(h) == 16 and int(h, 16) >= 0
+    for key, tr in bench.TRAFFIC.items():
+        assert set(tr) == {"bytes", "profile", "csrc_hash"}, key
+        assert os.path.exists(os.path.join(ROOT, tr["profile"])), tr["profile"]
+        assert tr["bytes"] > 0
