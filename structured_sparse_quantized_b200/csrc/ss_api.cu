@@ -384,6 +384,23 @@ int choose_bn(int64_t rowsB, int bn_max) {
     return static_cast<int>(r < bn_max ? r : bn_max);
 }
 
+// Groups the GEMM kernels walk the A tiles in (tile_coords).  A wave of CTA
+// pairs works on consecutive tiles: with g groups it re-reads 1/g of A and
+// touches about units * g / nA B tiles.  The smallest g whose per-wave set
+// (A / g plus those B tiles) fits in 40 MB keeps A in L2 across waves at the
+// cost of reading B g times; if no g fits (B tiles of long rows), one group
+// reads B once.  Measured on B200: Llama-3.1-8B gate/up 6:8 INT8, M = 16384
+// (A 55 MB, B tiles 2.75 MB): one group 551-561 us, two 528-535 us, four
+// 549 us; the down projection (B tiles 9.6 MB) runs best as one group.
+int a_groups_for(int64_t a_bytes, int64_t nA, int64_t units, int64_t b_tile_bytes) {
+    const int64_t budget = int64_t{40} << 20;
+    for (int64_t g = 1; g <= 8 && g <= nA; ++g) {
+        const int64_t b_tiles = (units * g + nA - 1) / nA;
+        if ((a_bytes + g - 1) / g + b_tiles * b_tile_bytes <= budget) return static_cast<int>(g);
+    }
+    return 1;
+}
+
 // Opt a row kernel into more than 48 KB of dynamic shared memory when needed.
 template <typename Kern>
 ss_status set_smem(Kern kern, int /*dev*/, size_t bytes) {
@@ -735,6 +752,9 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
     args.ldy = static_cast<int>(N);
     args.e_chunks = static_cast<int>(K_lp / 128);
     args.sf_k = 0;
+    // values + selectors of A; B tiles of bn rows (the wide kernel sets its own)
+    args.a_groups = a_groups_for(rowsA * (K_lp / 2 * eb + K_lp / 8), (rowsA + 255) / 256,
+                                 g_num_sms[dev] / 2, static_cast<int64_t>(bn) * K_lp * eb);
     args.s_a = s_a;
     args.s_b = s_b;
     args.y = Y;
@@ -765,6 +785,8 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
             return SS_ERR_CUDA;
         ss::GemmArgs wargs = args;
         wargs.bn = bnw;
+        wargs.a_groups = a_groups_for(rowsA * (K_lp / 2 + K_lp / 8), (rowsA + 255) / 256,
+                                      g_num_sms[dev] / 2, 2 * static_cast<int64_t>(bnw) * K_lp);
         wargs.k_stages = static_cast<int>(K_lp / CW::kStageK);
         if (args.a_is_w)
             return i8 ? launch_gemm_wide<true, true>(dev, wa, wb, te, ty, wargs, st_)
@@ -808,6 +830,8 @@ ss_status ss_dense_gemm(const void* Xq, const float* s_x, const void* Wq, const 
     args.ldy = static_cast<int>(N);
     args.e_chunks = 0;
     args.sf_k = 0;
+    args.a_groups = a_groups_for(N * K_p * eb, (N + 255) / 256, g_num_sms[dev] / 2,
+                                 static_cast<int64_t>(bn) * K_p * eb);
     args.s_a = s_w;
     args.s_b = s_x;
     args.y = Y;
@@ -1020,6 +1044,10 @@ ss_status gemm_nvfp4(const void* Av, const void* Am, const void* As, const float
     args.ldy = static_cast<int>(N);
     args.e_chunks = static_cast<int>(K_lp / 256);
     args.sf_k = static_cast<int>(nblk / 4);
+    // codes, block scales and (sparse) selectors of the weight
+    args.a_groups = a_groups_for(N * (kSparse ? K_lp / 4 + K_lp / 16 : K_lp / 2) + N * nblk,
+                                 (N + 255) / 256, g_num_sms[dev] / 2,
+                                 static_cast<int64_t>(bn) * (K_lp / 2 + K_lp / 16));
     args.s_a = g_w;
     args.s_b = g_x;
     args.y = Y;

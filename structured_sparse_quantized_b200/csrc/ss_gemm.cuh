@@ -181,6 +181,7 @@ struct GemmArgs {
     int e_chunks;     // K_lp / 128: 2 KB metadata tiles per 128 rows (tile-major)
                       // (block-scaled FP4: K_lp / 256)
     int sf_k;         // FP4: MMA k-blocks per 128-row scale tile (4 scales each)
+    int a_groups;     // A tiles are walked in this many groups (tile_coords)
     const float* s_a;
     const float* s_b;
     void* y;
@@ -196,6 +197,28 @@ __device__ __forceinline__ void store_scaled(void* y, int64_t off, uint32_t acc_
         reinterpret_cast<__nv_bfloat16*>(y)[off] = __float2bfloat16_rn(v);
     else
         reinterpret_cast<float*>(y)[off] = v;
+}
+
+// Output tile t -> (A tile ta, B tile tb).  Consecutive tiles (the ones a
+// wave of CTA pairs works on together) take consecutive A tiles for the same
+// B tile(s), so each B tile is read from L2 by many pairs at once.  With
+// a_groups > 1 the A tiles are split into that many groups and a group's A
+// tiles are walked for every B tile before the next group starts: the slice
+// of A that every wave re-reads is 1/a_groups of it, small enough to stay in
+// L2 while the B tiles and Y stream through (the host picks a_groups from the
+// size of A).
+__device__ __forceinline__ void tile_coords(int t, int nA, int nB, int groups, int& ta, int& tb) {
+    if (groups <= 1) {
+        ta = t % nA;
+        tb = t / nA;
+        return;
+    }
+    const int G = (nA + groups - 1) / groups;  // A tiles per group (the last may have fewer)
+    const int g = t / (G * nB);
+    const int rows = min(G, nA - g * G);
+    const int r = t - g * G * nB;
+    ta = g * G + r % rows;
+    tb = r / rows;
 }
 
 // Scale of row i, or 1 for the unscaled bf16 tier (the product with 1.0f
@@ -296,7 +319,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (args.a_is_w && unit < n_tiles) {
                 // A (and its metadata) is the weight: start streaming the first
                 // tile's K stages into L2 while the previous kernel finishes.
-                const int a0 = (unit % nA) * tile_a_rows + static_cast<int>(rank) * kTileA;
+                int ta0, tb0;
+                tile_coords(unit, nA, nB, args.a_groups, ta0, tb0);
+                const int a0 = ta0 * tile_a_rows + static_cast<int>(rank) * kTileA;
                 const int n_pre = args.k_stages < kL2PrefetchStages ? args.k_stages
                                                                     : kL2PrefetchStages;
                 for (int kb = 0; kb < n_pre; ++kb) {
@@ -318,8 +343,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         bool ok = true;
         const int skip_kb = g_skip_stage;  // test hook, -1 in normal use
         for (int t = unit; t < n_tiles && ok; t += n_units) {
-            const int a0 = (t % nA) * tile_a_rows + static_cast<int>(rank) * kTileA;
-            const int b0 = (t / nA) * args.bn + static_cast<int>(rank) * b_rows_cta;
+            int ta, tb;
+            tile_coords(t, nA, nB, args.a_groups, ta, tb);
+            const int a0 = ta * tile_a_rows + static_cast<int>(rank) * kTileA;
+            const int b0 = tb * args.bn + static_cast<int>(rank) * b_rows_cta;
             for (int kb = 0; kb < args.k_stages; ++kb) {
                 if (t == unit && kb == skip_kb) {  // this stage is never loaded
                     ok = false;
@@ -349,7 +376,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             tma_load_2d_pair_hint(
                                 st + C::kSfaOffset, &tm_sfa, fb, 0,
                                 ((a0 >> 7) * args.sf_k + kb * C::kMmaPerStage) * 4, keep);
-                            const int sfb_tile = (t / nA) * args.bn >> 7;
+                            const int sfb_tile = tb * args.bn >> 7;
 #pragma unroll
                             for (int u = 0; u < C::kSfbTiles; ++u)  // past the last: zero fill
                                 tma_load_2d_pair_hint(
@@ -553,8 +580,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int i = 0;
         bool ok = true;
         for (int t = unit; t < n_tiles && ok; t += n_units, ++i) {
-            const int a_tile0 = (t % nA) * tile_a_rows + static_cast<int>(rank) * kTileA;
-            const int b0 = (t / nA) * args.bn;
+            int ta, tb;
+            tile_coords(t, nA, nB, args.a_groups, ta, tb);
+            const int a_tile0 = ta * tile_a_rows + static_cast<int>(rank) * kTileA;
+            const int b0 = tb * args.bn;
             const int acc = C::kAccBufs == 2 ? (i & 1) : 0;
             const uint32_t aph = C::kAccBufs == 2 ? ((i >> 1) & 1) : (i & 1);
             // the four warps of a group take the same decision, so none is

@@ -151,7 +151,9 @@ __global__ void __launch_bounds__(kWideThreads, 1)
             tma_prefetch_desc(&tm_e);
             const int t0 = snake_tile(0, unit, n_units);
             if (kAIsW && t0 < n_tiles) {  // the weight's first tile into L2
-                const int a0 = (t0 % nA) * kPairRows + static_cast<int>(rank) * kTileA;
+                int ta0, tb0;
+                tile_coords(t0, nA, nB, args.a_groups, ta0, tb0);
+                const int a0 = ta0 * kPairRows + static_cast<int>(rank) * kTileA;
                 const int n_pre = args.k_stages < 2 * kL2PrefetchStages ? args.k_stages
                                                                         : 2 * kL2PrefetchStages;
                 for (int kb = 0; kb < n_pre; ++kb) {
@@ -169,8 +171,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         const int skip_kb = g_skip_stage;  // test hook, -1 in normal use
         for (int k = 0, t = snake_tile(0, unit, n_units); t < n_tiles && ok;
              ++k, t = snake_tile(k, unit, n_units)) {
-            const int a0 = (t % nA) * kPairRows + static_cast<int>(rank) * kTileA;
-            const int b0 = (t / nA) * tile_b_rows + static_cast<int>(rank) * b_rows_cta;
+            int ta, tb;
+            tile_coords(t, nA, nB, args.a_groups, ta, tb);
+            const int a0 = ta * kPairRows + static_cast<int>(rank) * kTileA;
+            const int b0 = tb * tile_b_rows + static_cast<int>(rank) * b_rows_cta;
             for (int kb = 0; kb < args.k_stages; ++kb) {
                 if (k == 0 && kb == skip_kb) {  // this stage is never loaded
                     ok = false;
@@ -309,8 +313,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         uint32_t chunk_iter = 0;
         for (int t = snake_tile(0, unit, n_units); t < n_tiles;
              ++i, t = snake_tile(i, unit, n_units)) {
-            const int a_cta0 = (t % nA) * kPairRows + static_cast<int>(rank) * kTileA;
-            const int tile_tok0 = (t / nA) * tile_b_rows;
+            int ta, tb_;
+            tile_coords(t, nA, nB, args.a_groups, ta, tb_);
+            const int a_cta0 = ta * kPairRows + static_cast<int>(rank) * kTileA;
+            const int tile_tok0 = tb_ * tile_b_rows;
             const int tok0 = tile_tok0 + bt * args.bn;
             // scales of this tile, fetched while its MMAs still run
             float sb_pre[2];
