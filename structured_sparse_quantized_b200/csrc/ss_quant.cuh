@@ -96,7 +96,8 @@ __device__ __forceinline__ void top2_of4(const float* v, int& i0, int& i1) {
 // the same order as top2_of4 for every non-NaN input (|bf16| bit patterns
 // are monotone in the value).  Returns the two kept bf16 values, lower index
 // in the low half, picked with one byte permute.
-__device__ __forceinline__ uint32_t top2_of4_bf16(uint32_t lo, uint32_t hi, int& i0, int& i1) {
+__device__ __forceinline__ uint32_t top2_of4_bf16(uint32_t lo, uint32_t hi, int& i0, int& i1,
+                                                  uint32_t& top) {
     const uint32_t k0 = (lo & 0x7FFFu) * 4u + 3u;
     const uint32_t k1 = ((lo >> 16) & 0x7FFFu) * 4u + 2u;
     const uint32_t k2 = (hi & 0x7FFFu) * 4u + 1u;
@@ -104,12 +105,18 @@ __device__ __forceinline__ uint32_t top2_of4_bf16(uint32_t lo, uint32_t hi, int&
     const uint32_t a = max(k0, k1), b = min(k0, k1), c = max(k2, k3), d = min(k2, k3);
     const uint32_t first = max(a, c);                   // the largest key
     const uint32_t second = max(min(a, c), max(b, d));  // the second largest
+    top = first;  // |x| bits of the group's largest magnitude, times 4, plus a tie tag
     const int ia = static_cast<int>((first & 3u) ^ 3u), ib = static_cast<int>((second & 3u) ^ 3u);
     i0 = min(ia, ib);
     i1 = max(ia, ib);
     // bytes 2 i0, 2 i0 + 1 -> low half; 2 i1, 2 i1 + 1 -> high half
     const uint32_t sel = static_cast<uint32_t>(i0) * 0x22u + static_cast<uint32_t>(i1) * 0x2200u + 0x1010u;
     return __byte_perm(lo, hi, sel);
+}
+
+__device__ __forceinline__ uint32_t top2_of4_bf16(uint32_t lo, uint32_t hi, int& i0, int& i1) {
+    uint32_t top;
+    return top2_of4_bf16(lo, hi, i0, i1, top);
 }
 
 // Value at local index i (0..3) of a group, without indexing registers
@@ -469,7 +476,9 @@ __global__ void __launch_bounds__(kWarpRowThreads, 1) prune_act_stream_kernel(
         const uint4* c4 = reinterpret_cast<const uint4*>(my_smem + b * (kPruneChunkMax * 2));
         uint32_t kept[kSteps][8];
         uint32_t nib[kSteps];
-        uint32_t amax_bits = 0;  // |bf16| bit patterns order as the magnitudes
+        // the largest selection key (|bf16| bits * 4 + tie tag): |bf16| bit
+        // patterns order as the magnitudes, and the largest of every group is kept
+        uint32_t amax_key = 0;
 #pragma unroll
         for (int i = 0; i < kSteps; ++i) {
             const int ls = 32 * i + lane;  // step within the chunk
@@ -483,17 +492,17 @@ __global__ void __launch_bounds__(kWarpRowThreads, 1) prune_act_stream_kernel(
 #pragma unroll
             for (int gi = 0; gi < 8; ++gi) {
                 int i0, i1;
-                const uint32_t k = top2_of4_bf16(w[2 * gi], w[2 * gi + 1], i0, i1);
-                kept[i][gi] = k;
-                amax_bits = max(amax_bits, max(k & 0x7FFFu, (k >> 16) & 0x7FFFu));
+                uint32_t top;
+                kept[i][gi] = top2_of4_bf16(w[2 * gi], w[2 * gi + 1], i0, i1, top);
+                amax_key = max(amax_key, top);
                 nibs |= static_cast<uint32_t>(i0 | (i1 << 2)) << (4 * gi);
             }
             nib[i] = nibs;  // steps past the chunk: zeros, indices 0, 1
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
-            amax_bits = max(amax_bits, __shfl_xor_sync(0xffffffffu, amax_bits, o));
-        float a = __uint_as_float(amax_bits << 16);
+            amax_key = max(amax_key, __shfl_xor_sync(0xffffffffu, amax_key, o));
+        float a = __uint_as_float((amax_key >> 2) << 16);
         if constexpr (kWpr > 1) {
             if (lane == 0) part[it & 1][slot][sub] = a;
             named_bar_sync(1 + slot, 32 * kWpr);
