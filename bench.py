@@ -55,26 +55,31 @@ IDEAL = {"2:4": 2.0, "4:6": 1.5, "6:8": 4.0 / 3.0, "8:10": 1.25}
 # DRAM bytes per launch of the dominant kernel (dram__bytes_read.sum +
 # dram__bytes_write.sum of one sparse-GEMM launch) from one ncu capture.
 # Keyed by (workload, M, pattern, qdtype) as run; each entry names the
-# profile summary it comes from and the hash of the kernel sources
-# (csrc_hash()) it was captured with.  A stored figure is reported only while
-# the sources still hash the same; otherwise "traffic" is null.
+# profile summary it comes from, the sources that make up that kernel (its
+# device code and the host code that picks its shape) and their hash at
+# capture time (csrc_hash).  A stored figure is reported only while those
+# sources still hash the same; otherwise "traffic" is null.
+GEMM_SOURCES = ("ss_api.cu", "ss_common.cuh", "ss_gemm.cuh", "ss_gemm_wide.cuh")
 TRAFFIC = {
     ("llama_layer_gate_up", 16384, "6:8", "int8"): {
         "bytes": (294.49e6 + 431.61e6 + 294.55e6 + 426.82e6) / 2,
         "profile": "profiles/gemm_llama_gateup_6of8_int8_m16384.md",
-        "csrc_hash": "dc7ee292358cd27d"},
+        "sources": GEMM_SOURCES,
+        "csrc_hash": "bc7026cd653631e8"},
 }
 
 
-def csrc_hash() -> str:
-    """sha256 (first 16 hex digits) of the library's CUDA sources."""
+def csrc_hash(files=None) -> str:
+    """sha256 (first 16 hex digits) of the named CUDA sources (all of them
+    when files is None)."""
     import hashlib
     d = os.path.join(HERE, "structured_sparse_quantized_b200", "csrc")
+    names = sorted(files) if files else sorted(n for n in os.listdir(d)
+                                               if n.endswith((".cu", ".cuh")))
     h = hashlib.sha256()
-    for name in sorted(os.listdir(d)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(d, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in names:
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
@@ -653,8 +658,7 @@ def main():
     line = base_line(args, args.workload, args.m, n)
     wl = synth.WORKLOADS[args.workload]
     tr = TRAFFIC.get((args.workload, args.m, wl["pattern"], wl["qdtype"]))
-    src_hash = csrc_hash()
-    traffic = tr["bytes"] if tr and tr["csrc_hash"] == src_hash else None
+    traffic = tr["bytes"] if tr and tr["csrc_hash"] == csrc_hash(tr["sources"]) else None
     line.update({
         "value": value, "ms_per_step": r["t_step_ms"],
         "dtype": path.q,

@@ -262,6 +262,7 @@ def test_stored_traffic_is_tied_to_the_sources():
     h = bench.csrc_hash()
     assert len(h) == 16 and int(h, 16) >= 0
     for key, tr in bench.TRAFFIC.items():
-        assert set(tr) == {"bytes", "profile", "csrc_hash"}, key
+        assert set(tr) == {"bytes", "profile", "sources", "csrc_hash"}, key
+        assert len(bench.csrc_hash(tr["sources"])) == 16
         assert os.path.exists(os.path.join(ROOT, tr["profile"])), tr["profile"]
         assert tr["bytes"] > 0
