@@ -154,7 +154,8 @@ ss_status ss_prune_act_2to4(const void *X, ss_in_dtype in_dtype, int64_t M, int6
  *                     s_b = s_w [N].
  * acc is exact int32 for INT8 and fp32 (tensor-core accumulation) for E4M3
  * and SS_BF16 (kind::f16; Av, B hold 2-byte values, s_a / s_b unused).
- * K_lp must be a positive multiple of 128; M, N in [1, 2^31).
+ * K_lp must be a positive multiple of 128; M, N in [1, 2^31) (SS_ERR_UNSUPPORTED when the
+ * output-tile count passes 2^31).
  * Kernel shape: with more than 128 weight rows and bf16 Y, large problems
  * run output tiles of 256 channels x 2 token tiles (one A slice feeds two
  * MMAs), the rest (and every SS_BF16 problem) 256 x 1.  The choice follows the wave count; the
@@ -223,7 +224,7 @@ ss_status ss_compress_weight_nvfp4(const void *W, ss_in_dtype in_dtype, int64_t 
                                    ss_pattern p, void *Wv, void *Wm, void *Ws, float *g_w,
                                    ss_stream_t stream);
 
-/* NVFP4 activation: ONE global scale for the tensor, g_x[0] = amax(X) / 2688
+/* NVFP4 activation (M up to 2^30 rows): ONE global scale for the tensor, g_x[0] = amax(X) / 2688
  * (the NVFP4 row: a global scale per tensor; the page calibrates it on a
  * data set, and with none here it is taken from this call's X, so the call
  * first reduces |X| over all M x K elements), the pair lift of pattern p,

@@ -401,6 +401,12 @@ int a_groups_for(int64_t a_bytes, int64_t nA, int64_t units, int64_t b_tile_byte
     return 1;
 }
 
+// The GEMM kernels count output tiles (A tiles of 128 or 256 rows x B tiles
+// of bn rows) in 32-bit integers.
+bool tiles_overflow(int64_t rowsA, int64_t rowsB, int bn) {
+    return (rowsA + 127) / 128 * ((rowsB + bn - 1) / bn) > INT32_MAX;
+}
+
 // Opt a row kernel into more than 48 KB of dynamic shared memory when needed.
 template <typename Kern>
 ss_status set_smem(Kern kern, int /*dev*/, size_t bytes) {
@@ -730,6 +736,7 @@ ss_status ss_sparse_gemm(int sparse_operand, const void* Av, const void* Am, con
     const int64_t rowsB = sparse_operand == 0 ? M : N;
     const int pair = rowsA > ss::kTileA ? 2 : 1;
     const int bn = choose_bn(rowsB, ss::GemmCfg<true, 1>::kBnMax);
+    if (tiles_overflow(rowsA, rowsB, bn)) return SS_ERR_UNSUPPORTED;
     // operand element bytes: the maps address bytes, so a bf16 row is twice as wide
     const int64_t eb = scaled ? 1 : 2;
     CUtensorMap ta, tb, te;
@@ -816,6 +823,7 @@ ss_status ss_dense_gemm(const void* Xq, const float* s_x, const void* Wq, const 
     if (st != SS_OK) return st;
     const int pair = N > ss::kTileA ? 2 : 1;
     const int bn = choose_bn(M, ss::GemmCfg<false, 1>::kBnMax);
+    if (tiles_overflow(N, M, bn)) return SS_ERR_UNSUPPORTED;
     const int64_t eb = scaled ? 1 : 2;  // operand element bytes
     CUtensorMap ta, tb;
     if (!make_map_2d(&ta, Wq, N, K_p * eb, ss::kTileA, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -1020,6 +1028,7 @@ ss_status gemm_nvfp4(const void* Av, const void* Am, const void* As, const float
     const int pair = N > ss::kTileA && (!kSparse || K_lp > 2048) ? 2 : 1;
     const int bn_max = pair == 2 ? ss::Fp4Cfg<kSparse, 2>::kBnMax : C::kBnMax;
     const int bn = M <= bn_max ? static_cast<int>(round_up(M, 32)) : bn_max;
+    if (tiles_overflow(N, M, bn)) return SS_ERR_UNSUPPORTED;
     const int64_t a_bytes = kSparse ? K_lp / 4 : K_lp / 2;  // bytes per A row
     const int64_t nblk = K_lp / block;
     CUtensorMap ta, tb, te, tsa, tsb;
