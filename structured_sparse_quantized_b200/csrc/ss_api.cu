@@ -673,18 +673,24 @@ ss_status ss_prune_act_2to4(const void* X, ss_in_dtype in_dtype, int64_t M, int6
             std::min<int64_t>(dev_sms, (M_pad + rows_per_cta - 1) / rows_per_cta));
         const auto* xb = static_cast<const __nv_bfloat16*>(X);
         const int Mi = static_cast<int>(M), Ki = static_cast<int>(K), Kl = static_cast<int>(K_lp);
-#define SS_PRUNE_ST(Q, S, W)                                                                  \
+#define SS_PRUNE_ST(Q, S, W, F)                                                               \
     do {                                                                                      \
-        auto kern = ss::prune_act_stream_kernel<Q, S, W>;                                     \
+        auto kern = ss::prune_act_stream_kernel<Q, S, W, F>;                                  \
         if ((st = set_smem(kern, dev, ss::kPruneSmem)) != SS_OK) return st;                   \
         return launch_ex(kern, dim3(pgrid), dim3(ss::kWarpRowThreads), ss::kPruneSmem, s, 1,  \
-                         xb, Mi, Ki, Kl, xv, xm, s_x);                                        \
+                         xb, Mi, Ki, Kl, xv, xm, s_x, 1u);                                    \
     } while (0)
+        // full: the chunks fill exactly S steps per lane and there are no
+        // padding steps
+        const bool full2 = K_lp == K && chunk_steps == 64;
+        const bool full4 = K_lp == K && chunk_steps == 128;
 #define SS_PRUNE_ST_W(Q, W)                                                                   \
     do {                                                                                      \
-        if (need <= 2) SS_PRUNE_ST(Q, 2, W);                                                  \
-        if (need <= 4) SS_PRUNE_ST(Q, 4, W);                                                  \
-        SS_PRUNE_ST(Q, 5, W);                                                                 \
+        if (full2) SS_PRUNE_ST(Q, 2, W, true);                                                \
+        if (full4) SS_PRUNE_ST(Q, 4, W, true);                                                \
+        if (need <= 2) SS_PRUNE_ST(Q, 2, W, false);                                           \
+        if (need <= 4) SS_PRUNE_ST(Q, 4, W, false);                                           \
+        SS_PRUNE_ST(Q, 5, W, false);                                                          \
     } while (0)
 #define SS_PRUNE_ST_Q(Q)                                                                      \
     do {                                                                                      \

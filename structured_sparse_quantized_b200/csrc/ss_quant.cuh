@@ -119,6 +119,30 @@ __device__ __forceinline__ uint32_t top2_of4_bf16(uint32_t lo, uint32_t hi, int&
     return top2_of4_bf16(lo, hi, i0, i1, top);
 }
 
+// top2_of4_bf16 for the streaming prune kernel, which is bound by the
+// integer ALU pipe: the keys are built with multiply-adds (FMA pipe) by the
+// multipliers c2 = 2 and c17 = 2^17, which the caller passes in registers the
+// compiler cannot fold.  key_i = |x_i| bits in bits 31..17, tie tag 3 - i in
+// bits 1..0 (x_0 * 2^17 drops its sign bit and x_1; (x_1's half) * 2 drops
+// its sign bit): the same order as top2_of4_bf16.  Returns the kept pair
+// (lower index in the low half), the nibble i0 | i1 << 2 and the largest key.
+__device__ __forceinline__ uint32_t top2_of4_bf16_keys(uint32_t lo, uint32_t hi, uint32_t c2,
+                                                       uint32_t c17, uint32_t& nib,
+                                                       uint32_t& top) {
+    const uint32_t k0 = lo * c17 + 3u;
+    const uint32_t k1 = (lo & 0xFFFF0000u) * c2 + 2u;
+    const uint32_t k2 = hi * c17 + 1u;
+    const uint32_t k3 = (hi & 0xFFFF0000u) * c2;
+    const uint32_t a = max(k0, k1), b = min(k0, k1), c = max(k2, k3), d = min(k2, k3);
+    const uint32_t first = max(a, c);
+    const uint32_t second = max(min(a, c), max(b, d));
+    top = first;
+    const uint32_t ia = (first & 3u) ^ 3u, ib = (second & 3u) ^ 3u;
+    const uint32_t i0 = min(ia, ib), i1 = max(ia, ib);
+    nib = i1 * 4u + i0;
+    return __byte_perm(lo, hi, i0 * 0x22u + i1 * 0x2200u + 0x1010u);
+}
+
 // Value at local index i (0..3) of a group, without indexing registers
 // dynamically.
 __device__ __forceinline__ float pick4(const float* v, int i) {
@@ -415,11 +439,17 @@ constexpr int kPruneChunkMax = 4096;  // elements per chunk (8 KB of bf16)
 constexpr int kPruneSlots = 3;
 constexpr int kPruneSmem = 8 * kPruneSlots * kPruneChunkMax * 2;  // 8 warps
 
-template <int kQ, int kSteps, int kWpr>
+// kFull: every warp's chunk is exactly kSteps steps per lane and K_lp = K
+// (no bounds test on the loads, no padding steps).  `one` is 1: the
+// multipliers built from it are opaque to the compiler, so that products
+// with them stay multiply-adds on the FMA pipe.
+template <int kQ, int kSteps, int kWpr, bool kFull>
 __global__ void __launch_bounds__(kWarpRowThreads, 1) prune_act_stream_kernel(
     const __nv_bfloat16* __restrict__ X, int M, int K, int K_lp, uint8_t* __restrict__ Xv,
-    uint8_t* __restrict__ Xm, float* __restrict__ s_x) {
+    uint8_t* __restrict__ Xm, float* __restrict__ s_x, uint32_t one) {
     constexpr bool kInt8 = kQ == kQInt8;
+    const uint32_t c2 = one << 1, c16 = one << 4, c17 = one << 17;
+    const uint32_t c65536 = one << 16;
     constexpr int kRowsPerCta = kWarpRowThreads / (32 * kWpr);
     extern __shared__ __align__(16) uint8_t smem_raw[];
     __shared__ uint64_t full[8][kPruneSlots];
@@ -473,10 +503,10 @@ __global__ void __launch_bounds__(kWarpRowThreads, 1) prune_act_stream_kernel(
                                          static_cast<uint32_t>((it / kPruneSlots) & 1), abort_flag);
         if (!__all_sync(0xffffffffu, got)) ok = false;
         if (got) pending &= ~(1u << b);
-        const uint4* c4 = reinterpret_cast<const uint4*>(my_smem + b * (kPruneChunkMax * 2));
+        const uint4* c4s = reinterpret_cast<const uint4*>(my_smem + b * (kPruneChunkMax * 2));
         uint32_t kept[kSteps][8];
         uint32_t nib[kSteps];
-        // the largest selection key (|bf16| bits * 4 + tie tag): |bf16| bit
+        // the largest selection key (|bf16| bits << 17 + tie tag): |bf16| bit
         // patterns order as the magnitudes, and the largest of every group is kept
         uint32_t amax_key = 0;
 #pragma unroll
@@ -485,24 +515,25 @@ __global__ void __launch_bounds__(kWarpRowThreads, 1) prune_act_stream_kernel(
             uint32_t w[16];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const uint4 v = (ok && ls < chunk_steps) ? c4[4 * ls + j] : make_uint4(0u, 0u, 0u, 0u);
+                const uint4 v = (kFull || ls < chunk_steps) ? c4s[4 * ls + j]
+                                                             : make_uint4(0u, 0u, 0u, 0u);
                 w[4 * j] = v.x, w[4 * j + 1] = v.y, w[4 * j + 2] = v.z, w[4 * j + 3] = v.w;
             }
+            // the nibbles of groups 7 .. 0, Horner-style in multiply-adds
             uint32_t nibs = 0;
 #pragma unroll
-            for (int gi = 0; gi < 8; ++gi) {
-                int i0, i1;
-                uint32_t top;
-                kept[i][gi] = top2_of4_bf16(w[2 * gi], w[2 * gi + 1], i0, i1, top);
+            for (int gi = 7; gi >= 0; --gi) {
+                uint32_t top, n;
+                kept[i][gi] = top2_of4_bf16_keys(w[2 * gi], w[2 * gi + 1], c2, c17, n, top);
                 amax_key = max(amax_key, top);
-                nibs |= static_cast<uint32_t>(i0 | (i1 << 2)) << (4 * gi);
+                nibs = nibs * c16 + n;
             }
             nib[i] = nibs;  // steps past the chunk: zeros, indices 0, 1
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
             amax_key = max(amax_key, __shfl_xor_sync(0xffffffffu, amax_key, o));
-        float a = __uint_as_float((amax_key >> 2) << 16);
+        float a = __uint_as_float((amax_key >> 17) << 16);
         if constexpr (kWpr > 1) {
             if (lane == 0) part[it & 1][slot][sub] = a;
             named_bar_sync(1 + slot, 32 * kWpr);
@@ -512,27 +543,39 @@ __global__ void __launch_bounds__(kWarpRowThreads, 1) prune_act_stream_kernel(
         float inv, s;
         scale_from_absmax<kInt8>(a, inv, s);
         if (lane == 0 && sub == 0) s_x[m] = s;
-        uint4* vout = reinterpret_cast<uint4*>(Xv + static_cast<int64_t>(m) * (K_lp / 2));
+        // this lane's first step; a step 32 further is 16 value bytes x 32 and
+        // eight 2 KB metadata tiles further
+        const int st0 = sub * chunk_steps + lane;
+        uint4* vout = reinterpret_cast<uint4*>(Xv + static_cast<int64_t>(m) * (K_lp / 2)) + st0;
+        uint32_t* mout = reinterpret_cast<uint32_t*>(Xm + meta_offset(m, 4 * st0, K_lp));
 #pragma unroll
         for (int i = 0; i < kSteps; ++i) {
             // the chunk's steps, then (last warp of the row) the padding steps
             const int ls = 32 * i + lane;
-            const int st = sub * chunk_steps + ls;
-            const bool mine = ls < chunk_steps || (sub == kWpr - 1 && st < n_steps);
+            const bool mine =
+                kFull || ls < chunk_steps || (sub == kWpr - 1 && st0 + 32 * i < n_steps);
             if (mine) {
                 uint32_t vals[4];
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
-                    const uint32_t q0 = quantize_pair<kInt8>(
-                        __uint_as_float(kept[i][2 * h] << 16),
-                        __uint_as_float(kept[i][2 * h] & 0xFFFF0000u), inv);
-                    const uint32_t q1 = quantize_pair<kInt8>(
-                        __uint_as_float(kept[i][2 * h + 1] << 16),
-                        __uint_as_float(kept[i][2 * h + 1] & 0xFFFF0000u), inv);
-                    vals[h] = q0 | (q1 << 16);
+                    const uint32_t p0 = kept[i][2 * h], p1 = kept[i][2 * h + 1];
+                    if constexpr (kInt8) {
+                        const uint32_t b0 = int8_code(__uint_as_float(p0 * c65536), inv);
+                        const uint32_t b1 = int8_code(__uint_as_float(p0 & 0xFFFF0000u), inv);
+                        const uint32_t b2 = int8_code(__uint_as_float(p1 * c65536), inv);
+                        const uint32_t b3 = int8_code(__uint_as_float(p1 & 0xFFFF0000u), inv);
+                        vals[h] = __byte_perm(__byte_perm(b0, b1, 0x0040),
+                                              __byte_perm(b2, b3, 0x0040), 0x5410);
+                    } else {
+                        const uint32_t q0 = quantize_pair<false>(
+                            __uint_as_float(p0 * c65536), __uint_as_float(p0 & 0xFFFF0000u), inv);
+                        const uint32_t q1 = quantize_pair<false>(
+                            __uint_as_float(p1 * c65536), __uint_as_float(p1 & 0xFFFF0000u), inv);
+                        vals[h] = q1 * c65536 + q0;
+                    }
                 }
-                __stcs(vout + st, make_uint4(vals[0], vals[1], vals[2], vals[3]));
-                __stcs(reinterpret_cast<uint32_t*>(Xm + meta_offset(m, 4 * st, K_lp)), nib[i]);
+                __stcs(vout + 32 * i, make_uint4(vals[0], vals[1], vals[2], vals[3]));
+                __stcs(mout + 4096 * i, nib[i]);
             }
         }
     }

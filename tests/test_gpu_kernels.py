@@ -75,12 +75,18 @@ def test_prune_act_2to4_many_rows(q, M, K):
     np.testing.assert_array_equal(host(Xv), Xv_ref)
 
 
-# The single-pass prune kernel (bf16 rows, K % 32 == 0): 1 warp per row with
-# 1, 4 and 8 steps of 32 elements per lane, 2 warps with 7 and 8, 4 warps
-# with 8; K = 96 and 160 leave zero-filled padding steps up to K_lp.
+# The single-pass prune kernel (bf16 rows, chunks of up to 4096 elements per
+# warp).  Chunks that fill whole steps per lane with no padding (the
+# bounds-free form): K = 2048 (2 steps per lane), 4096, 8192 and 16384 (4
+# steps, 1, 2 and 4 warps per row).  The bounds-checked form: K = 96 and 160
+# (zero-filled padding steps up to K_lp), 1024, 2080, 4032 (padding steps in
+# the last step), 6208 and 8320 (2 and 4 warps per row), 8128 (a fifth step
+# for the last warp's padding) and 14336.  K = 32768 takes the two-pass kernel.
 @pytest.mark.parametrize("q", ["int8", "fp8"])
-@pytest.mark.parametrize("M,K", [(300, 96), (257, 160), (2000, 1024), (3000, 4096),
-                                 (1000, 8192), (700, 14336), (600, 16384), (200, 32768)])
+@pytest.mark.parametrize("M,K", [(300, 96), (257, 160), (2000, 1024), (1000, 2048), (1000, 2080),
+                                 (3000, 4096), (400, 4032), (600, 6208), (300, 8128),
+                                 (1000, 8192), (300, 8320), (700, 14336), (600, 16384),
+                                 (200, 32768)])
 def test_prune_act_2to4_register_rows(q, M, K):
     X = synth.gaussian_with_heavy_tails(M, K, seed=K + 1)
     Xv_ref, Xm_ref, s_ref = oracle.prune_act_2to4(X, Q[q])
