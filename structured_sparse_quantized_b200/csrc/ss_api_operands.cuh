@@ -107,7 +107,7 @@ ss_status ss_quant_lift_act(const void* X, ss_in_dtype in_dtype, int64_t M, int6
         st = launch_ex(kern, dim3(grid), dim3(warps * 32), smem, s, 1,                        \
                        static_cast<const T*>(X), M, K, Nh, K_lift, K_lp, q_stride, xq, s_x);  \
     } while (0)
-    // bf16 rows of up to 4096 elements (K % 16 == 0) are read once, into registers
+    // bf16 rows of up to kRegK = 16384 elements (K % 16 == 0) are read once, into registers
     const bool reg_path = in_dtype == SS_IN_BF16 && K % 16 == 0 && K <= ss::kRegK;
     if (reg_path) {
         // registers for the row: 1, 2 or 4 warps per row, each lane holding

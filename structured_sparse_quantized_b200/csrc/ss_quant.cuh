@@ -1,21 +1,31 @@
 // ss_quant.cuh -- memory-bound activation kernels.
 //
-//  quant_lift_warp_kernel  fused per-token absmax, quantisation and activation
-//                          lifting (SlideSparse, 66bd.net: lifting is an index
-//                          map fused into the per-token quant kernel;
-//                          SlideSparse write-up, omica.com.cn, 3.2: one kernel
-//                          computes the absmax, the scale, the clamped
-//                          quantised values, the window remap and the packed
-//                          stores, iterating over output windows).
-//  prune_act_warp_kernel   online 2:4 prune + compress of an activation ("add
-//                          2:4 or drop a precision tier?", paper-daily
-//                          2610.28947, sections 1 and 2.3).
+//  quant_lift_reg_kernel    fused per-token absmax, quantisation and activation
+//                           lifting for bf16 rows of up to 16384 elements: the
+//                           row is read once, into registers (1, 2 or 4 warps
+//                           per row) (SlideSparse, 66bd.net: lifting is an
+//                           index map fused into the per-token quant kernel;
+//                           SlideSparse write-up, omica.com.cn, 3.2: one kernel
+//                           computes the absmax, the scale, the clamped
+//                           quantised values, the window remap and the packed
+//                           stores, iterating over output windows).
+//  quant_lift_warp_kernel   the same for any other row (fp32 rows, longer or
+//                           ragged K): pass 1 streams the row with 16-byte loads
+//                           for its absmax, pass 2 streams it again (from L2)
+//                           and quantises.
+//  prune_act_stream_kernel  online 2:4 prune + compress of bf16 rows for the
+//                           8-bit tiers, single pass: rows stream through shared
+//                           memory, the kept half stays in registers ("add 2:4
+//                           or drop a precision tier?", paper-daily 2610.28947,
+//                           sections 1 and 2.3).
+//  prune_act_warp_kernel    the same for other rows and for the bf16 tier, in
+//                           two passes like quant_lift_warp_kernel.
+//  lift_bf16_kernel         the lift alone, for the bf16 tier (no scale).
 //
-// One warp per token row, no block-wide barrier on the path: pass 1 streams
-// the row with 16-byte loads for its absmax, pass 2 streams it again (from
-// L2) and quantises; outputs leave in 16-byte stores -- four lifted windows
-// (or sixteen identity bytes) per store for the lift, eight 2:4 groups (16
-// value bytes + one 32-bit nibble word) per step for the prune.
+// One warp (or a few) per token row, no block-wide barrier on the path;
+// outputs leave in 16-byte stores -- four lifted windows (or sixteen identity
+// bytes) per store for the lift, eight 2:4 groups (16 value bytes + one 32-bit
+// nibble word) per step for the prune.
 #pragma once
 
 #include "ss_common.cuh"
