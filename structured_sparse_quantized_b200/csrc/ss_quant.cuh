@@ -431,8 +431,8 @@ __global__ void __launch_bounds__(kWarpRowThreads) prune_act_warp_kernel(
 
 // Single-pass online 2:4 prune of bf16 rows (8-bit tiers), streamed through
 // shared memory.  A row is split into kWpr chunks of C = K / kWpr elements
-// (C a multiple of 32, at most kChunkMax); the kWpr warps of a row slot each
-// take one chunk.  Each warp owns kSlots shared-memory slots and keeps the
+// (C a multiple of 32, at most kPruneChunkMax); the kWpr warps of a row slot
+// each take one chunk.  Each warp owns kPruneSlots shared-memory slots and keeps the
 // 1-D bulk copies of its next chunks in flight while it works on the current
 // one, so X is read from HBM once at full overlap:
 //   - select: lane l takes the 32-element steps l, l + 32, ... of the chunk
